@@ -1,0 +1,215 @@
+"""CPU oracle for the DSA / CSA sparse-attention path -- TEST INFRASTRUCTURE.
+
+Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA product never imports it, and
+it imports nothing from the product.  All arithmetic lives in ``oracle.c``
+(plain C, double precision); this module only compiles it with gcc, converts
+arrays and marshals arguments.
+
+Functions and the passages they follow are listed in the header of
+``oracle.c``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_OUT_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_OUT_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FP32, BF16, FP8 = 0, 1, 2
+
+_I32P = ctypes.POINTER(ctypes.c_int32)
+_F32P = ctypes.POINTER(ctypes.c_float)
+_F64P = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into _build/liboracle.so (gcc, -O2, OpenMP)."""
+    os.makedirs(_OUT_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                           "-Wall", "-Wno-unknown-pragmas", _SRC, "-o", tmp, "-lm"])
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            L.oracle_bf16_to_double.restype = ctypes.c_double
+            L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+            L.oracle_fp8_e4m3_to_double.restype = ctypes.c_double
+            L.oracle_fp8_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            L.oracle_double_to_bf16_rne.restype = ctypes.c_uint16
+            L.oracle_double_to_bf16_rne.argtypes = [ctypes.c_double]
+            L.oracle_csa_compress.restype = None
+            L.oracle_csa_compress.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+            L.oracle_index_scores.restype = None
+            L.oracle_index_scores.argtypes = [ctypes.c_void_p, ctypes.c_int, _F32P, ctypes.c_void_p,
+                                              ctypes.c_int, _F32P, _I32P, _I32P, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32P,
+                                              ctypes.c_int, _F64P]
+            L.oracle_topk.restype = None
+            L.oracle_topk.argtypes = [_F64P, ctypes.c_int64, _I32P, ctypes.c_int, ctypes.c_int, _I32P]
+            L.oracle_sparse_mla.restype = None
+            L.oracle_sparse_mla.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, _I32P,
+                                            ctypes.c_int, ctypes.c_int, _I32P, _I32P, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_double, _I32P, ctypes.c_int,
+                                            _F64P, _F64P, _F64P]
+            L.oracle_max_threads.restype = ctypes.c_int
+            L.oracle_max_threads.argtypes = []
+            _lib = L
+    return _lib
+
+
+# ---- array marshalling -------------------------------------------------------
+
+def _host(t) -> np.ndarray:
+    """Contiguous host numpy view of a tensor/array; bf16 -> raw uint16 bits,
+    fp8 -> raw uint8 codes."""
+    if isinstance(t, (list, tuple)):
+        t = np.asarray(t)
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t)
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype in (torch.float8_e4m3fn,):
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
+def _dtype_code(t) -> int:
+    if isinstance(t, np.ndarray):
+        return {np.dtype(np.float32): FP32, np.dtype(np.uint16): BF16, np.dtype(np.uint8): FP8}[t.dtype]
+    return {torch.float32: FP32, torch.bfloat16: BF16, torch.uint8: FP8,
+            torch.float8_e4m3fn: FP8}[t.dtype]
+
+
+def _p(a: np.ndarray, typ):
+    return a.ctypes.data_as(typ)
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(_host(a), dtype=np.int32)
+
+
+def max_threads() -> int:
+    return int(lib().oracle_max_threads())
+
+
+# ---- element formats -----------------------------------------------------------
+
+def bf16_to_double(bits: int) -> float:
+    return float(lib().oracle_bf16_to_double(int(bits) & 0xFFFF))
+
+
+def fp8_e4m3_to_double(code: int) -> float:
+    return float(lib().oracle_fp8_e4m3_to_double(int(code) & 0xFF))
+
+
+def double_to_bf16_bits(x: float) -> int:
+    return int(lib().oracle_double_to_bf16_rne(float(x)))
+
+
+# ---- the path -------------------------------------------------------------------
+
+def csa_compress(src, m: int) -> np.ndarray:
+    """src [B, L, D] (bf16 or fp32) -> [B, L/m, D] of the same storage type
+    (bf16 as raw uint16 bits)."""
+    a = _host(src)
+    B, L, D = a.shape
+    if L % m:
+        raise ValueError("L must be a multiple of m")
+    out = np.empty((B, L // m, D), dtype=a.dtype)
+    lib().oracle_csa_compress(a.ctypes.data, _dtype_code(a), B, L, D, m, out.ctypes.data)
+    return out
+
+
+def index_scores(q_idx, w, k_idx, row_batch, row_pos, k_scale=None, row_ids=None) -> np.ndarray:
+    """Index scores of the requested query rows: float64 [n, L]."""
+    q = _host(q_idx)
+    k = _host(k_idx)
+    wf = np.ascontiguousarray(_host(w), dtype=np.float32)
+    rows, H_I, D_I = q.shape
+    B, L, D_I2 = k.shape
+    assert D_I2 == D_I
+    kd = _dtype_code(k)
+    ks = None
+    if kd == FP8:
+        ks = np.ascontiguousarray(_host(k_scale), dtype=np.float32)
+        assert ks.shape == (B, L)
+    rb, rp = _i32(row_batch), _i32(row_pos)
+    ids = np.arange(rows, dtype=np.int32) if row_ids is None else _i32(row_ids)
+    out = np.empty((len(ids), L), dtype=np.float64)
+    lib().oracle_index_scores(q.ctypes.data, _dtype_code(q), _p(wf, _F32P), k.ctypes.data, kd,
+                              _p(ks, _F32P) if ks is not None else None, _p(rb, _I32P), _p(rp, _I32P),
+                              B, L, H_I, D_I, _p(ids, _I32P), len(ids), _p(out, _F64P))
+    return out
+
+
+def topk(scores, pos, k: int) -> np.ndarray:
+    """scores [n, ld] (any float type; converted exactly to double), pos [n]:
+    last visible key of each row.  Returns int32 [n, k] in rank order, -1 tail."""
+    s = np.ascontiguousarray(_host(scores), dtype=np.float64)
+    n, ld = s.shape
+    p = _i32(pos)
+    assert p.shape == (n,)
+    if np.any(p >= ld):
+        raise ValueError("pos beyond the score row")
+    idx = np.empty((n, k), dtype=np.int32)
+    lib().oracle_topk(_p(s, _F64P), ld, _p(p, _I32P), n, k, _p(idx, _I32P))
+    return idx
+
+
+def sparse_mla(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int,
+               page_table=None, row_ids=None, want_probs: bool = False):
+    """Attention of each requested query row over its selected latent rows.
+
+    q [rows, H, D_K]; kv [B, L, D_K] or paged [pages, page, D_K]; idx
+    [rows, k] key positions (-1 = unused).  Returns (out [n,H,D_V] f64,
+    lse [n,H] f64, probs [n,H,k] f64 or None)."""
+    qa, kva = _host(q), _host(kv)
+    assert _dtype_code(qa) == _dtype_code(kva)
+    rows, H, D_K = qa.shape
+    ia = _i32(idx)
+    k = ia.shape[1]
+    rb = _i32(row_batch)
+    if page_table is not None:
+        pt = _i32(page_table)
+        B, pages_per_seq = pt.shape
+        page = kva.shape[1]
+        assert pages_per_seq * page == ctx
+    else:
+        pt, pages_per_seq, page = None, 0, 0
+        B = kva.shape[0]
+        assert kva.shape[1] == ctx
+    ids = np.arange(rows, dtype=np.int32) if row_ids is None else _i32(row_ids)
+    n = len(ids)
+    out = np.empty((n, H, d_v), dtype=np.float64)
+    lse = np.empty((n, H), dtype=np.float64)
+    probs = np.empty((n, H, k), dtype=np.float64) if want_probs else None
+    lib().oracle_sparse_mla(qa.ctypes.data, kva.ctypes.data, _dtype_code(qa),
+                            _p(pt, _I32P) if pt is not None else None, page, pages_per_seq,
+                            _p(rb, _I32P), _p(ia, _I32P), k, B, ctx, H, D_K, d_v, float(scale),
+                            _p(ids, _I32P), n, _p(out, _F64P), _p(lse, _F64P),
+                            _p(probs, _F64P) if probs is not None else None)
+    return out, lse, probs
