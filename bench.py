@@ -1,0 +1,467 @@
+"""Benchmark of the DSA hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+lightning-indexer scores -> per-query top-k -> sparse MLA over the selected
+latent rows.  Default workload: DSA decode, 32 sequences of 32,768 cached
+tokens, one new query each, top-2048, 128 MLA heads (576/512), bf16.  A
+second line of measurement on the 16,384-token causal prefill workload is
+reported under "prefill" in the same JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched by torchrun, one process per GPU): every rank runs its
+own independent batch (replicas, weak scaling, no collective on the data
+path); the step time is the max over ranks.
+
+Timing: CUDA events on the launching stream around each step; a 256 MB
+buffer is written between steps to flush L2 (outside the events); per-kernel
+times come from events between the kernels of the same steps.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+INDEXER_SRC = "indexer_simt.cu"   # source of the kernel that runs the bf16 indexer
+METRIC = "DSA decode queries/s @32K ctx & prefill tok/s; fraction of HBM/tensor roofline"
+
+
+# ------------------------------------------------------------------ ranks ----
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------ roofline ----
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def indexer_bytes(wl) -> int:
+    """Algorithmic bytes of one indexer launch: every visible key row read
+    once, the queries and weights read once, the visible scores written."""
+    key_b = {"bf16": 2, "fp32": 4, "fp8": 1}[wl.idx_key_dtype]
+    scale_b = 4 if wl.idx_key_dtype == "fp8" else 0
+    q_b = 2 if wl.dtype == "bf16" else 4
+    if wl.mode == "decode":
+        vis = wl.ctx * wl.rows          # one query per cache in these workloads
+        keys = wl.batch * wl.ctx
+    else:
+        vis = wl.rows * (wl.rows + 1) // 2
+        keys = wl.ctx
+    return keys * wl.idx_dim * key_b + keys * scale_b + wl.rows * wl.idx_heads * (wl.idx_dim * q_b + 4) + vis * 4
+
+
+def indexer_flops(wl) -> int:
+    vis = wl.ctx * wl.rows if wl.mode == "decode" else wl.rows * (wl.rows + 1) // 2
+    return 2 * vis * wl.idx_heads * wl.idx_dim
+
+
+def mla_flops(wl) -> int:
+    sel = wl.rows * wl.topk if wl.mode == "decode" else sum(min(t + 1, wl.topk) for t in range(wl.rows))
+    return 2 * sel * wl.heads * (wl.d_qk + wl.d_v)
+
+
+def mla_bytes(wl) -> int:
+    sel = wl.rows * wl.topk if wl.mode == "decode" else sum(min(t + 1, wl.topk) for t in range(wl.rows))
+    e = 2 if wl.dtype == "bf16" else 4
+    return sel * wl.d_qk * e + wl.rows * wl.heads * (wl.d_qk + wl.d_v) * e + wl.rows * wl.topk * 4
+
+
+def profiled_traffic(kernel: str, workload: str, source_file: str):
+    """DRAM bytes per launch from a committed ncu summary, if the summary was
+    taken on the current source of the kernel (same sha256 prefix)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.md")
+    if not os.path.exists(path) or not os.path.exists(source_file):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", txt)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(source_file, "rb").read()).hexdigest()
+    if not cur.startswith(h.group(1)):
+        return None
+    return float(m.group(1))
+
+
+# --------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            p = [x.strip() for x in l.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax = float(p[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ our arm ----
+
+class DecodeStep:
+    """Preallocated buffers and the three library calls of one step."""
+
+    def __init__(self, dsa, wl, inp, device):
+        import torch
+        self.dsa, self.wl, self.inp = dsa, wl, inp
+        self.logits = torch.empty((wl.rows, wl.ctx), dtype=torch.float32, device=device)
+        self.idx = torch.empty((wl.rows, wl.topk), dtype=torch.int32, device=device)
+        self.out = torch.empty((wl.rows, wl.heads, wl.d_v), dtype=inp["q"].dtype, device=device)
+        self.lse = torch.empty((wl.rows, wl.heads), dtype=torch.float32, device=device)
+        n = dsa.topk_workspace_size(wl.rows, wl.ctx, wl.topk)
+        self.topk_ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device) if n else None
+        n = dsa.sparse_mla_workspace_size(wl.rows, wl.topk, wl.heads, wl.d_qk, wl.d_v, inp["q"].dtype)
+        self.mla_ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device) if n else None
+
+    def run(self, events=None):
+        d, wl, i = self.dsa, self.wl, self.inp
+        if events: events[0].record()
+        d.indexer_logits(i["q_idx"], i["w"], i["k_idx"], i["row_batch"], i["row_pos"], k_scale=i.get("k_scale"),
+                         out=self.logits)
+        if events: events[1].record()
+        d.topk(self.logits, i["row_pos"], wl.topk, ctx_len=wl.ctx, out=self.idx, workspace=self.topk_ws)
+        if events: events[2].record()
+        d.sparse_mla(i["q"], i["kv"], self.idx, i["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx,
+                     page_table=i.get("page_table"), out=self.out, lse=self.lse, workspace=self.mla_ws)
+        if events: events[3].record()
+
+
+def time_steps(step, steps, warmup, device, flush):
+    """Warm up, then time `steps` steps with per-step and per-kernel events.
+    Returns (mean step ms, {kernel: mean ms}, launches during the timed steps)."""
+    import torch
+    dsa = step.dsa
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    n0 = dsa.launch_count()
+    for s in range(steps):
+        flush.zero_()                        # L2 flush, outside the step's events
+        step.run(evs[s])
+    torch.cuda.synchronize(device)
+    barrier(device)
+    launches = dsa.launch_count() - n0
+    per = [e[0].elapsed_time(e[3]) for e in evs]
+    kern = {"dsa_indexer_logits": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+            "dsa_topk": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
+            "dsa_sparse_mla": statistics.mean(e[2].elapsed_time(e[3]) for e in evs)}
+    return statistics.mean(per), kern, launches
+
+
+def e2e_decode(dsa, wl, inp, step, steps, device):
+    """Same metric through the public API with host buffers: every step copies
+    the step's new inputs (the queries, and the new token's indexer-key and
+    latent rows appended to each cache) from pinned host memory, runs the
+    path, and reads the attention output and lse back."""
+    import torch
+    g = torch.Generator().manual_seed(1234)
+    h_qidx = inp["q_idx"].cpu().pin_memory()
+    h_w = inp["w"].cpu().pin_memory()
+    h_q = inp["q"].cpu().pin_memory()
+    new_k = (torch.randn((wl.batch, wl.idx_dim), generator=g) / math.sqrt(wl.idx_dim)).to(inp["k_idx"].dtype).pin_memory()
+    new_kv = (torch.randn((wl.batch, wl.d_qk), generator=g) / math.sqrt(wl.d_qk)).to(inp["kv"].dtype).pin_memory()
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h_lse = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_qidx, h_w, h_q, new_k, new_kv))
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * 4
+    last = wl.ctx - 1
+
+    def one():
+        inp["q_idx"].copy_(h_qidx, non_blocking=True)
+        inp["w"].copy_(h_w, non_blocking=True)
+        inp["q"].copy_(h_q, non_blocking=True)
+        inp["k_idx"][:, last].copy_(new_k, non_blocking=True)
+        if "page_table" not in inp:
+            inp["kv"][:, last].copy_(new_kv, non_blocking=True)
+        step.run()
+        h_out.copy_(step.out, non_blocking=True)
+        h_lse.copy_(step.lse, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize(device)
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+def cpu_baseline_decode(wl, inp, budget_s: float = 12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    whole query rows (index scores over all keys, top-k, attention) until the
+    time budget is used.  Returns (queries/s, rows done, threads)."""
+    import numpy as np
+    import oracle
+    import torch
+    done, t_used = 0, 0.0
+    for r in range(wl.rows):
+        b = int(inp["row_batch"][r])
+        q_idx = inp["q_idx"][r:r + 1].cpu()
+        w = inp["w"][r:r + 1].cpu()
+        kb = inp["k_idx"][b:b + 1].cpu()
+        ks = inp["k_scale"][b:b + 1].cpu() if "k_scale" in inp else None
+        rb0 = torch.zeros(1, dtype=torch.int32)
+        rp = inp["row_pos"][r:r + 1].cpu()
+        if "page_table" in inp:
+            pt = inp["page_table"][b:b + 1].cpu()
+            kv = inp["kv"].index_select(0, inp["page_table"][b].long()).cpu()
+            table = torch.arange(pt.shape[1], dtype=torch.int32).view(1, -1)
+        else:
+            kv = inp["kv"][b:b + 1].cpu()
+            table = None
+        q = inp["q"][r:r + 1].cpu()
+        t0 = time.perf_counter()
+        scores = oracle.index_scores(q_idx, w, kb, rb0, rp, k_scale=ks)
+        idx = oracle.topk(scores, rp, wl.topk)
+        oracle.sparse_mla(q, kv, idx, rb0, wl.softmax_scale, wl.d_v, wl.ctx, page_table=table)
+        t_used += time.perf_counter() - t0
+        done += 1
+        if t_used >= budget_s:
+            break
+    return done / t_used, done, oracle.max_threads(), t_used
+
+
+def run_ours(args):
+    import torch
+    rank, world = init_dist("nccl")
+    _, _, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import sparse_attention_logits_b200 as dsa
+    import workloads
+
+    wl = workloads.BY_NAME[args.workload]
+    inp = workloads.generate(wl, device=device, seed=rank)
+    step = DecodeStep(dsa, wl, inp, device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    peaks = measured_peaks()
+
+    with ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
+        ms, kern, launches = time_steps(step, args.steps, args.warmup, device, flush)
+    dsa.get_device_error(device)
+    ms_max = max_over_ranks(ms, device)
+    value = wl.rows * world / (ms_max / 1e3)
+
+    ib = indexer_bytes(wl)
+    ach = ib / (kern["dsa_indexer_logits"] / 1e3) / 1e9
+    traffic = profiled_traffic("dsa_indexer_logits", wl.name, os.path.join(ROOT, "sparse_attention_logits_b200",
+                                                                            "csrc", INDEXER_SRC))
+    roof = {"kernel": "dsa_indexer_logits", "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic,
+            "algorithmic_bytes": ib, "peak_source": peaks["source"]}
+
+    e2e_ms, h2d, d2h = e2e_decode(dsa, wl, inp, step, max(3, args.steps // 2), device)
+    e2e_ms = max_over_ranks(e2e_ms, device)
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "topk": wl.topk,
+                   "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "mla": f"{wl.heads}h {wl.d_qk}/{wl.d_v}",
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (keys 268 MB, latent cache 1.2 GB); 256 MB write between steps"},
+        "roofline": roof,
+        "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+        "gpu_launches": launches,
+        "e2e": {"value": round(wl.rows * world / (e2e_ms / 1e3), 1), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+    }
+    if args.prefill:
+        result["prefill"] = run_prefill(dsa, workloads, device, peaks, args)
+    if world == 1 and rank == 0 and args.cpu_baseline:
+        qps, n, cores, secs = cpu_baseline_decode(wl, inp)
+        result["cpu_baseline"] = {"value": round(qps, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
+                                  "sample": f"{n} whole query rows of {wl.name} ({secs:.1f} s of CPU work)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    _finish()
+
+
+def run_prefill(dsa, workloads, device, peaks, args):
+    import torch
+    rank, world, _ = dist_env()
+    wl = workloads.PREFILL_16K
+    inp = workloads.generate(wl, device=device, seed=100 + rank)
+    step = DecodeStep(dsa, wl, inp, device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    steps = max(2, args.steps // 4)
+    ms, kern, launches = time_steps(step, steps, max(3, args.warmup // 2), device, flush)
+    ms_max = max_over_ranks(ms, device)
+    fl_i, fl_m = indexer_flops(wl), mla_flops(wl)
+    pk = peaks["bf16_tflops"]
+    mla_t = fl_m / (kern["dsa_sparse_mla"] / 1e3) / 1e12
+    idx_t = fl_i / (kern["dsa_indexer_logits"] / 1e3) / 1e12
+    del inp, step, flush
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "value": round(wl.rows * world / (ms_max / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms_max, 3), "steps": steps,
+            "kernels_ms": {k: round(v, 3) for k, v in kern.items()},
+            "roofline": {"kernel": "dsa_sparse_mla", "bound": "tensor", "achieved": round(mla_t, 1), "peak": pk,
+                         "unit": "TFLOP/s", "frac": round(mla_t / pk, 4), "traffic": None,
+                         "algorithmic_flops": fl_m},
+            "indexer_roofline": {"bound": "tensor", "achieved": round(idx_t, 1), "peak": pk, "unit": "TFLOP/s",
+                                 "frac": round(idx_t / pk, 4), "algorithmic_flops": fl_i}}
+
+
+def _finish():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------- reference arm ----
+
+def run_reference(args):
+    """The oracle (plain C, fp64) timed on the host cores on a bounded sample
+    of the same workload: each step = whole query rows until ~budget s."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    import workloads
+    wl = workloads.BY_NAME[args.workload]
+    # inputs drawn on the host: only the rows the sample touches are needed,
+    # but the caches are drawn whole so the sample sees the same workload
+    inp = workloads.generate(wl, device="cpu", seed=0)
+    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline_decode(wl, inp, budget_s=budget / 4)
+    vals, secs, rows_done = [], 0.0, 0
+    for _ in range(args.steps):
+        qps, n, cores, s = cpu_baseline_decode(wl, inp, budget_s=budget)
+        vals.append(qps)
+        secs += s
+        rows_done += n
+    value = rows_done / secs
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "topk": wl.topk,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_done} whole query rows over {args.steps} steps"},
+        "e2e": {"value": round(value, 4), "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dsa_decode_bf16_B32_L32768_k2048")
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

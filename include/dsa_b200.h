@@ -1,0 +1,188 @@
+/*
+ * dsa_b200.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention path.
+ *
+ * The path has four steps, each one entry point:
+ *
+ *   csa_compress        CSA: pool every m consecutive cache rows into one entry
+ *   dsa_indexer_logits  lightning indexer: one score per (query row, cached key)
+ *   dsa_topk            per query row, the k best-scoring visible keys
+ *   dsa_sparse_mla      MQA-mode MLA attention over the selected latent rows
+ *
+ * Conventions shared by every entry point
+ *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
+ *     never allocates or frees device memory; scratch space, where a step
+ *     needs some, is a caller-provided workspace whose size the matching
+ *     *_workspace_size() function returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on that stream and returns; it
+ *     never synchronizes, except dsa_get_device_error().
+ *   - Every call returns a dsa_status_t.  Arguments are validated on the host
+ *     before anything is launched: an invalid argument returns
+ *     DSA_ERR_INVALID_ARG, a shape or type combination for which no kernel is
+ *     built returns DSA_ERR_UNSUPPORTED, and nothing is enqueued in either
+ *     case.  A failed launch returns DSA_ERR_CUDA.  dsa_last_error() gives a
+ *     one-line reason for the most recent failure on the calling thread.
+ *   - Kernels that wait on asynchronous copies bound every wait; a wait that
+ *     runs out records a device error instead of hanging, readable with
+ *     dsa_get_device_error().
+ *   - Tensor layouts are dense, row-major, innermost dimension last, with no
+ *     padding unless a leading dimension argument says otherwise.
+ *   - Nothing is thrown across this interface.
+ *
+ * Sources are cited by page title and section.  "DSA article" below is
+ * "DeepSeek-V3.2稀疏注意力机制原理与TPU适配" (trdm.cn); "V4 CSA summary" is the
+ * xhh.club summary of DeepSeek-V4's compressed sparse attention.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misaligned pointer ... */
+    DSA_ERR_UNSUPPORTED = 2,    /* valid, but no kernel is built for this shape/type */
+    DSA_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+    DSA_ERR_DEVICE_TIMEOUT = 4  /* a kernel gave up a bounded wait (see dsa_get_device_error) */
+} dsa_status_t;
+
+typedef enum {
+    DSA_FP32 = 0,
+    DSA_BF16 = 1,
+    DSA_FP8_E4M3 = 2            /* OCP e4m3 "fn": bias 7, max 448, no infinities */
+} dsa_dtype_t;
+
+/* Library version (major*10000 + minor*100 + patch). */
+DSA_API int dsa_version(void);
+
+/* One-line reason for the most recent non-DSA_OK status on this thread. */
+DSA_API const char* dsa_last_error(void);
+
+/* Number of kernels this library has launched from the calling thread since
+ * the process started (a plain counter, for benchmarks and tests). */
+DSA_API uint64_t dsa_launch_count(void);
+
+/*
+ * csa_compress -- CSA token compression.
+ *   dst[b, i, :] = (1/m) * sum_{r<m} src[b, m*i + r, :]
+ * Every m consecutive rows of a cache become one "super entry" (V4 CSA
+ * summary: 4 tokens -> 1; "解密DeepSeek-V4 ..." section 4.3: average pooling or
+ * a small network -- average pooling is what is built).  Used on both the
+ * MLA latent cache (D = 576) and the indexer key cache (D = 128).
+ *
+ *   src    [batch, len, dim]   of `dtype` (DSA_BF16 or DSA_FP32)
+ *   dst    [batch, len/m, dim] of `dtype`
+ * The sum is formed exactly (double precision) and rounded once to the
+ * storage type, round-to-nearest-even.  len must be a multiple of m;
+ * m in [1, 64]; src and dst must not overlap; both 16-byte aligned.
+ */
+DSA_API dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch, int len, int dim, int m,
+                          void* dst, void* stream);
+
+/*
+ * dsa_indexer_logits -- lightning-indexer scores (DSA article, section 1.3,
+ * 闪电索引器; section 3, Step 2 "compute mqa logits").
+ *   logits[t, s] = sum_{j<n_heads} w[t, j] * ReLU( sum_{d<head_dim} q[t, j, d] * k[b, s, d] )
+ * for every key s <= row_pos[t] of cache b = row_batch[t].  The keys are
+ * shared by all indexer heads (MQA style); w is per query row and head.
+ *
+ *   q          [rows, n_heads, head_dim]  of q_dtype (DSA_FP32 or DSA_BF16)
+ *   w          [rows, n_heads] fp32
+ *   k          [batch, ctx_len, head_dim] of k_dtype (DSA_FP32, DSA_BF16 or DSA_FP8_E4M3)
+ *   k_scale    [batch, ctx_len] fp32, one dequantisation scale per fp8 key row
+ *              (stored key = code * scale); must be NULL unless k is fp8
+ *   row_batch  [rows] int32, cache of each query row, in [0, batch)
+ *   row_pos    [rows] int32, last visible key of each row, in [0, ctx_len):
+ *              prefill rows use their own position (causal), decode rows use
+ *              ctx_len-1
+ *   logits     [rows, ld_logits] fp32, ld_logits >= ctx_len.  Entries
+ *              s <= row_pos[t] are written; entries beyond row_pos[t] are
+ *              left untouched (dsa_topk never reads them).
+ * Accumulation is fp32.  Supported: head_dim in {32, 64, 128}; q and k of the
+ * same floating type, or bf16 q with fp8 k; n_heads <= 128.
+ */
+DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float* w,
+                                const void* k, dsa_dtype_t k_dtype, const float* k_scale,
+                                const int32_t* row_batch, const int32_t* row_pos,
+                                int rows, int batch, int ctx_len, int n_heads, int head_dim,
+                                float* logits, int64_t ld_logits, void* stream);
+
+/* Workspace bytes dsa_topk needs for these sizes (0 = none). */
+DSA_API size_t dsa_topk_workspace_size(int rows, int ctx_len, int k);
+
+/*
+ * dsa_topk -- per-row top-k selection (DSA article, section 1.3: keep only
+ * the key-value entries of the top-k index scores; section 3, Step 3: when
+ * the visible context is no longer than k, every token is kept).
+ *
+ *   logits     [rows, ld] fp32; row t is read at s = 0 .. row_pos[t]
+ *   row_pos    [rows] int32, last visible key of each row
+ *   idx        [rows, k] int32 output: the selected key positions in
+ *              ascending position order, then -1 in every unused slot
+ *              (a row with n = row_pos+1 <= k visible keys selects all n).
+ * Order of scores: larger first; equal scores (with -0.0 == +0.0) go to the
+ * lower position; -inf is the lowest score.  The selection is exact and
+ * deterministic.  NaN scores are not supported.  k in [1, 8192];
+ * ctx_len <= ld.
+ */
+DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, int rows, int ctx_len,
+                      int k, int32_t* idx, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes dsa_sparse_mla needs for these sizes (0 = none). */
+DSA_API size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int d_v, dsa_dtype_t dtype);
+
+/*
+ * dsa_sparse_mla -- attention over the selected latent rows only, MLA in
+ * MQA mode (DSA article, section 1.3 细粒度稀疏注意力; section 1.4: every
+ * latent KV entry is shared by all query heads; section 3, Step 4: decode
+ * reads only the selected KV rows, index_mask drops the rest).
+ *   z_s        = scale * q[t, h, :] . c_s[0:d_qk]           for s in idx[t, :], s >= 0
+ *   out[t,h,:] = sum_s softmax_s(z) * c_s[0:d_v]
+ *   lse[t,h]   = log sum_s exp(z_s)
+ * where c_s is latent row s of cache b = row_batch[t].
+ *
+ *   q          [rows, n_heads, d_qk] of dtype (DSA_BF16 or DSA_FP32)
+ *   kv         contiguous cache [batch, ctx_len, d_qk] when page_table is NULL;
+ *              paged cache [n_pages, page_size, d_qk] otherwise, with
+ *              c_s = kv[page_table[b, s / page_size], s % page_size, :]
+ *   page_table [batch, ctx_len / page_size] int32 physical page ids, or NULL
+ *   row_batch  [rows] int32
+ *   idx        [rows, k] int32 key positions in [0, ctx_len); -1 = unused
+ *              slot (skipped).  Order within a row does not matter.
+ *   out        [rows, n_heads, d_v] of dtype (bf16 rounded to nearest even)
+ *   lse        [rows, n_heads] fp32 natural-log sum of exp of the scaled
+ *              logits; -inf (and out = 0) for a row with no selected key.
+ * Supported: (d_qk, d_v) = (576, 512) bf16 with n_heads = 128, or
+ * d_qk, d_v <= 64 multiples of 32 in fp32 or bf16 with n_heads a multiple of 8.
+ */
+DSA_API dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype,
+                            const int32_t* page_table, int page_size,
+                            const int32_t* row_batch, const int32_t* idx, int k,
+                            int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
+                            float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dsa_get_device_error -- synchronizes `stream`, then reads and clears the
+ * library's device error word on the current device.  Returns DSA_OK when
+ * no kernel recorded an error, DSA_ERR_DEVICE_TIMEOUT when a kernel gave up
+ * a bounded wait, DSA_ERR_CUDA when the synchronization itself failed.
+ */
+DSA_API dsa_status_t dsa_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H */

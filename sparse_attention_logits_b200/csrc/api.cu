@@ -1,0 +1,186 @@
+// extern "C" entry points of libdsa_b200.so: argument validation, kernel
+// selection and the device error word.  Declarations and contracts are in
+// include/dsa_b200.h.
+#include <stdio.h>
+#include <stdarg.h>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+thread_local uint64_t g_launches = 0;
+
+dsa_status_t fail(dsa_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+dsa_status_t cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return DSA_OK;
+    return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// One error word per device; its device address is looked up once per device.
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
+
+dsa_status_t make_launch(void* stream, dsa::Launch* L) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_error);
+        if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(device error word)");
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_status(e, "cudaDeviceGetAttribute");
+        g_num_sms[dev] = sms;
+        g_err_ptr[dev] = (unsigned*)p;
+    }
+    L->stream = (cudaStream_t)stream;
+    L->err = g_err_ptr[dev];
+    L->num_sms = g_num_sms[dev];
+    return DSA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+size_t dtype_size(dsa_dtype_t t) { return t == DSA_FP32 ? 4 : t == DSA_BF16 ? 2 : 1; }
+bool valid_dtype(dsa_dtype_t t) { return t == DSA_FP32 || t == DSA_BF16 || t == DSA_FP8_E4M3; }
+
+}  // namespace
+
+namespace dsa {
+void count_launch(int n) { g_launches += (uint64_t)n; }
+}  // namespace dsa
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+uint64_t dsa_launch_count(void) { return g_launches; }
+
+const char* dsa_last_error(void) { return g_last_error; }
+
+dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch, int len, int dim, int m, void* dst,
+                          void* stream) {
+    if (!src || !dst) return fail(DSA_ERR_INVALID_ARG, "csa_compress: null pointer");
+    if (batch < 0 || len < 0 || dim <= 0 || m < 1 || m > 64)
+        return fail(DSA_ERR_INVALID_ARG, "csa_compress: bad sizes (batch=%d len=%d dim=%d m=%d)", batch, len, dim, m);
+    if (len % m) return fail(DSA_ERR_INVALID_ARG, "csa_compress: len=%d not a multiple of m=%d", len, m);
+    if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "csa_compress: dtype must be bf16 or fp32");
+    if ((dim * dtype_size(dtype)) % 16) return fail(DSA_ERR_UNSUPPORTED, "csa_compress: dim*elem_size must be a multiple of 16 bytes");
+    if (!aligned(src, 16) || !aligned(dst, 16)) return fail(DSA_ERR_INVALID_ARG, "csa_compress: pointers must be 16-byte aligned");
+    const size_t bytes_in = (size_t)batch * len * dim * dtype_size(dtype);
+    const size_t bytes_out = bytes_in / m;
+    const char* s = (const char*)src; const char* d = (const char*)dst;
+    if (bytes_in && s < d + bytes_out && d < s + bytes_in) return fail(DSA_ERR_INVALID_ARG, "csa_compress: src and dst overlap");
+    dsa::Launch L;
+    dsa_status_t st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_csa_compress(L, src, dtype, batch, len, dim, m, dst), "csa_compress launch");
+}
+
+dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float* w, const void* k,
+                                dsa_dtype_t k_dtype, const float* k_scale, const int32_t* row_batch,
+                                const int32_t* row_pos, int rows, int batch, int ctx_len, int n_heads,
+                                int head_dim, float* logits, int64_t ld_logits, void* stream) {
+    if (rows < 0 || batch <= 0 || ctx_len < 0 || n_heads <= 0 || head_dim <= 0)
+        return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: bad sizes");
+    if (rows == 0 || ctx_len == 0) return DSA_OK;
+    if (!q || !w || !k || !row_batch || !row_pos || !logits)
+        return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: null pointer");
+    if (!valid_dtype(q_dtype) || !valid_dtype(k_dtype)) return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: bad dtype");
+    if (ld_logits < ctx_len) return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: ld_logits < ctx_len");
+    if ((k_dtype == DSA_FP8_E4M3) != (k_scale != nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: k_scale must be given exactly when k is fp8");
+    const bool combo_ok = (q_dtype == DSA_FP32 && k_dtype == DSA_FP32) || (q_dtype == DSA_BF16 && k_dtype == DSA_BF16) ||
+                          (q_dtype == DSA_BF16 && k_dtype == DSA_FP8_E4M3);
+    if (!combo_ok) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: unsupported q/k dtype pair");
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128)
+        return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: head_dim must be 32, 64 or 128");
+    if (n_heads > 128) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: n_heads > 128");
+    dsa::Launch L;
+    dsa_status_t st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_indexer_simt(L, q, q_dtype, w, k, k_dtype, k_scale, row_batch, row_pos, rows,
+                                                batch, ctx_len, n_heads, head_dim, logits, ld_logits),
+                       "dsa_indexer_logits launch");
+}
+
+size_t dsa_topk_workspace_size(int rows, int ctx_len, int k) { return dsa::topk_workspace_bytes(rows, ctx_len, k); }
+
+dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, int rows, int ctx_len, int k,
+                      int32_t* idx, void* workspace, size_t workspace_bytes, void* stream) {
+    if (rows < 0 || ctx_len < 0 || k < 1 || k > 8192) return fail(DSA_ERR_INVALID_ARG, "dsa_topk: bad sizes (k must be in [1, 8192])");
+    if (rows == 0) return DSA_OK;
+    if (!logits || !row_pos || !idx) return fail(DSA_ERR_INVALID_ARG, "dsa_topk: null pointer");
+    if (ld < ctx_len) return fail(DSA_ERR_INVALID_ARG, "dsa_topk: ld < ctx_len");
+    const size_t need = dsa::topk_workspace_bytes(rows, ctx_len, k);
+    if (need && (!workspace || workspace_bytes < need))
+        return fail(DSA_ERR_INVALID_ARG, "dsa_topk: workspace of %zu bytes needed", need);
+    dsa::Launch L;
+    dsa_status_t st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_topk(L, logits, ld, row_pos, rows, ctx_len, k, idx, workspace, workspace_bytes),
+                       "dsa_topk launch");
+}
+
+size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int d_v, dsa_dtype_t dtype) {
+    (void)rows; (void)k; (void)n_heads; (void)d_qk; (void)d_v; (void)dtype;
+    return 0;
+}
+
+dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
+                            int page_size, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                            int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    (void)workspace; (void)workspace_bytes;
+    if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 1 || n_heads <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk)
+        return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: bad sizes");
+    if (rows == 0) return DSA_OK;
+    if (!q || !kv || !row_batch || !idx || !out || !lse) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: null pointer");
+    if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "dsa_sparse_mla: dtype must be bf16 or fp32");
+    if (page_table) {
+        if (page_size <= 0 || ctx_len % page_size)
+            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: ctx_len must be a multiple of page_size");
+    }
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: scale must be positive and finite");
+    if (!dsa::mla_simt_supported(d_qk, d_v, n_heads))
+        return fail(DSA_ERR_UNSUPPORTED, "dsa_sparse_mla: no kernel for d_qk=%d d_v=%d n_heads=%d", d_qk, d_v, n_heads);
+    dsa::Launch L;
+    dsa_status_t st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, row_batch, idx, k, rows, batch,
+                                            ctx_len, n_heads, d_qk, d_v, scale, out, lse),
+                       "dsa_sparse_mla launch");
+}
+
+dsa_status_t dsa_get_device_error(void* stream) {
+    dsa::Launch L;
+    dsa_status_t st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(L.stream);
+    if (e != cudaSuccess) return cuda_status(e, "dsa_get_device_error: stream synchronize");
+    unsigned word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof word);
+    if (e != cudaSuccess) return cuda_status(e, "dsa_get_device_error: read");
+    if (word == 0) return DSA_OK;
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_status(e, "dsa_get_device_error: clear");
+    if (word & (dsa::DEV_ERR_TIMEOUT_TMA | dsa::DEV_ERR_TIMEOUT_MMA | dsa::DEV_ERR_TIMEOUT_PEER))
+        return fail(DSA_ERR_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (device error word 0x%x)", word);
+    return fail(DSA_ERR_INVALID_ARG, "a kernel met an out-of-range index and skipped it (device error word 0x%x)", word);
+}
+
+}  // extern "C"

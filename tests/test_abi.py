@@ -1,0 +1,86 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects invalid arguments on the host (no GPU needed, no kernel launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_logits_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = _build.build_library()
+    return ctypes.CDLL(path)
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"DSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"csa_compress", "dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla", "dsa_get_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_only_the_abi_is_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _build.LIB_PATH], capture_output=True, text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    extra = {s for s in syms if not (s.startswith("dsa_") or s == "csa_compress" or s.startswith("_"))}
+    assert not extra, f"unexpected exports: {sorted(extra)[:10]}"
+
+
+def test_version(lib):
+    assert lib.dsa_version() >= 100
+
+
+def _err(lib):
+    lib.dsa_last_error.restype = ctypes.c_char_p
+    return lib.dsa_last_error().decode()
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)      # never dereferenced: validation fails first
+    # top-k with k = 0
+    lib.dsa_topk.argtypes = [vp, ctypes.c_int64, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp,
+                             ctypes.c_size_t, vp]
+    assert lib.dsa_topk(fake, 100, fake, 4, 100, 0, fake, None, 0, None) == 1
+    assert "k must be" in _err(lib)
+    # ld < ctx_len
+    assert lib.dsa_topk(fake, 10, fake, 4, 100, 5, fake, None, 0, None) == 1
+    # compress: len not a multiple of m
+    lib.csa_compress.argtypes = [vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
+    assert lib.csa_compress(fake, 1, 2, 10, 576, 4, vp(0x100000), None) == 1
+    # compress: unsupported dtype (fp8)
+    assert lib.csa_compress(fake, 2, 2, 8, 576, 4, vp(0x100000), None) == 2
+    # compress: overlapping buffers
+    assert lib.csa_compress(vp(0x10000), 1, 1, 8, 64, 4, vp(0x10000 + 64), None) == 1
+    # indexer: fp8 keys without scales
+    lib.dsa_indexer_logits.argtypes = [vp, ctypes.c_int, vp, vp, ctypes.c_int, vp, vp, vp, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, ctypes.c_int64, vp]
+    assert lib.dsa_indexer_logits(fake, 1, fake, fake, 2, None, fake, fake, 4, 4, 128, 64, 128, fake, 128, None) == 1
+    # indexer: unsupported head dim
+    assert lib.dsa_indexer_logits(fake, 1, fake, fake, 1, None, fake, fake, 4, 4, 128, 64, 96, fake, 128, None) == 2
+    # sparse MLA: null output
+    lib.dsa_sparse_mla.argtypes = [vp, vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
+    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, fake, fake, 2048, 4, 4, 4096, 128, 576, 512, 0.04, None,
+                              fake, None, 0, None) == 1
+    # sparse MLA: unbuilt head geometry
+    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, fake, fake, 2048, 4, 4, 4096, 100, 576, 512, 0.04, fake,
+                              fake, None, 0, None) == 2
+    # zero rows is a no-op success without touching the device
+    assert lib.dsa_topk(fake, 100, fake, 0, 100, 5, fake, None, 0, None) == 0
