@@ -112,6 +112,13 @@ dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float*
     dsa::Launch L;
     dsa_status_t st = make_launch(stream, &L);
     if (st != DSA_OK) return st;
+    if (dsa::indexer_tc_supported(q_dtype, k_dtype, n_heads, head_dim)) {
+        if (!aligned(q, 16) || !aligned(k, 16))
+            return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: q and k must be 16-byte aligned");
+        return cuda_status(dsa::launch_indexer_tc(L, q, k_dtype, w, k, k_scale, row_batch, row_pos, rows, batch,
+                                                  ctx_len, logits, ld_logits),
+                           "dsa_indexer_logits (tensor-core) launch");
+    }
     return cuda_status(dsa::launch_indexer_simt(L, q, q_dtype, w, k, k_dtype, k_scale, row_batch, row_pos, rows,
                                                 batch, ctx_len, n_heads, head_dim, logits, ld_logits),
                        "dsa_indexer_logits launch");

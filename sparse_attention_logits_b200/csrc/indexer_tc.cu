@@ -1,0 +1,473 @@
+// Lightning-indexer scores on the 5th-generation tensor cores (tcgen05)
+// ("DeepSeek-V3.2稀疏注意力机制原理与TPU适配", section 1.3 闪电索引器 and section 3
+// Step 2; xhh.club DeepSeek-V4 CSA summary: 64 heads x 128 dims, ReLU-weighted
+// sum):
+//   logits[t, s] = sum_{j<64} w[t, j] * ReLU(q[t, j, :] . k[b, s, :])
+//
+// Per work unit (a group of NQ query rows x a tile of 128 cached keys):
+//   D[128 keys, NQ*64 (query,head)] = K_tile[128 x 128] . Q[NQ*64 x 128]^T
+// one tcgen05.mma chain (M=128, N=NQ*64, K=128) with the fp32 accumulator in
+// TMEM, then an epilogue in which each thread owns one key (one TMEM lane)
+// and reduces its NQ*64 columns to NQ scores: ReLU, times w, sum over heads
+// (times the key's dequantisation scale for fp8 keys).  Scores are written
+// coalesced (32 consecutive keys per warp store).
+//
+// Warp roles (512 threads, one CTA per SM, persistent):
+//   warp 0      TMA producer: key tiles (ring of STAGES), query tiles (x2)
+//   warp 1      MMA issuer (one thread); allocates / frees TMEM
+//   warps 4-7   fp8 only: widen e4m3 key codes to bf16 straight into TMEM
+//               (the MMA then reads its A operand from TMEM, which keeps
+//               shared-memory traffic below the HBM rate)
+//   warps 8-11  epilogue for query columns [0, 128)
+//   warps 12-15 epilogue for query columns [128, 256) (NQ = 4 only)
+//
+// Decode (NQ = 1): units are the flattened (row, key tile) space split into
+// equal contiguous ranges, one per CTA -- the kernel streams the key cache
+// once at HBM rate.  Single-sequence prefill (NQ = 4): CTAs take groups of 4
+// query rows in a zig-zag order (causal work grows with the position) and
+// every visible key tile of each group; fully invisible tiles are never
+// loaded.
+#include "common.cuh"
+#include "launchers.h"
+#include "sm100.cuh"
+
+namespace dsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int KT = 128;      // keys per tile = MMA M
+constexpr int DI = 128;      // indexer head dim = MMA K
+constexpr int HI = 64;       // indexer heads
+constexpr int THREADS = 512;
+
+template <int NQ, bool FP8>
+struct Cfg {
+    static constexpr int N = NQ * HI;
+    static constexpr int STAGES = FP8 ? 8 : (NQ == 1 ? 6 : 3);
+    static constexpr int KBYTES = FP8 ? KT * DI : KT * DI * 2;      // one key tile in shared memory
+    static constexpr int QBYTES = N * DI * 2;                        // one query tile (bf16)
+    static constexpr int ACC_COLS = N;
+    static constexpr int A_COL0 = 2 * ACC_COLS;                     // fp8: bf16 key tiles in TMEM
+    static constexpr int A_COLS = DI / 2;                            // 128 bf16 = 64 columns
+    static constexpr int TMEM_NEED = 2 * ACC_COLS + (FP8 ? 2 * A_COLS : 0);
+    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+    static constexpr int EPI_WARPS = NQ == 1 ? 4 : 8;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * KBYTES + 2 * (size_t)QBYTES + 256;
+    static_assert(TMEM_NEED <= 512, "TMEM budget");
+    static_assert(N % 16 == 0 && N <= 256, "MMA N");
+};
+
+struct Params {
+    const float* w;
+    const float* k_scale;
+    const int32_t* row_batch;
+    const int32_t* row_pos;
+    float* logits;
+    int64_t ld;
+    int rows, batch, ctx;
+    unsigned* err;
+};
+
+struct Unit {
+    int t0;        // first query row of the group
+    int tile;      // key tile index
+    bool first;    // first unit of a query group (load / wait the query tile)
+    bool last;     // last unit of a query group (release the query tile)
+};
+
+__device__ __forceinline__ int last_visible(const Params& p, int t) {
+    int pos = __ldg(p.row_pos + t);
+    return pos < p.ctx - 1 ? pos : p.ctx - 1;     // may be < 0 (nothing visible)
+}
+
+// Deterministic schedule, walked identically by every warp role.
+template <int NQ>
+struct Sched {
+    // flat (NQ == 1)
+    int64_t u, u_end;
+    int tpr, last_t;
+    // zig-zag groups (NQ == 4)
+    int groups, round, g, tile, ntiles;
+
+    __device__ void init(const Params& p) {
+        if (NQ == 1) {
+            tpr = (p.ctx + KT - 1) / KT;
+            const int64_t total = (int64_t)p.rows * tpr;
+            u = total * blockIdx.x / gridDim.x;
+            u_end = total * (blockIdx.x + 1) / gridDim.x;
+            last_t = -1;
+        } else {
+            groups = (p.rows + NQ - 1) / NQ;
+            round = -1;
+            g = -1;
+            tile = ntiles = 0;
+        }
+    }
+
+    __device__ bool next(const Params& p, Unit& out) {
+        if (NQ == 1) {
+            while (u < u_end) {
+                const int t = (int)(u / tpr), j = (int)(u - (int64_t)t * tpr);
+                const int nt = last_visible(p, t) / KT + 1;          // 0 if nothing visible
+                if (last_visible(p, t) < 0 || j >= nt) {             // rest of this row is invisible
+                    u = (int64_t)(t + 1) * tpr;
+                    continue;
+                }
+                out.t0 = t;
+                out.tile = j;
+                out.first = t != last_t;
+                last_t = t;
+                out.last = (j + 1 >= nt) || (u + 1 >= u_end);
+                ++u;
+                return true;
+            }
+            return false;
+        } else {
+            while (true) {
+                if (tile < ntiles) {
+                    out.t0 = g * NQ;
+                    out.tile = tile;
+                    out.first = tile == 0;
+                    out.last = tile + 1 == ntiles;
+                    ++tile;
+                    return true;
+                }
+                ++round;
+                if ((int64_t)round * gridDim.x >= groups) return false;
+                g = (round & 1) ? (round + 1) * (int)gridDim.x - 1 - (int)blockIdx.x
+                                : round * (int)gridDim.x + (int)blockIdx.x;
+                if (g >= groups) { ntiles = 0; tile = 0; continue; }
+                int mp = -1;
+                for (int r = 0; r < NQ; ++r)
+                    if (g * NQ + r < p.rows) mp = max(mp, last_visible(p, g * NQ + r));
+                ntiles = mp < 0 ? 0 : mp / KT + 1;
+                tile = 0;
+            }
+        }
+    }
+};
+
+// e4m3 pair (low byte = first element) -> bf16 pair, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
+    const float lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    const float hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+}  // namespace
+
+template <int NQ, bool FP8>
+__global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                                                                const __grid_constant__ CUtensorMap tmap_q,
+                                                                const Params p) {
+    using C = Cfg<NQ, FP8>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* kbuf = smem;                                            // [STAGES][KBYTES]
+    uint8_t* qbuf = kbuf + (size_t)C::STAGES * C::KBYTES;            // [2][QBYTES]
+    uint64_t* bars = (uint64_t*)(qbuf + 2 * (size_t)C::QBYTES);
+    uint64_t* kfull = bars;                       // [STAGES]
+    uint64_t* kempty = kfull + C::STAGES;         // [STAGES]
+    uint64_t* qfull = kempty + C::STAGES;         // [2]
+    uint64_t* qempty = qfull + 2;                 // [2]
+    uint64_t* accfull = qempty + 2;               // [2]
+    uint64_t* accempty = accfull + 2;             // [2]
+    uint64_t* afull = accempty + 2;               // [2] (fp8)
+    uint64_t* aempty = afull + 2;                 // [2] (fp8)
+    uint32_t* tmem_slot = (uint32_t*)(aempty + 2);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&kfull[i], 1);
+            mbar_init(&kempty[i], FP8 ? 4 : 1);       // fp8: the 4 converter warps free the stage
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], 1);
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], C::EPI_WARPS);
+            mbar_init(&afull[i], 4);
+            mbar_init(&aempty[i], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    Sched<NQ> sch;
+    Unit un;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        if (elect_one()) {
+            sch.init(p);
+            const uint64_t pol_stream = l2_policy_evict_first();
+            int i = 0, qe = -1;
+            while (sch.next(p, un)) {
+                if (un.first) {
+                    ++qe;
+                    const int qb = qe & 1;
+                    if (!mbar_wait(&qempty[qb], ((qe >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+                    mbar_arrive_expect_tx(&qfull[qb], C::QBYTES);
+                    uint8_t* qdst = qbuf + (size_t)qb * C::QBYTES;
+                    tma_load_2d(qdst, &tmap_q, 0, un.t0 * HI, &qfull[qb]);
+                    tma_load_2d(qdst + C::N * 128, &tmap_q, 64, un.t0 * HI, &qfull[qb]);
+                }
+                const int st = i % C::STAGES;
+                if (!mbar_wait(&kempty[st], ((i / C::STAGES) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+                mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
+                const int b = __ldg(p.row_batch + un.t0);
+                const int row = b * p.ctx + un.tile * KT;
+                uint8_t* kdst = kbuf + (size_t)st * C::KBYTES;
+                if (NQ == 1) {       // decode: every key is read once -> stream it past L2
+                    tma_load_2d_hint(kdst, &tmap_k, 0, row, &kfull[st], pol_stream);
+                    if (!FP8) tma_load_2d_hint(kdst + KT * 128, &tmap_k, 64, row, &kfull[st], pol_stream);
+                } else {             // prefill: every key tile is re-read by later query groups
+                    tma_load_2d(kdst, &tmap_k, 0, row, &kfull[st]);
+                    if (!FP8) tma_load_2d(kdst + KT * 128, &tmap_k, 64, row, &kfull[st]);
+                }
+                ++i;
+            }
+            if (*abort_flag) {
+                // let the copies already issued land before the CTA exits
+                for (int j = (i > C::STAGES ? i - C::STAGES : 0); j < i; ++j)
+                    mbar_wait(&kfull[j % C::STAGES], (j / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ----
+        if (elect_one()) {
+            sch.init(p);
+            constexpr uint32_t idesc = idesc_bf16_f32(KT, C::N, 0, 0);
+            const uint32_t kbase = smem_u32(kbuf), qbase = smem_u32(qbuf);
+            int i = 0, qe = -1;
+            bool ok = true;
+            while (ok && sch.next(p, un)) {
+                if (un.first) {
+                    ++qe;
+                    ok = mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                    if (!ok) break;
+                }
+                const int st = i % C::STAGES, acc = i & 1;
+                if (FP8) {
+                    ok = mbar_wait(&afull[acc], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                } else {
+                    ok = mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                }
+                if (!ok) break;
+                ok = mbar_wait(&accempty[acc], ((i >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d = tmem + acc * C::ACC_COLS;
+                const uint32_t qaddr = qbase + (uint32_t)((qe & 1) * C::QBYTES);
+#pragma unroll
+                for (int kk = 0; kk < DI / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)((kk >> 2) * (C::N * 128) + (kk & 3) * 32);
+                    const uint64_t bdesc = desc_sw128(qaddr + koff, 1024);
+                    if (FP8) {
+                        mma_ts(d, tmem + C::A_COL0 + acc * C::A_COLS + kk * 8, bdesc, idesc, kk > 0);
+                    } else {
+                        const uint32_t aoff = (uint32_t)(st * C::KBYTES + (kk >> 2) * (KT * 128) + (kk & 3) * 32);
+                        mma_ss(d, desc_sw128(kbase + aoff, 1024), bdesc, idesc, kk > 0);
+                    }
+                }
+                if (FP8) mma_commit(&aempty[acc]);
+                else mma_commit(&kempty[st]);
+                mma_commit(&accfull[acc]);
+                if (un.last) mma_commit(&qempty[qe & 1]);
+                ++i;
+            }
+        }
+    } else if (FP8 && warp >= 4 && warp < 8) {
+        // ------------------------- fp8 -> bf16 key widening into TMEM ----
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;                  // key row of the tile = TMEM lane
+        sch.init(p);
+        int i = 0;
+        while (sch.next(p, un)) {
+            const int st = i % C::STAGES, ab = i & 1;
+            if (!mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
+            if (!mbar_wait(&aempty[ab], ((i >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+            tc_fence_after();
+            const uint8_t* src = kbuf + (size_t)st * C::KBYTES + r * 128;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + ab * C::A_COLS;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t words[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int c = half * 4 + c4;                         // 16-byte chunk of the row
+                    const uint4 x = *(const uint4*)(src + ((c ^ (r & 7)) << 4));
+                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        words[c4 * 8 + 2 * e] = e4m3x2_to_bf16x2((uint16_t)(xs[e] & 0xFFFFu));
+                        words[c4 * 8 + 2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(xs[e] >> 16));
+                    }
+                }
+                uint32_t lo[16], hi[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) { lo[m] = words[m]; hi[m] = words[16 + m]; }
+                tmem_st16(taddr + half * 32, lo);
+                tmem_st16(taddr + half * 32 + 16, hi);
+            }
+            tmem_st_wait();
+            __syncwarp();
+            tc_fence_before();
+            if (lane == 0) {
+                mbar_arrive(&kempty[st]);
+                mbar_arrive(&afull[ab]);
+            }
+            ++i;
+        }
+    } else if (warp >= 8 && warp < 8 + C::EPI_WARPS) {
+        // --------------------------------------------------- epilogue ----
+        const int quarter = warp & 3;
+        const int col_half = (warp - 8) >> 2;              // which 128 query columns (NQ = 4)
+        sch.init(p);
+        int i = 0;
+        while (sch.next(p, un)) {
+            const int acc = i & 1;
+            if (!mbar_wait(&accfull[acc], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+            tc_fence_after();
+            const int key = un.tile * KT + quarter * 32 + lane;
+            const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * C::ACC_COLS;
+            constexpr int QPW = NQ == 1 ? 1 : 2;           // query rows per epilogue warp
+            float score[QPW];
+#pragma unroll
+            for (int qq = 0; qq < QPW; ++qq) {
+                const int qi = col_half * 2 + qq;          // query within the group
+                float v0[32], v1[32];
+                tmem_ld32(tbase + qi * HI, v0);
+                tmem_ld32(tbase + qi * HI + 32, v1);
+                tmem_ld_wait();
+                const int t = min(un.t0 + qi, p.rows - 1);
+                const float* wr = p.w + (int64_t)t * HI;
+                float s = 0.f;
+#pragma unroll
+                for (int h = 0; h < 32; ++h) s = fmaf(__ldg(wr + h), fmaxf(v0[h], 0.f), s);
+#pragma unroll
+                for (int h = 0; h < 32; ++h) s = fmaf(__ldg(wr + 32 + h), fmaxf(v1[h], 0.f), s);
+                score[qq] = s;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            const int b = __ldg(p.row_batch + un.t0);
+            const bool b_ok = b >= 0 && b < p.batch;
+            if (!b_ok && lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
+            float ks = 1.f;
+            if (FP8 && b_ok && key < p.ctx) ks = __ldg(p.k_scale + (int64_t)b * p.ctx + key);
+#pragma unroll
+            for (int qq = 0; qq < QPW; ++qq) {
+                const int t = un.t0 + col_half * 2 + qq;
+                if (b_ok && t < p.rows && key <= last_visible(p, t))
+                    p.logits[(int64_t)t * p.ld + key] = FP8 ? score[qq] * ks : score[qq];
+            }
+            ++i;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------ host --
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = (EncodeTiledFn)p;
+    }
+    return fn;
+}
+
+// 2-D row-major tensor [rows, cols] with 128-byte-swizzled boxes.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+              uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NQ, bool FP8>
+cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Params& p) {
+    using C = Cfg<NQ, FP8>;
+    CUtensorMap mk, mq;
+    const uint64_t krows = (uint64_t)p.batch * p.ctx;
+    bool ok = FP8 ? make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
+                  : make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, DI, krows, 64, KT);
+    ok = ok && make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DI, (uint64_t)p.rows * HI, 64, NQ * HI);
+    if (!ok) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<NQ, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    int64_t units;
+    if (NQ == 1) units = (int64_t)p.rows * ((p.ctx + KT - 1) / KT);
+    else units = (p.rows + NQ - 1) / NQ;
+    const int grid = (int)(units < L.num_sms ? units : L.num_sms);
+    indexer_tc_kernel<NQ, FP8><<<grid, THREADS, C::SMEM, L.stream>>>(mk, mq, p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool indexer_tc_supported(dsa_dtype_t q_dtype, dsa_dtype_t k_dtype, int n_heads, int head_dim) {
+    return q_dtype == DSA_BF16 && (k_dtype == DSA_BF16 || k_dtype == DSA_FP8_E4M3) && n_heads == HI &&
+           head_dim == DI;
+}
+
+cudaError_t launch_indexer_tc(const Launch& L, const void* q, dsa_dtype_t k_dtype, const float* w, const void* k,
+                              const float* k_scale, const int32_t* row_batch, const int32_t* row_pos, int rows,
+                              int batch, int ctx_len, float* logits, int64_t ld) {
+    if (rows == 0 || ctx_len == 0) return cudaSuccess;
+    Params p{w, k_scale, row_batch, row_pos, logits, ld, rows, batch, ctx_len, L.err};
+    if (k_dtype == DSA_FP8_E4M3) return launch_cfg<1, true>(L, q, k, p);
+    // Groups of 4 query rows share a key tile only when every row reads the
+    // same cache (one sequence): then the MMA N grows to 256 and each key
+    // tile is reused for 4 queries.
+    if (batch == 1 && rows >= 4 * L.num_sms) return launch_cfg<4, false>(L, q, k, p);
+    return launch_cfg<1, false>(L, q, k, p);
+}
+
+}  // namespace dsa

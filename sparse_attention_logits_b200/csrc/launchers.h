@@ -14,6 +14,11 @@ cudaError_t launch_indexer_simt(const Launch& L, const void* q, dsa_dtype_t q_dt
                                 const int32_t* row_pos, int rows, int batch, int ctx_len, int n_heads,
                                 int head_dim, float* logits, int64_t ld);
 
+bool indexer_tc_supported(dsa_dtype_t q_dtype, dsa_dtype_t k_dtype, int n_heads, int head_dim);
+cudaError_t launch_indexer_tc(const Launch& L, const void* q, dsa_dtype_t k_dtype, const float* w, const void* k,
+                              const float* k_scale, const int32_t* row_batch, const int32_t* row_pos, int rows,
+                              int batch, int ctx_len, float* logits, int64_t ld);
+
 cudaError_t launch_topk(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows,
                         int ctx_len, int k, int32_t* idx, void* workspace, size_t ws_bytes);
 size_t topk_workspace_bytes(int rows, int ctx_len, int k);

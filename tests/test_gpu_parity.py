@@ -53,9 +53,11 @@ def test_compress_bit_exact(cuda_device, dtype, B, L, D, m):
 @pytest.mark.parametrize("wl", [
     workloads.TINY_PREFILL_FP32,
     workloads.DECODE_32K.with_(batch=3, rows=3, ctx=1000),              # ragged tail
-    workloads.PREFILL_16K.with_(ctx=300, rows=300),                     # causal, ragged
+    workloads.PREFILL_16K.with_(ctx=300, rows=300),                     # causal, ragged, 1 query per tile
+    workloads.PREFILL_16K.with_(ctx=1001, rows=1001),                   # causal, 4 queries per tile, ragged
     workloads.DECODE_128K_FP8_PAGED.with_(batch=2, rows=2, ctx=4096 + 64),
-], ids=lambda w: w.name)
+    workloads.DECODE_128K_FP8_PAGED.with_(batch=5, rows=5, ctx=777),    # fp8, ragged tail
+], ids=lambda w: f"{w.name}-ctx{w.ctx}")
 def test_indexer_matches_oracle(cuda_device, wl):
     inp = workloads.generate(wl, parts=("indexer",))
     dv = _cuda(inp, cuda_device)
@@ -136,8 +138,8 @@ def test_sparse_mla_on_given_indices(cuda_device, wl, pad):
 @pytest.mark.parametrize("wl", [
     workloads.TINY_PREFILL_FP32,
     workloads.DECODE_32K.with_(batch=4, rows=4, ctx=5000),
-    workloads.PREFILL_16K.with_(ctx=2300, rows=2300, topk=256),
-], ids=lambda w: w.name)
+    workloads.PREFILL_16K.with_(ctx=1200, rows=1200, topk=256),
+], ids=lambda w: f"{w.name}-ctx{w.ctx}")
 def test_chain_matches_oracle(cuda_device, wl):
     inp = workloads.generate(wl)
     dv = _cuda(inp, cuda_device)
