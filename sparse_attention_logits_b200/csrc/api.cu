@@ -143,15 +143,17 @@ dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, i
 }
 
 size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int d_v, dsa_dtype_t dtype) {
-    (void)rows; (void)k; (void)n_heads; (void)d_qk; (void)d_v; (void)dtype;
-    return 0;
+    if (rows <= 0 || k <= 0 || !dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v)) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 1;     // no device: size for the smallest GPU (most splits)
+    return dsa::mla_tc_workspace_bytes(rows, k, sms);
 }
 
 dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
                             int page_size, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
                             int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream) {
-    (void)workspace; (void)workspace_bytes;
     if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 1 || n_heads <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk)
         return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: bad sizes");
     if (rows == 0) return DSA_OK;
@@ -162,11 +164,22 @@ dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, co
             return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: ctx_len must be a multiple of page_size");
     }
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: scale must be positive and finite");
-    if (!dsa::mla_simt_supported(d_qk, d_v, n_heads))
+    const bool tc = dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v);
+    if (!tc && !dsa::mla_simt_supported(d_qk, d_v, n_heads))
         return fail(DSA_ERR_UNSUPPORTED, "dsa_sparse_mla: no kernel for d_qk=%d d_v=%d n_heads=%d", d_qk, d_v, n_heads);
     dsa::Launch L;
     dsa_status_t st = make_launch(stream, &L);
     if (st != DSA_OK) return st;
+    if (tc) {
+        if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16))
+            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: q, kv and out must be 16-byte aligned");
+        const size_t need = dsa::mla_tc_workspace_bytes(rows, k, L.num_sms);
+        if (need && (!workspace || workspace_bytes < need))
+            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: workspace of %zu bytes needed", need);
+        return cuda_status(dsa::launch_mla_tc(L, q, kv, page_table, page_size, row_batch, idx, k, rows, batch,
+                                              ctx_len, scale, out, lse, workspace, workspace_bytes),
+                           "dsa_sparse_mla (tensor-core) launch");
+    }
     return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, row_batch, idx, k, rows, batch,
                                             ctx_len, n_heads, d_qk, d_v, scale, out, lse),
                        "dsa_sparse_mla launch");

@@ -1,0 +1,560 @@
+// Sparse MLA (MQA mode) on the 5th-generation tensor cores
+// ("DeepSeek-V3.2稀疏注意力机制原理与TPU适配", sections 1.3 细粒度稀疏注意力 and 1.4,
+// section 3 Step 4): for every query row t and each of its 128 heads,
+// attention over the selected latent rows only; one 576-d latent row is
+// shared by all heads (512 latent + 64 rope dims); the value is its first
+// 512 dims.
+//
+// Why a 2-CTA cluster: the output accumulator of one query row is
+// 128 heads x 512 dims fp32 = 256 KB, exactly the tensor memory of one SM.
+// So the work of a (query row, key split) is split by role across the two
+// SMs of a cluster:
+//
+//   score CTA (rank 0)  Q [128 x 576] lives in TMEM (A operand of the MMA).
+//                       Per chunk of 64 selected keys: gather the 576-d rows
+//                       into 128-B-swizzled shared memory (cp.async), S = Q K^T
+//                       (tcgen05, M=128 heads, N=64 keys, K=576) into one of
+//                       two TMEM buffers, online softmax in base 2 with lazy
+//                       rescaling (the running max moves only when a score
+//                       exceeds it by more than 2^8), P rounded to bf16 and
+//                       bulk-copied with its per-head rescale factors into the
+//                       value CTA's shared memory (DSMEM).
+//   value CTA (rank 1)  gathers the first 512 dims of the same rows (the MMA
+//                       reads them as an MN-major B operand), rescales O only
+//                       for chunks whose max moved, accumulates
+//                       O += P V (M=128, N=2x256, K=64) in its 512 TMEM
+//                       columns, and at the end writes O / l and
+//                       lse = ln(sum exp) -- or, when the key list is split
+//                       over several clusters, normalised fp32 partials that
+//                       dsa_mla_combine merges.
+//
+// Warps (both CTAs): 0-3 gather producers, 4-7 softmax (score CTA) or
+// rescale + epilogue (value CTA), one thread per head / TMEM lane, 8 MMA
+// issuer and TMEM owner.  Every wait is bounded; the two CTAs only exchange
+// data through bulk copies and mbarrier arrivals that the receiver waits on.
+#include "common.cuh"
+#include "launchers.h"
+#include "sm100.cuh"
+
+namespace dsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int H = 128;              // query heads = MMA M
+constexpr int DK = 576;             // latent + rope
+constexpr int DV = 512;             // value dims
+constexpr int NK = 64;              // keys per chunk
+constexpr int THREADS = 288;        // 9 warps
+constexpr int KSTAGE = NK * DK * 2; // 73728 B
+constexpr int VSTAGE = NK * DV * 2; // 65536 B
+constexpr int STAGES = 2;
+constexpr int REGION = (STAGES * KSTAGE > STAGES * VSTAGE) ? STAGES * KSTAGE : STAGES * VSTAGE;
+constexpr int PBYTES = H * NK * 2;  // 16384: P [128 heads x 64 keys] bf16
+constexpr int ABYTES = H * 4;       // rescale factor per head
+constexpr int SBYTES = 2 * H * 4;   // final running max and sum per head
+constexpr int S_COL = 320;          // score CTA: Q in TMEM columns [0, 288), S buffers at 320, 384
+constexpr int TMEM_COLS = 512;
+constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between rescales)
+constexpr float LN2 = 0.6931471805599453f;
+
+struct Bars {                       // same offset in both CTAs of a cluster
+    uint64_t kfull[2], kempty[2], sfull[2], sempty[2], pready[2], pempty[2], qready, statready, statack;
+    uint64_t vfull[2], vempty[2], pfull[2], ready[2], odone, statfull;
+    uint32_t tmem;
+    int abort;
+};
+
+struct MlaParams {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* kv;
+    const int32_t* page_table;
+    const int32_t* row_batch;
+    const int32_t* idx;
+    __nv_bfloat16* out;
+    float* lse;
+    float* part_o;                  // [rows, splits, H, DV] when splits > 1
+    float* part_lse;                // [rows, splits, H]
+    unsigned* err;
+    int page_size, pages_per_seq;
+    int k, rows, batch, ctx, splits, per_split;
+    float scale_log2;
+};
+
+struct Work {
+    int t, split, slot0, slot_end, nchunks, b;
+    bool b_ok;
+};
+
+__device__ __forceinline__ Work work_of(const MlaParams& p) {
+    Work w;
+    const int item = blockIdx.x >> 1;
+    w.t = item / p.splits;
+    w.split = item - w.t * p.splits;
+    w.slot0 = w.split * p.per_split;
+    w.slot_end = min(p.k, w.slot0 + p.per_split);
+    w.nchunks = (w.slot_end - w.slot0 + NK - 1) / NK;
+    w.b = __ldg(p.row_batch + w.t);
+    w.b_ok = w.b >= 0 && w.b < p.batch;
+    return w;
+}
+
+// Cache row of key position s (or -1 if the slot is unused / invalid).
+__device__ __forceinline__ int64_t key_row(const MlaParams& p, const Work& w, int slot) {
+    if (!w.b_ok || slot >= w.slot_end) return -1;
+    const int s = __ldg(p.idx + (int64_t)w.t * p.k + slot);
+    if (s < 0) return -1;
+    if (s >= p.ctx) {
+        record_error(p.err, DEV_ERR_BAD_INDEX);
+        return -1;
+    }
+    if (p.page_table) {
+        const int pg = __ldg(p.page_table + (int64_t)w.b * p.pages_per_seq + s / p.page_size);
+        return (int64_t)pg * p.page_size + s % p.page_size;
+    }
+    return (int64_t)w.b * p.ctx + s;
+}
+
+// Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
+    uint8_t* pbuf = gbuf + REGION;                          // [2][PBYTES]
+    float* abuf = (float*)(pbuf + 2 * PBYTES);              // [2][H]
+    float* sbuf = abuf + 2 * H;                             // [2*H]: running max, running sum
+    Bars* bars = (Bars*)(sbuf + 2 * H);
+    volatile int* abort_flag = &bars->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const Work w = work_of(p);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->kfull[i], 128);
+            mbar_init(&bars->kempty[i], 1);
+            mbar_init(&bars->sfull[i], 1);
+            mbar_init(&bars->sempty[i], 4);
+            mbar_init(&bars->pready[i], 4);
+            mbar_init(&bars->pempty[i], 1);
+            mbar_init(&bars->vfull[i], 128);
+            mbar_init(&bars->vempty[i], 1);
+            mbar_init(&bars->pfull[i], 1);
+            mbar_init(&bars->ready[i], 4);
+        }
+        mbar_init(&bars->qready, 4);
+        mbar_init(&bars->statready, 4);
+        mbar_init(&bars->statack, 4);
+        mbar_init(&bars->odone, 1);
+        mbar_init(&bars->statfull, 1);
+        bars->abort = 0;
+        if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
+        if (rank == 1) {
+            // arm the first phase of each P slot and the final-statistics slot
+            mbar_arrive_expect_tx(&bars->pfull[0], PBYTES + ABYTES);
+            if (w.nchunks > 1) mbar_arrive_expect_tx(&bars->pfull[1], PBYTES + ABYTES);
+            mbar_arrive_expect_tx(&bars->statfull, SBYTES);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(&bars->tmem, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    cluster_sync_all();                 // both CTAs' barriers exist before any remote traffic
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem;
+    const uint32_t peer = rank ^ 1u;
+
+    if (warp < 4) {
+        // ------------------------------------------------ gather producers ----
+        const int tid = threadIdx.x;
+        const int row_chunks = rank == 0 ? DK / 8 : DV / 8;    // 16-byte chunks per gathered row
+        const int stage_bytes = rank == 0 ? KSTAGE : VSTAGE;
+        uint64_t* full = rank == 0 ? bars->kfull : bars->vfull;
+        uint64_t* empty = rank == 0 ? bars->kempty : bars->vempty;
+        for (int c = 0; c < w.nchunks; ++c) {
+            const int st = c & 1;
+            if (!mbar_wait(&empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+            uint8_t* base = gbuf + (size_t)st * stage_bytes;
+            int cur_r = -1;
+            int64_t row = -1;
+            for (int i = tid; i < NK * row_chunks; i += 128) {
+                const int r = i / row_chunks, ci = i - r * row_chunks;
+                if (r != cur_r) {
+                    cur_r = r;
+                    row = key_row(p, w, w.slot0 + c * NK + r);
+                }
+                const __nv_bfloat16* src = row >= 0 ? p.kv + row * DK + ci * 8 : p.kv;
+                cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(&full[st]);
+        }
+    } else if (warp < 8 && rank == 0) {
+        // ------------------------------------- score CTA: Q load + softmax ----
+        const int h = (warp - 4) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        {   // Q row of head h -> TMEM lane h, columns [0, 288) (bf16 pairs)
+            const uint4* qrow = (const uint4*)(p.q + ((int64_t)w.t * H + h) * DK);
+#pragma unroll 1
+            for (int m = 0; m < DK / 32; ++m) {
+                uint32_t words[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 x = __ldg(qrow + m * 4 + v);
+                    words[4 * v] = x.x; words[4 * v + 1] = x.y; words[4 * v + 2] = x.z; words[4 * v + 3] = x.w;
+                }
+                tmem_st16(tmem + lane_base + m * 16, words);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->qready);
+        }
+        float m_run = -INFINITY, l_run = 0.f;
+        const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
+        const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
+        bool ok = true;
+        for (int c = 0; c < w.nchunks && ok; ++c) {
+            const int sb = c & 1;
+            // which of the 64 keys of this chunk are real
+            const bool va = key_row(p, w, w.slot0 + c * NK + lane) >= 0;
+            const bool vb = key_row(p, w, w.slot0 + c * NK + 32 + lane) >= 0;
+            const uint32_t mlo = __ballot_sync(0xffffffffu, va), mhi = __ballot_sync(0xffffffffu, vb);
+            ok = mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            float s0[32], s1[32];
+            tmem_ld32(tmem + lane_base + S_COL + sb * NK, s0);
+            tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32, s1);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+            float mc = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                s0[j] = ((mlo >> j) & 1u) ? s0[j] * p.scale_log2 : -INFINITY;
+                s1[j] = ((mhi >> j) & 1u) ? s1[j] * p.scale_log2 : -INFINITY;
+                mc = fmaxf(mc, fmaxf(s0[j], s1[j]));
+            }
+            float alpha = 1.f;
+            if (mc > -INFINITY) {
+                if (m_run == -INFINITY) {
+                    m_run = mc;
+                } else if (mc > m_run + RESCALE_LOG2) {
+                    alpha = exp2f(m_run - mc);
+                    l_run *= alpha;
+                    m_run = mc;
+                }
+            }
+            uint32_t pk[32];
+            float lsum = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float a0 = s0[2 * j] == -INFINITY ? 0.f : exp2f(s0[2 * j] - m_run);
+                const float a1 = s0[2 * j + 1] == -INFINITY ? 0.f : exp2f(s0[2 * j + 1] - m_run);
+                const float b0 = s1[2 * j] == -INFINITY ? 0.f : exp2f(s1[2 * j] - m_run);
+                const float b1 = s1[2 * j + 1] == -INFINITY ? 0.f : exp2f(s1[2 * j + 1] - m_run);
+                const __nv_bfloat162 pa = __floats2bfloat162_rn(a0, a1);
+                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(b0, b1);
+                lsum += __low2float(pa) + __high2float(pa) + __low2float(pb2) + __high2float(pb2);
+                pk[j] = *(const uint32_t*)&pa;
+                pk[16 + j] = *(const uint32_t*)&pb2;
+            }
+            l_run += lsum;
+            const int pb = c & 1;
+            ok = mbar_wait_cluster(&bars->pempty[pb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (!ok) break;
+            uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *(uint4*)(prow + sw128(h & 7, j)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            abuf[pb * H + h] = alpha;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->pready[pb]);
+            if (warp == 4 && lane == 0) {
+                ok = mbar_wait(&bars->pready[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                if (ok) {
+                    const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
+                    bulk_copy_s2cluster(peer_pbuf + pb * PBYTES, pbuf + pb * PBYTES, PBYTES, rbar);
+                    bulk_copy_s2cluster(peer_abuf + pb * ABYTES, abuf + pb * H, ABYTES, rbar);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+        }
+        // final statistics -> value CTA
+        sbuf[h] = m_run;
+        sbuf[H + h] = l_run;
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->statready);
+        if (warp == 4 && lane == 0 && !*abort_flag) {
+            if (mbar_wait(&bars->statready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag))
+                bulk_copy_s2cluster(mapa_shared(smem_u32(sbuf), peer), sbuf, SBYTES,
+                                    mapa_shared(smem_u32(&bars->statfull), peer));
+        }
+        // stay alive until the value CTA has read the statistics and its last
+        // MMA commits (which arrive on our P-slot barriers) have landed
+        mbar_wait_cluster(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+        for (int c = max(0, w.nchunks - 2); c < w.nchunks; ++c)
+            mbar_wait_cluster(&bars->pempty[c & 1], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+    } else if (warp < 8) {
+        // ------------------------- value CTA: rescale of O, then epilogue ----
+        const int h = (warp - 4) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        bool ok = true;
+        for (int c = 0; c < w.nchunks && ok; ++c) {
+            const int pb = c & 1;
+            ok = mbar_wait_cluster(&bars->pfull[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (!ok) break;
+            if (warp == 4 && lane == 0 && c + 2 < w.nchunks)
+                mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
+            const float alpha = abuf[pb * H + h];
+            if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                ok = mbar_wait(&bars->odone, (c - 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int j = 0; j < DV / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + j * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] *= alpha;
+                    tmem_st32(tmem + lane_base + j * 32, v);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->ready[pb]);
+        }
+        if (ok) ok = mbar_wait(&bars->odone, (w.nchunks - 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+        if (ok) ok = mbar_wait_cluster(&bars->statfull, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+        float m = -INFINITY, l = 0.f;
+        if (ok) {
+            m = sbuf[h];
+            l = sbuf[H + h];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->statack), peer));
+        if (ok) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float lse = l > 0.f ? (m + log2f(l)) * LN2 : -INFINITY;
+            if (p.splits == 1) {
+                uint4* orow = (uint4*)(p.out + ((int64_t)w.t * H + h) * DV);
+#pragma unroll 1
+                for (int j = 0; j < DV / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + j * 32, v);
+                    tmem_ld_wait();
+                    uint32_t o[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const __nv_bfloat162 x = __floats2bfloat162_rn(v[2 * e] * inv, v[2 * e + 1] * inv);
+                        o[e] = *(const uint32_t*)&x;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) orow[j * 4 + e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                }
+                p.lse[(int64_t)w.t * H + h] = lse;
+            } else {
+                const int64_t pr = ((int64_t)w.t * p.splits + w.split) * H + h;
+                float4* orow = (float4*)(p.part_o + pr * DV);
+#pragma unroll 1
+                for (int j = 0; j < DV / 32; ++j) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + j * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        orow[j * 8 + e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv, v[4 * e + 3] * inv);
+                }
+                p.part_lse[pr] = lse;
+            }
+        }
+    } else if (warp == 8) {
+        // ----------------------------------------------------- MMA issuer ----
+        if (elect_one()) {
+            if (rank == 0) {
+                constexpr uint32_t idesc = idesc_bf16_f32(H, NK, 0, 0);
+                const uint32_t kbase = smem_u32(gbuf);
+                bool ok = mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                tc_fence_after();
+                for (int c = 0; c < w.nchunks && ok; ++c) {
+                    const int st = c & 1, sb = c & 1;
+                    ok = mbar_wait(&bars->kfull[st], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
+                         mbar_wait(&bars->sempty[sb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    if (!ok) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t boff = (uint32_t)(st * KSTAGE + (kk >> 2) * (NK * 128) + (kk & 3) * 32);
+                        mma_ts(tmem + S_COL + sb * NK, tmem + kk * 8, desc_sw128(kbase + boff, 1024), idesc, kk > 0);
+                    }
+                    mma_commit(&bars->kempty[st]);
+                    mma_commit(&bars->sfull[sb]);
+                }
+            } else {
+                constexpr uint32_t idesc = idesc_bf16_f32(H, 256, 0, 1);
+                const uint32_t vbase = smem_u32(gbuf), pbase = smem_u32(pbuf);
+                bool ok = true;
+                for (int c = 0; c < w.nchunks && ok; ++c) {
+                    const int st = c & 1, pb = c & 1;
+                    ok = mbar_wait(&bars->vfull[st], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
+                         mbar_wait(&bars->ready[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    if (!ok) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < NK / 16; ++kk) {
+                        const uint64_t adesc = desc_sw128(pbase + pb * PBYTES + kk * 32, 1024);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const uint32_t boff = (uint32_t)(st * VSTAGE + half * 4 * (NK * 128) + kk * 16 * 128);
+                            mma_ss(tmem + half * 256, adesc, desc_sw128_mn(vbase + boff, NK * 128, 1024), idesc,
+                                   (c > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&bars->vempty[st]);
+                    mma_commit_multicast(&bars->pempty[pb], (uint16_t)0x3);
+                    mma_commit(&bars->odone);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// Merge of split partials: out = sum_s exp(lse_s - lse) * O_s, lse = log sum_s exp(lse_s).
+__global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse, int splits,
+                                                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    const int t = blockIdx.x, h = blockIdx.y;
+    const int d = threadIdx.x * 4;
+    float mx = -INFINITY;
+    for (int s = 0; s < splits; ++s) mx = fmaxf(mx, __ldg(part_lse + ((int64_t)t * splits + s) * H + h));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    if (mx > -INFINITY) {
+        for (int s = 0; s < splits; ++s) {
+            const int64_t pr = ((int64_t)t * splits + s) * H + h;
+            const float ls = __ldg(part_lse + pr);
+            if (ls == -INFINITY) continue;
+            const float wgt = __expf(ls - mx);
+            den += wgt;
+            const float4 o = __ldg((const float4*)(part_o + pr * DV + d));
+            acc.x = fmaf(wgt, o.x, acc.x); acc.y = fmaf(wgt, o.y, acc.y);
+            acc.z = fmaf(wgt, o.z, acc.z); acc.w = fmaf(wgt, o.w, acc.w);
+        }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 pk = make_uint2(*(uint32_t*)&lo, *(uint32_t*)&hi);
+    *(uint2*)(out + ((int64_t)t * H + h) * DV + d) = pk;
+    if (threadIdx.x == 0) lse[(int64_t)t * H + h] = den > 0.f ? mx + __logf(den) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ host --
+
+namespace {
+
+constexpr size_t MLA_SMEM = 1024 + REGION + 2 * PBYTES + 2 * ABYTES + SBYTES + 256;
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+int choose_splits(int rows, int k, int num_sms) {
+    const int clusters = num_sms / 2;
+    const int max_split = (k + NK - 1) / NK;
+    int s = rows >= clusters ? 1 : clusters / rows;
+    if (s > max_split) s = max_split;
+    return s < 1 ? 1 : s;
+}
+
+}  // namespace
+
+bool mla_tc_supported(dsa_dtype_t dtype, int n_heads, int d_qk, int d_v) {
+    return dtype == DSA_BF16 && n_heads == H && d_qk == DK && d_v == DV;
+}
+
+size_t mla_tc_workspace_bytes(int rows, int k, int num_sms) {
+    const int s = choose_splits(rows, k, num_sms);
+    if (s == 1) return 0;
+    return (size_t)rows * s * H * (DV + 1) * sizeof(float);
+}
+
+cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
+                          const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch, int ctx_len,
+                          float scale, void* out, float* lse, void* workspace, size_t ws_bytes) {
+    if (rows == 0) return cudaSuccess;
+    MlaParams p;
+    p.q = (const __nv_bfloat16*)q;
+    p.kv = (const __nv_bfloat16*)kv;
+    p.page_table = page_table;
+    p.row_batch = row_batch;
+    p.idx = idx;
+    p.out = (__nv_bfloat16*)out;
+    p.lse = lse;
+    p.err = L.err;
+    p.page_size = page_table ? page_size : 1;
+    p.pages_per_seq = page_table ? ctx_len / page_size : 0;
+    p.k = k;
+    p.rows = rows;
+    p.batch = batch;
+    p.ctx = ctx_len;
+    p.splits = choose_splits(rows, k, L.num_sms);
+    const int per = (k + p.splits - 1) / p.splits;
+    p.per_split = (per + NK - 1) / NK * NK;
+    p.splits = (k + p.per_split - 1) / p.per_split;            // no empty split
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
+    if (p.splits > 1) {
+        const size_t need = (size_t)rows * p.splits * H * (DV + 1) * sizeof(float);
+        if (!workspace || ws_bytes < need) return cudaErrorInvalidValue;
+        p.part_o = (float*)workspace;
+        p.part_lse = p.part_o + (size_t)rows * p.splits * H * DV;
+    }
+    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * (unsigned)rows * (unsigned)p.splits);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = MLA_SMEM;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, p);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    if (p.splits > 1) {
+        mla_combine_kernel<<<dim3(rows, H), 128, 0, L.stream>>>(p.part_o, p.part_lse, p.splits,
+                                                               (__nv_bfloat16*)out, lse);
+        count_launch();
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

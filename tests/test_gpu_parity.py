@@ -133,6 +133,43 @@ def test_sparse_mla_on_given_indices(cuda_device, wl, pad):
     assert lerr <= ATOL_LSE[wl.dtype], lerr
 
 
+@pytest.mark.parametrize("order", ["ascending", "descending", "shuffled"])
+def test_sparse_mla_running_max_moves(cuda_device, order):
+    """Scores that climb by many e-folds across the key list, so the running
+    maximum moves again and again (the lazy-rescale path of the kernel)."""
+    wl = workloads.DECODE_32K.with_(batch=2, rows=3, ctx=4096)
+    inp = workloads.generate(wl, parts=("mla",))
+    q, kv = inp["q"].float(), inp["kv"].float()
+    ramp = torch.arange(wl.ctx, dtype=torch.float32) * 0.02           # rope dims carry the ramp
+    kv[:, :, 512:] = ramp.view(1, -1, 1)
+    q[:, :, 512:] = 1.0
+    q, kv = q.to(torch.bfloat16), kv.to(torch.bfloat16)
+    g = torch.Generator().manual_seed(11)
+    idx = _random_idx(wl.rows, 2048, wl.ctx, g)
+    if order == "ascending":
+        idx = idx.sort(dim=1).values
+    elif order == "descending":
+        idx = idx.sort(dim=1, descending=True).values
+    out, lse = dsa.sparse_mla(q.to(cuda_device), kv.to(cuda_device), idx.to(cuda_device),
+                              inp["row_batch"].to(cuda_device), wl.softmax_scale, wl.d_v, wl.ctx)
+    ro, rl, _ = oracle.sparse_mla(q, kv, idx, inp["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
+    assert np.abs(out.float().cpu().numpy() - ro).max() <= ATOL_OUT["bf16"]
+    assert np.abs(lse.cpu().numpy() - rl).max() <= ATOL_LSE["bf16"]
+
+
+def test_sparse_mla_all_slots_unused(cuda_device):
+    wl = workloads.DECODE_32K.with_(batch=2, rows=2, ctx=512)
+    inp = workloads.generate(wl, parts=("mla",))
+    idx = torch.full((2, 300), -1, dtype=torch.int32)
+    idx[1, 7] = 5
+    dv = _cuda(inp, cuda_device)
+    out, lse = dsa.sparse_mla(dv["q"], dv["kv"], idx.to(cuda_device), dv["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
+    o, l = out.float().cpu().numpy(), lse.cpu().numpy()
+    assert np.all(o[0] == 0) and np.all(np.isneginf(l[0]))
+    row = inp["kv"][1, 5, :512].float().numpy()
+    assert np.abs(o[1] - row[None, :]).max() <= 1e-2
+
+
 # ----------------------------------------------------------- whole chain ----
 
 @pytest.mark.parametrize("wl", [
