@@ -319,6 +319,42 @@ def cpu_baseline_decode(wl, inp, budget_s: float = 12.0):
     return done / t_used, done, oracle.max_threads(), t_used
 
 
+def run_kernel_only(args):
+    """One kernel of the step, alone, on the workload's real inputs (the step
+    runs once first so that top-k indices exist).  Used for profiler captures
+    of a single kernel; prints its mean event time."""
+    import torch
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import sparse_attention_logits_b200 as dsa
+    import workloads
+    wl = workloads.BY_NAME[args.workload]
+    inp = workloads.generate(wl, device=device, seed=0)
+    step = DecodeStep(dsa, wl, inp, device)
+    step.run()
+    i = inp
+    launch = {
+        "indexer": lambda: dsa.indexer_logits(i["q_idx"], i["w"], i["k_idx"], i["row_batch"], i["row_pos"],
+                                              k_scale=i.get("k_scale"), out=step.logits),
+        "topk": lambda: dsa.topk(step.logits, i["row_pos"], wl.topk, ctx_len=wl.ctx, out=step.idx,
+                                 workspace=step.topk_ws),
+        "mla": lambda: dsa.sparse_mla(i["q"], i["kv"], step.idx, i["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx,
+                                      page_table=i.get("page_table"), out=step.out, lse=step.lse,
+                                      workspace=step.mla_ws),
+    }[args.kernel_only]
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        launch()
+    b.record()
+    torch.cuda.synchronize()
+    dsa.get_device_error(device)
+    print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": a.elapsed_time(b) / args.steps}))
+
+
 def run_ours(args):
     import torch
     rank, world = init_dist("nccl")
@@ -454,10 +490,14 @@ def main(argv=None):
     ap.add_argument("--workload", default="dsa_decode_bf16_B32_L32768_k2048")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla"], default=None,
+                    help="time one kernel of the step alone (for profiler captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.kernel_only:
+        run_kernel_only(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -28,8 +28,8 @@
 //                       over several clusters, normalised fp32 partials that
 //                       dsa_mla_combine merges.
 //
-// Warps (both CTAs): 0-3 gather producers, 4-7 softmax (score CTA) or
-// rescale + epilogue (value CTA), one thread per head / TMEM lane, 8 MMA
+// Warps (both CTAs): 0-7 gather producers, 8-11 softmax (score CTA) or
+// rescale + epilogue (value CTA), one thread per head / TMEM lane, 12 MMA
 // issuer and TMEM owner.  Every wait is bounded; the two CTAs only exchange
 // data through bulk copies and mbarrier arrivals that the receiver waits on.
 #include "common.cuh"
@@ -46,12 +46,17 @@ constexpr int H = 128;              // query heads = MMA M
 constexpr int DK = 576;             // latent + rope
 constexpr int DV = 512;             // value dims
 constexpr int NK = 64;              // keys per chunk
-constexpr int THREADS = 288;        // 9 warps
+constexpr int PWARPS = 8;           // gather producer warps (each keeps its own copies in flight)
+constexpr int ROWS_PER_PW = NK / PWARPS;
+constexpr int SWARP0 = PWARPS;      // first of the 4 softmax / rescale-epilogue warps
+constexpr int MWARP = PWARPS + 4;   // MMA issuer, TMEM owner
+constexpr int THREADS = 32 * (PWARPS + 5);
 constexpr int KSTAGE = NK * DK * 2; // 73728 B
 constexpr int VSTAGE = NK * DV * 2; // 65536 B
 constexpr int STAGES = 2;
 constexpr int REGION = (STAGES * KSTAGE > STAGES * VSTAGE) ? STAGES * KSTAGE : STAGES * VSTAGE;
 constexpr int PBYTES = H * NK * 2;  // 16384: P [128 heads x 64 keys] bf16
+constexpr int PSLOTS = 4;           // P ring depth (score CTA may run this many chunks ahead)
 constexpr int ABYTES = H * 4;       // rescale factor per head
 constexpr int SBYTES = 2 * H * 4;   // final running max and sum per head
 constexpr int S_COL = 320;          // score CTA: Q in TMEM columns [0, 288), S buffers at 320, 384
@@ -60,8 +65,8 @@ constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between 
 constexpr float LN2 = 0.6931471805599453f;
 
 struct Bars {                       // same offset in both CTAs of a cluster
-    uint64_t kfull[2], kempty[2], sfull[2], sempty[2], pready[2], pempty[2], qready, statready, statack;
-    uint64_t vfull[2], vempty[2], pfull[2], ready[2], odone, statfull;
+    uint64_t kfull[2], kempty[2], sfull[2], sempty[2], pready[PSLOTS], pempty[PSLOTS], qready, statready, statack;
+    uint64_t vfull[2], vempty[2], pfull[PSLOTS], ready[PSLOTS], odone, statfull;
     uint32_t tmem;
     int abort;
 };
@@ -116,8 +121,38 @@ __device__ __forceinline__ int64_t key_row(const MlaParams& p, const Work& w, in
     return (int64_t)w.b * p.ctx + s;
 }
 
+// 2^x on the MUFU unit (ex2.approx, flush-to-zero): relative error ~2^-22,
+// far below the bf16 rounding that P goes through next; -inf -> +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+template <int RC>   // 16-byte pieces per gathered row
+__device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, int stage_bytes,
+                                            uint64_t* full, uint64_t* empty, int warp, int lane,
+                                            volatile int* abort_flag) {
+    for (int c = 0; c < w.nchunks; ++c) {
+        const int st = c & 1;
+        if (!mbar_wait(&empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+        const int64_t myrow = key_row(p, w, w.slot0 + c * NK + warp * ROWS_PER_PW + (lane % ROWS_PER_PW));
+        const int myrow_lo = (int)(myrow >= 0 ? myrow : -1);       // row indices fit in 31 bits
+        uint8_t* base = gbuf + (size_t)st * stage_bytes;
+#pragma unroll 4
+        for (int i = lane; i < ROWS_PER_PW * RC; i += 32) {
+            const int rl = i / RC, ci = i - rl * RC;
+            const int row = __shfl_sync(0xffffffffu, myrow_lo, rl);
+            const int r = warp * ROWS_PER_PW + rl;
+            const __nv_bfloat16* src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8 : p.kv;
+            cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(&full[st]);
+    }
+}
 
 }  // namespace
 
@@ -125,9 +160,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
-    uint8_t* pbuf = gbuf + REGION;                          // [2][PBYTES]
-    float* abuf = (float*)(pbuf + 2 * PBYTES);              // [2][H]
-    float* sbuf = abuf + 2 * H;                             // [2*H]: running max, running sum
+    uint8_t* pbuf = gbuf + REGION;                          // [PSLOTS][PBYTES]
+    float* abuf = (float*)(pbuf + PSLOTS * PBYTES);         // [PSLOTS][H]
+    float* sbuf = abuf + PSLOTS * H;                        // [2*H]: running max, running sum
     Bars* bars = (Bars*)(sbuf + 2 * H);
     volatile int* abort_flag = &bars->abort;
 
@@ -137,14 +172,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars->kfull[i], 128);
+            mbar_init(&bars->kfull[i], PWARPS * 32);
             mbar_init(&bars->kempty[i], 1);
             mbar_init(&bars->sfull[i], 1);
             mbar_init(&bars->sempty[i], 4);
+            mbar_init(&bars->vfull[i], PWARPS * 32);
+            mbar_init(&bars->vempty[i], 1);
+        }
+        for (int i = 0; i < PSLOTS; ++i) {
             mbar_init(&bars->pready[i], 4);
             mbar_init(&bars->pempty[i], 1);
-            mbar_init(&bars->vfull[i], 128);
-            mbar_init(&bars->vempty[i], 1);
             mbar_init(&bars->pfull[i], 1);
             mbar_init(&bars->ready[i], 4);
         }
@@ -157,13 +194,12 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
         if (rank == 1) {
             // arm the first phase of each P slot and the final-statistics slot
-            mbar_arrive_expect_tx(&bars->pfull[0], PBYTES + ABYTES);
-            if (w.nchunks > 1) mbar_arrive_expect_tx(&bars->pfull[1], PBYTES + ABYTES);
+            for (int i = 0; i < PSLOTS && i < w.nchunks; ++i) mbar_arrive_expect_tx(&bars->pfull[i], PBYTES + ABYTES);
             mbar_arrive_expect_tx(&bars->statfull, SBYTES);
         }
         fence_mbar_init();
     }
-    if (warp == 8) {
+    if (warp == MWARP) {
         tmem_alloc(&bars->tmem, TMEM_COLS);
         tmem_relinquish();
     }
@@ -173,45 +209,36 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
     const uint32_t tmem = bars->tmem;
     const uint32_t peer = rank ^ 1u;
 
-    if (warp < 4) {
+    if (warp < PWARPS) {
         // ------------------------------------------------ gather producers ----
-        const int tid = threadIdx.x;
-        const int row_chunks = rank == 0 ? DK / 8 : DV / 8;    // 16-byte chunks per gathered row
-        const int stage_bytes = rank == 0 ? KSTAGE : VSTAGE;
-        uint64_t* full = rank == 0 ? bars->kfull : bars->vfull;
-        uint64_t* empty = rank == 0 ? bars->kempty : bars->vempty;
-        for (int c = 0; c < w.nchunks; ++c) {
-            const int st = c & 1;
-            if (!mbar_wait(&empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
-            uint8_t* base = gbuf + (size_t)st * stage_bytes;
-            int cur_r = -1;
-            int64_t row = -1;
-            for (int i = tid; i < NK * row_chunks; i += 128) {
-                const int r = i / row_chunks, ci = i - r * row_chunks;
-                if (r != cur_r) {
-                    cur_r = r;
-                    row = key_row(p, w, w.slot0 + c * NK + r);
-                }
-                const __nv_bfloat16* src = row >= 0 ? p.kv + row * DK + ci * 8 : p.kv;
-                cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(&full[st]);
-        }
-    } else if (warp < 8 && rank == 0) {
+        // Warp w owns rows [8w, 8w+8) of every chunk: lane l resolves one of
+        // them once per chunk (one index load per lane, all in flight
+        // together); the copy loop then walks the warp's rows with consecutive
+        // lanes on consecutive 16-byte pieces of a row.  Several warps are
+        // used because each keeps only a bounded number of copies in flight.
+        if (rank == 0) gather_rows<DK / 8>(p, w, gbuf, KSTAGE, bars->kfull, bars->kempty, warp, lane, abort_flag);
+        else gather_rows<DV / 8>(p, w, gbuf, VSTAGE, bars->vfull, bars->vempty, warp, lane, abort_flag);
+    } else if (warp < SWARP0 + 4 && rank == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
-        const int h = (warp - 4) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        const int h = (warp - SWARP0) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp - SWARP0) * 32) << 16;
         {   // Q row of head h -> TMEM lane h, columns [0, 288) (bf16 pairs)
             const uint4* qrow = (const uint4*)(p.q + ((int64_t)w.t * H + h) * DK);
 #pragma unroll 1
-            for (int m = 0; m < DK / 32; ++m) {
-                uint32_t words[16];
+            for (int m0 = 0; m0 < DK / 32; m0 += 6) {          // 3 batches, 24 loads in flight each
+                uint4 x[24];
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 x = __ldg(qrow + m * 4 + v);
-                    words[4 * v] = x.x; words[4 * v + 1] = x.y; words[4 * v + 2] = x.z; words[4 * v + 3] = x.w;
+                for (int v = 0; v < 24; ++v) x[v] = __ldg(qrow + m0 * 4 + v);
+#pragma unroll
+                for (int m = 0; m < 6; ++m) {
+                    uint32_t words[16];
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        words[4 * v] = x[4 * m + v].x; words[4 * v + 1] = x[4 * m + v].y;
+                        words[4 * v + 2] = x[4 * m + v].z; words[4 * v + 3] = x[4 * m + v].w;
+                    }
+                    tmem_st16(tmem + lane_base + (m0 + m) * 16, words);
                 }
-                tmem_st16(tmem + lane_base + m * 16, words);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -222,12 +249,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
         bool ok = true;
+        // which of the 64 keys of a chunk are real (looked up one chunk ahead)
+        bool va_next = key_row(p, w, w.slot0 + lane) >= 0;
+        bool vb_next = key_row(p, w, w.slot0 + 32 + lane) >= 0;
         for (int c = 0; c < w.nchunks && ok; ++c) {
             const int sb = c & 1;
-            // which of the 64 keys of this chunk are real
-            const bool va = key_row(p, w, w.slot0 + c * NK + lane) >= 0;
-            const bool vb = key_row(p, w, w.slot0 + c * NK + 32 + lane) >= 0;
-            const uint32_t mlo = __ballot_sync(0xffffffffu, va), mhi = __ballot_sync(0xffffffffu, vb);
+            const uint32_t mlo = __ballot_sync(0xffffffffu, va_next), mhi = __ballot_sync(0xffffffffu, vb_next);
+            if (c + 1 < w.nchunks) {
+                va_next = key_row(p, w, w.slot0 + (c + 1) * NK + lane) >= 0;
+                vb_next = key_row(p, w, w.slot0 + (c + 1) * NK + 32 + lane) >= 0;
+            }
             ok = mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
             if (!ok) break;
             tc_fence_after();
@@ -238,13 +269,19 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->sempty[sb]);
-            float mc = -INFINITY;
+            float mx[16];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 s0[j] = ((mlo >> j) & 1u) ? s0[j] * p.scale_log2 : -INFINITY;
                 s1[j] = ((mhi >> j) & 1u) ? s1[j] * p.scale_log2 : -INFINITY;
-                mc = fmaxf(mc, fmaxf(s0[j], s1[j]));
             }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(fmaxf(s0[2 * j], s0[2 * j + 1]), fmaxf(s1[2 * j], s1[2 * j + 1]));
+#pragma unroll
+            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
+            const float mc = mx[0];
             float alpha = 1.f;
             if (mc > -INFINITY) {
                 if (m_run == -INFINITY) {
@@ -256,22 +293,25 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 }
             }
             uint32_t pk[32];
-            float lsum = 0.f;
+            float ls[16];
+            // exp2 of (score - running max): arguments are <= 2^3 above 0 at most
+            // (lazy rescale) and -inf for unused keys, which ex2 maps to +0.
+            const float mr = m_run == -INFINITY ? 0.f : m_run;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float a0 = s0[2 * j] == -INFINITY ? 0.f : exp2f(s0[2 * j] - m_run);
-                const float a1 = s0[2 * j + 1] == -INFINITY ? 0.f : exp2f(s0[2 * j + 1] - m_run);
-                const float b0 = s1[2 * j] == -INFINITY ? 0.f : exp2f(s1[2 * j] - m_run);
-                const float b1 = s1[2 * j + 1] == -INFINITY ? 0.f : exp2f(s1[2 * j + 1] - m_run);
-                const __nv_bfloat162 pa = __floats2bfloat162_rn(a0, a1);
-                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(b0, b1);
-                lsum += __low2float(pa) + __high2float(pa) + __low2float(pb2) + __high2float(pb2);
+                const __nv_bfloat162 pa = __floats2bfloat162_rn(fast_exp2(s0[2 * j] - mr), fast_exp2(s0[2 * j + 1] - mr));
+                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(fast_exp2(s1[2 * j] - mr), fast_exp2(s1[2 * j + 1] - mr));
+                ls[j] = (__low2float(pa) + __high2float(pa)) + (__low2float(pb2) + __high2float(pb2));
                 pk[j] = *(const uint32_t*)&pa;
                 pk[16 + j] = *(const uint32_t*)&pb2;
             }
-            l_run += lsum;
-            const int pb = c & 1;
-            ok = mbar_wait_cluster(&bars->pempty[pb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+#pragma unroll
+            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
+            l_run += ls[0];
+            const int pb = c % PSLOTS, pu = c / PSLOTS;
+            ok = mbar_wait_cluster(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
             if (!ok) break;
             uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
 #pragma unroll
@@ -281,8 +321,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->pready[pb]);
-            if (warp == 4 && lane == 0) {
-                ok = mbar_wait(&bars->pready[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (warp == SWARP0 && lane == 0) {
+                ok = mbar_wait(&bars->pready[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 if (ok) {
                     const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
                     bulk_copy_s2cluster(peer_pbuf + pb * PBYTES, pbuf + pb * PBYTES, PBYTES, rbar);
@@ -297,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->statready);
-        if (warp == 4 && lane == 0 && !*abort_flag) {
+        if (warp == SWARP0 && lane == 0 && !*abort_flag) {
             if (mbar_wait(&bars->statready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag))
                 bulk_copy_s2cluster(mapa_shared(smem_u32(sbuf), peer), sbuf, SBYTES,
                                     mapa_shared(smem_u32(&bars->statfull), peer));
@@ -305,18 +345,18 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         // stay alive until the value CTA has read the statistics and its last
         // MMA commits (which arrive on our P-slot barriers) have landed
         mbar_wait_cluster(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-        for (int c = max(0, w.nchunks - 2); c < w.nchunks; ++c)
-            mbar_wait_cluster(&bars->pempty[c & 1], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-    } else if (warp < 8) {
+        for (int c = max(0, w.nchunks - PSLOTS); c < w.nchunks; ++c)
+            mbar_wait_cluster(&bars->pempty[c % PSLOTS], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+    } else if (warp < SWARP0 + 4) {
         // ------------------------- value CTA: rescale of O, then epilogue ----
-        const int h = (warp - 4) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)((warp - 4) * 32) << 16;
+        const int h = (warp - SWARP0) * 32 + lane;
+        const uint32_t lane_base = (uint32_t)((warp - SWARP0) * 32) << 16;
         bool ok = true;
         for (int c = 0; c < w.nchunks && ok; ++c) {
-            const int pb = c & 1;
-            ok = mbar_wait_cluster(&bars->pfull[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            const int pb = c % PSLOTS, pu = c / PSLOTS;
+            ok = mbar_wait_cluster(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
             if (!ok) break;
-            if (warp == 4 && lane == 0 && c + 2 < w.nchunks)
+            if (warp == SWARP0 && lane == 0 && c + PSLOTS < w.nchunks)
                 mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
             const float alpha = abuf[pb * H + h];
             if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -383,7 +423,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 p.part_lse[pr] = lse;
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == MWARP) {
         // ----------------------------------------------------- MMA issuer ----
         if (elect_one()) {
             if (rank == 0) {
@@ -411,9 +451,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 const uint32_t vbase = smem_u32(gbuf), pbase = smem_u32(pbuf);
                 bool ok = true;
                 for (int c = 0; c < w.nchunks && ok; ++c) {
-                    const int st = c & 1, pb = c & 1;
+                    const int st = c & 1, pb = c % PSLOTS;
                     ok = mbar_wait(&bars->vfull[st], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
-                         mbar_wait(&bars->ready[pb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                         mbar_wait(&bars->ready[pb], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                     if (!ok) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
@@ -437,7 +477,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == MWARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -477,8 +517,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restric
 
 namespace {
 
-constexpr size_t MLA_SMEM = 1024 + REGION + 2 * PBYTES + 2 * ABYTES + SBYTES + 256;
-static_assert(sizeof(Bars) <= 256, "barrier block");
+constexpr size_t MLA_SMEM = 1024 + REGION + PSLOTS * (PBYTES + ABYTES) + SBYTES + 512;
+static_assert(sizeof(Bars) <= 512, "barrier block");
 
 int choose_splits(int rows, int k, int num_sms) {
     const int clusters = num_sms / 2;
