@@ -129,6 +129,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// Raw key position stored in a slot (-1 past the end of this split's slots).
+__device__ __forceinline__ int slot_index(const MlaParams& p, const Work& w, int slot) {
+    return slot < w.slot_end ? __ldg(p.idx + (int64_t)w.t * p.k + slot) : -1;
+}
+
 // Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
@@ -136,11 +141,12 @@ template <int RC>   // 16-byte pieces per gathered row
 __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, int stage_bytes,
                                             uint64_t* full, uint64_t* empty, int warp, int lane,
                                             volatile int* abort_flag) {
+    const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
+    int64_t next_row = key_row(p, w, w.slot0 + my_slot);
     for (int c = 0; c < w.nchunks; ++c) {
         const int st = c & 1;
         if (!mbar_wait(&empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
-        const int64_t myrow = key_row(p, w, w.slot0 + c * NK + warp * ROWS_PER_PW + (lane % ROWS_PER_PW));
-        const int myrow_lo = (int)(myrow >= 0 ? myrow : -1);       // row indices fit in 31 bits
+        const int myrow_lo = (int)(next_row >= 0 ? next_row : -1);  // row indices fit in 31 bits
         uint8_t* base = gbuf + (size_t)st * stage_bytes;
 #pragma unroll 4
         for (int i = lane; i < ROWS_PER_PW * RC; i += 32) {
@@ -151,6 +157,8 @@ __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, u
             cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
         }
         cp_async_arrive_noinc(&full[st]);
+        // look up the next chunk's row while this chunk's copies are in flight
+        if (c + 1 < w.nchunks) next_row = key_row(p, w, w.slot0 + (c + 1) * NK + my_slot);
     }
 }
 
@@ -249,15 +257,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
         bool ok = true;
-        // which of the 64 keys of a chunk are real (looked up one chunk ahead)
-        bool va_next = key_row(p, w, w.slot0 + lane) >= 0;
-        bool vb_next = key_row(p, w, w.slot0 + 32 + lane) >= 0;
+        // which of the 64 keys of a chunk are real: the raw indices are loaded
+        // one chunk ahead and only inspected in the next iteration
+        int sa_next = slot_index(p, w, w.slot0 + lane), sb_next = slot_index(p, w, w.slot0 + 32 + lane);
         for (int c = 0; c < w.nchunks && ok; ++c) {
             const int sb = c & 1;
-            const uint32_t mlo = __ballot_sync(0xffffffffu, va_next), mhi = __ballot_sync(0xffffffffu, vb_next);
+            const uint32_t mlo = __ballot_sync(0xffffffffu, w.b_ok && sa_next >= 0 && sa_next < p.ctx);
+            const uint32_t mhi = __ballot_sync(0xffffffffu, w.b_ok && sb_next >= 0 && sb_next < p.ctx);
             if (c + 1 < w.nchunks) {
-                va_next = key_row(p, w, w.slot0 + (c + 1) * NK + lane) >= 0;
-                vb_next = key_row(p, w, w.slot0 + (c + 1) * NK + 32 + lane) >= 0;
+                sa_next = slot_index(p, w, w.slot0 + (c + 1) * NK + lane);
+                sb_next = slot_index(p, w, w.slot0 + (c + 1) * NK + 32 + lane);
             }
             ok = mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
             if (!ok) break;
@@ -311,7 +320,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
             l_run += ls[0];
             const int pb = c % PSLOTS, pu = c / PSLOTS;
-            ok = mbar_wait_cluster(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            ok = mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
             if (!ok) break;
             uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
 #pragma unroll
@@ -344,9 +353,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         }
         // stay alive until the value CTA has read the statistics and its last
         // MMA commits (which arrive on our P-slot barriers) have landed
-        mbar_wait_cluster(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+        mbar_wait(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         for (int c = max(0, w.nchunks - PSLOTS); c < w.nchunks; ++c)
-            mbar_wait_cluster(&bars->pempty[c % PSLOTS], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            mbar_wait(&bars->pempty[c % PSLOTS], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
     } else if (warp < SWARP0 + 4) {
         // ------------------------- value CTA: rescale of O, then epilogue ----
         const int h = (warp - SWARP0) * 32 + lane;
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         bool ok = true;
         for (int c = 0; c < w.nchunks && ok; ++c) {
             const int pb = c % PSLOTS, pu = c / PSLOTS;
-            ok = mbar_wait_cluster(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            ok = mbar_wait(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
             if (!ok) break;
             if (warp == SWARP0 && lane == 0 && c + PSLOTS < w.nchunks)
                 mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
@@ -379,7 +388,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             if (lane == 0) mbar_arrive(&bars->ready[pb]);
         }
         if (ok) ok = mbar_wait(&bars->odone, (w.nchunks - 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
-        if (ok) ok = mbar_wait_cluster(&bars->statfull, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+        if (ok) ok = mbar_wait(&bars->statfull, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         float m = -INFINITY, l = 0.f;
         if (ok) {
             m = sbuf[h];
