@@ -189,11 +189,20 @@ class ClockSampler:
 
 # ------------------------------------------------------------ our arm ----
 
+def pool_caches(dsa, wl, inp):
+    """CSA workloads: pool the raw caches m:1 (csa_compress) into block caches."""
+    if wl.compress_m > 1:
+        inp["k_idx"] = dsa.csa_compress(inp["k_idx"], wl.compress_m)
+        inp["kv"] = dsa.csa_compress(inp["kv"], wl.compress_m)
+    return inp
+
+
 class DecodeStep:
     """Preallocated buffers and the three library calls of one step."""
 
     def __init__(self, dsa, wl, inp, device):
         import torch
+        pool_caches(dsa, wl, inp)
         self.dsa, self.wl, self.inp = dsa, wl, inp
         self.logits = torch.empty((wl.rows, wl.ctx), dtype=torch.float32, device=device)
         self.idx = torch.empty((wl.rows, wl.topk), dtype=torch.int32, device=device)
@@ -204,42 +213,77 @@ class DecodeStep:
         n = dsa.sparse_mla_workspace_size(wl.rows, wl.topk, wl.heads, wl.d_qk, wl.d_v, inp["q"].dtype)
         self.mla_ws = torch.empty(max(n, 1), dtype=torch.uint8, device=device) if n else None
 
-    def run(self, events=None):
+    def run_one(self, name):
         d, wl, i = self.dsa, self.wl, self.inp
-        if events: events[0].record()
-        d.indexer_logits(i["q_idx"], i["w"], i["k_idx"], i["row_batch"], i["row_pos"], k_scale=i.get("k_scale"),
-                         out=self.logits)
-        if events: events[1].record()
-        d.topk(self.logits, i["row_pos"], wl.topk, ctx_len=wl.ctx, out=self.idx, workspace=self.topk_ws)
-        if events: events[2].record()
-        d.sparse_mla(i["q"], i["kv"], self.idx, i["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx,
-                     page_table=i.get("page_table"), out=self.out, lse=self.lse, workspace=self.mla_ws)
-        if events: events[3].record()
+        if name == "dsa_indexer_logits":
+            d.indexer_logits(i["q_idx"], i["w"], i["k_idx"], i["row_batch"], i["row_pos"],
+                             k_scale=i.get("k_scale"), out=self.logits)
+        elif name == "dsa_topk":
+            d.topk(self.logits, i["row_pos"], wl.topk, ctx_len=wl.ctx, out=self.idx, workspace=self.topk_ws)
+        else:
+            d.sparse_mla(i["q"], i["kv"], self.idx, i["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx,
+                         page_table=i.get("page_table"), out=self.out, lse=self.lse, workspace=self.mla_ws)
+
+    def run(self):
+        for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla"):
+            self.run_one(name)
+
+
+def _graph(fn):
+    """Capture fn() (library calls on the current stream) into a CUDA graph."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()                                  # warm (kernel attributes, tensor maps) outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, steps, device, flush):
+    """Replay `g` `steps` times with an L2 flush before each replay (outside
+    the events); returns the mean device time of one replay in ms."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
 def time_steps(step, steps, warmup, device, flush):
-    """Warm up, then time `steps` steps with per-step and per-kernel events.
-    Returns (mean step ms, {kernel: mean ms}, launches during the timed steps)."""
+    """The step (indexer -> top-k -> sparse MLA) is captured once into a CUDA
+    graph and replayed: timings are device time, free of host launch gaps.
+    Per-kernel times come from graphs holding one library call each.
+    Returns (mean step ms, {kernel: mean ms}, library kernel launches in the
+    timed steps)."""
     import torch
     dsa = step.dsa
-    for _ in range(warmup):
-        step.run()
-    torch.cuda.synchronize(device)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
-    barrier(device)
-    torch.cuda.synchronize(device)
     n0 = dsa.launch_count()
-    for s in range(steps):
-        flush.zero_()                        # L2 flush, outside the step's events
-        step.run(evs[s])
+    g_step = _graph(step.run)
+    per_step = (dsa.launch_count() - n0) // 2          # launches recorded by the warm run + the capture
+    for _ in range(warmup):
+        g_step.replay()
     torch.cuda.synchronize(device)
-    barrier(device)
-    launches = dsa.launch_count() - n0
-    per = [e[0].elapsed_time(e[3]) for e in evs]
-    kern = {"dsa_indexer_logits": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
-            "dsa_topk": statistics.mean(e[1].elapsed_time(e[2]) for e in evs),
-            "dsa_sparse_mla": statistics.mean(e[2].elapsed_time(e[3]) for e in evs)}
-    return statistics.mean(per), kern, launches
+    ms = time_graph(g_step, steps, device, flush)
+    kern = {}
+    for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla"):
+        g = _graph(lambda n=name: step.run_one(n))
+        g.replay()
+        kern[name] = time_graph(g, max(3, steps // 2), device, flush)
+        del g
+    return ms, kern, per_step * steps
 
 
 def e2e_decode(dsa, wl, inp, step, steps, device):
@@ -352,7 +396,11 @@ def run_kernel_only(args):
     b.record()
     torch.cuda.synchronize()
     dsa.get_device_error(device)
-    print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": a.elapsed_time(b) / args.steps}))
+    host_ms = a.elapsed_time(b) / args.steps
+    g = _graph(launch)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    dev_ms = time_graph(g, args.steps, device, flush)
+    print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": dev_ms, "ms_stream_launches": host_ms}))
 
 
 def run_ours(args):
@@ -393,7 +441,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "topk": wl.topk,
                    "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "mla": f"{wl.heads}h {wl.d_qk}/{wl.d_v}",
-                   "parallelism": f"replicas{world}",
+                   "parallelism": f"replicas{world}", "launch": "CUDA graph of the step (device time)",
                    "l2": "inputs larger than L2 (keys 268 MB, latent cache 1.2 GB); 256 MB write between steps"},
         "roofline": roof,
         "kernels_ms": {k: round(v, 4) for k, v in kern.items()},

@@ -134,7 +134,7 @@ DSA_API size_t dsa_topk_workspace_size(int rows, int ctx_len, int k);
  * Order of scores: larger first; equal scores (with -0.0 == +0.0) go to the
  * lower position; -inf is the lowest score.  The selection is exact and
  * deterministic.  NaN scores are not supported.  k in [1, 8192];
- * ctx_len <= ld.
+ * ctx_len <= ld; ctx_len <= 327680 (a row is held on chip by at most 8 SMs).
  */
 DSA_API dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, int rows, int ctx_len,
                       int k, int32_t* idx, void* workspace, size_t workspace_bytes, void* stream);

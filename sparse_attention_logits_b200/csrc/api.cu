@@ -132,6 +132,7 @@ dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, i
     if (rows == 0) return DSA_OK;
     if (!logits || !row_pos || !idx) return fail(DSA_ERR_INVALID_ARG, "dsa_topk: null pointer");
     if (ld < ctx_len) return fail(DSA_ERR_INVALID_ARG, "dsa_topk: ld < ctx_len");
+    if (!dsa::topk_supported(ctx_len)) return fail(DSA_ERR_UNSUPPORTED, "dsa_topk: ctx_len %d above the supported maximum", ctx_len);
     const size_t need = dsa::topk_workspace_bytes(rows, ctx_len, k);
     if (need && (!workspace || workspace_bytes < need))
         return fail(DSA_ERR_INVALID_ARG, "dsa_topk: workspace of %zu bytes needed", need);

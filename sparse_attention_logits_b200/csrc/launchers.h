@@ -22,6 +22,7 @@ cudaError_t launch_indexer_tc(const Launch& L, const void* q, dsa_dtype_t k_dtyp
 cudaError_t launch_topk(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows,
                         int ctx_len, int k, int32_t* idx, void* workspace, size_t ws_bytes);
 size_t topk_workspace_bytes(int rows, int ctx_len, int k);
+bool topk_supported(int ctx_len);
 
 bool mla_simt_supported(int d_qk, int d_v, int n_heads);
 cudaError_t launch_mla_simt(const Launch& L, const void* q, const void* kv, dsa_dtype_t dtype,

@@ -3,24 +3,34 @@
 // lower position first among equal scores, every visible key when no more
 // than k are visible.
 //
-// Exact radix select on order-preserving 32-bit keys, one CTA of 1024
-// threads per query row:
-//   1. four 8-bit digit passes, most significant first, each a shared-memory
-//      histogram of the keys that still match the digits chosen so far; the
-//      digit holding the k-th largest key is found by a suffix scan, which
-//      yields the exact k-th key T and the number of keys above it;
-//   2. an ordered compaction: every key > T, plus the first (in position
-//      order) keys equal to T until k are taken.  Threads own contiguous
-//      position ranges and a block-wide scan gives each its output offset,
-//      so the output is in ascending position order and deterministic.
-// The scores of a row (<= 1 MB) stay L2-resident between passes.
+// Exact radix select on order-preserving 32-bit keys.  One thread-block
+// cluster of CL CTAs (1..8) handles one query row; CTA r of the cluster owns
+// a contiguous slice of the row, loaded once into shared memory as keys.
+//   1. three digit passes (11, 11, 10 bits, most significant first): every
+//      CTA histograms the keys of its slice that still match the digits
+//      chosen so far; the CTAs add up each other's histograms through
+//      distributed shared memory and each finds, by a suffix scan, the digit
+//      that holds the k-th largest key.  After the last pass every CTA knows
+//      the exact k-th key T and how many keys equal to T must be taken.
+//   2. ordered compaction: every key > T, plus the first keys == T in
+//      position order until k are taken.  Per-CTA counts are exchanged
+//      through distributed shared memory, so the output of the whole row is
+//      in ascending position order and deterministic.
+// -0.0 is mapped to +0.0 before the key map, so the two zeros tie.
 #include "common.cuh"
 #include "launchers.h"
+#include "sm100.cuh"
 
 namespace dsa {
 
+using namespace sm100;
+
 namespace {
+
 constexpr int TOPK_THREADS = 1024;
+constexpr int NBINS = 2048;                    // 11-bit digits
+constexpr int SLICE_CAP = 40960;               // keys per CTA kept in shared memory (160 KB)
+constexpr int SMEM_FIXED = 4 * NBINS * 4 + 64 * 4 + 8 * 16;   // hist, 3 per-pass merged histograms, scratch
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -41,7 +51,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
             uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
             if (lane >= o) inc += y;
         }
-        warp_sums[lane] = inc - s;     // exclusive prefix of warp totals
+        warp_sums[lane] = inc - s;
         if (lane == 31) warp_sums[32] = inc;
     }
     __syncthreads();
@@ -50,97 +60,351 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_s
     __syncthreads();
     return r;
 }
+
+template <int CL>
+__device__ __forceinline__ void cl_sync() {
+    if (CL > 1) cluster_sync_all();
+    else __syncthreads();
+}
+
+template <int CL>
+__device__ __forceinline__ uint32_t cl_rank() {
+    return CL > 1 ? cluster_ctarank() : 0u;
+}
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint2 ld_cluster_v2(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared::cluster.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
+    asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 }  // namespace
 
-__global__ void __launch_bounds__(TOPK_THREADS, 1) topk_radix_kernel(
+template <int CL>
+__global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     const float* __restrict__ logits, int64_t ld, const int32_t* __restrict__ row_pos, int ctx_len, int k,
     int32_t* __restrict__ idx) {
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t warp_sums[33];
-    __shared__ uint32_t s_digit, s_above;
-    const int t = blockIdx.x;
+    extern __shared__ uint8_t tk_smem_raw[];
+    // the runtime's placement of dynamic shared memory is not relied upon:
+    // the base is rounded up here (the launch reserves the slack)
+    uint32_t* tk_smem = (uint32_t*)(((uintptr_t)tk_smem_raw + 127) & ~(uintptr_t)127);
+    uint32_t* hist = tk_smem;                    // [NBINS]   this CTA's histogram
+    uint32_t* merged = hist + NBINS;             // [NBINS]   scratch for the suffix scan
+    uint32_t* cl_hist = merged + NBINS;          // [2][NBINS] cluster-wide histograms (rank 0 holds them)
+    uint32_t* warp_sums = cl_hist + 2 * NBINS;   // [33]
+    uint32_t* shared_res = warp_sums + 40;       // digit, count above
+    uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers)
+    uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
+
+    const int row = blockIdx.x / CL;
+    const uint32_t rank = cl_rank<CL>();
     const int tid = threadIdx.x;
-    const float* x = logits + (int64_t)t * ld;
-    int32_t* out = idx + (int64_t)t * k;
-    int n = row_pos[t] + 1;
+    const float* x = logits + (int64_t)row * ld;
+    int32_t* out = idx + (int64_t)row * k;
+    int n = row_pos[row] + 1;
     if (n > ctx_len) n = ctx_len;
     if (n < 0) n = 0;
 
-    if (n <= k) {                                   // keep-all rule
-        for (int i = tid; i < k; i += TOPK_THREADS) out[i] = i < n ? i : -1;
+    if (n <= k) {                                // keep-all rule (uniform over the cluster)
+        if (rank == 0)
+            for (int i = tid; i < k; i += TOPK_THREADS) out[i] = i < n ? i : -1;
         return;
     }
 
-    // ---- 1. radix select of the k-th largest key ----
-    uint32_t prefix = 0u, himask = 0u;
-    uint32_t remaining = (uint32_t)k;               // still to take among keys matching `prefix`
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += TOPK_THREADS) hist[i] = 0u;
-        __syncthreads();
-        for (int i = tid; i < n; i += TOPK_THREADS) {
-            uint32_t key = score_key(__ldg(x + i));
-            if (((key ^ prefix) & himask) == 0u) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    // ---- load this CTA's slice as order-preserving keys ----
+    const int per = ((n + CL - 1) / CL + 3) & ~3;
+    const int lo = min(n, (int)rank * per), hi = min(n, lo + per);
+    const int cnt = hi - lo;
+    // 8 independent 16-byte loads in flight per thread (one memory round trip
+    // for a 32K-key slice); scalar path for rows that are not 16-byte aligned
+    if ((((uintptr_t)(x + lo)) & 15u) == 0u) {
+        const float4* x4 = (const float4*)(x + lo);
+        const int n4 = cnt >> 2;
+        for (int i0 = tid; i0 < n4; i0 += 8 * TOPK_THREADS) {
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * TOPK_THREADS < n4) v[u] = __ldg(x4 + i0 + u * TOPK_THREADS);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * TOPK_THREADS < n4)
+                    *(uint4*)(keys + 4 * (i0 + u * TOPK_THREADS)) =
+                        make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w));
         }
-        __syncthreads();
-        if (tid < 32) {
-            const int lane = tid;
-            uint32_t h[8];
-            uint32_t mine = 0;
+        for (int i = 4 * n4 + tid; i < cnt; i += TOPK_THREADS) keys[i] = score_key(__ldg(x + lo + i));
+    } else {
+        for (int i0 = tid; i0 < cnt; i0 += 8 * TOPK_THREADS) {
+            float v[8];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) { h[b] = hist[lane * 8 + b]; mine += h[b]; }
-            // exclusive suffix sum over lanes: counts in bins above this lane's bins
-            uint32_t incl = mine;
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * TOPK_THREADS < cnt) v[u] = __ldg(x + lo + i0 + u * TOPK_THREADS);
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                uint32_t y = __shfl_down_sync(0xffffffffu, incl, o);
-                if (lane + o < 32) incl += y;
-            }
-            uint32_t cum = incl - mine;
-#pragma unroll
-            for (int b = 7; b >= 0; --b) {
-                if (cum < remaining && cum + h[b] >= remaining) { s_digit = (uint32_t)(lane * 8 + b); s_above = cum; }
-                cum += h[b];
-            }
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u * TOPK_THREADS < cnt) keys[i0 + u * TOPK_THREADS] = score_key(v[u]);
         }
-        __syncthreads();
-        prefix |= s_digit << shift;
-        himask |= 255u << shift;
-        remaining -= s_above;
-        __syncthreads();
     }
-    const uint32_t T = prefix;                      // the k-th largest key; `remaining` keys == T to take
+    if (CL > 1)
+        for (int i = tid; i < 2 * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
+    cl_sync<CL>();                               // cluster histograms are zero before anyone adds
+
+    // ---- 1. select the exact k-th largest key ----
+    // Adaptive range narrowing: the candidate keys lie in [lo, hi]; each pass
+    // buckets (key - lo) >> s into at most NBINS bins (s chosen from the
+    // range's width), finds the bucket that holds the remaining-th largest
+    // candidate and shrinks [lo, hi] to it.  Bucketing by the actual range
+    // spreads keys over the bins even when all scores share one exponent.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = tid; i < cnt; i += TOPK_THREADS) {
+        const uint32_t key = keys[i];
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    if ((tid & 31) == 0) {
+        merged[tid >> 5] = kmin;
+        merged[32 + (tid >> 5)] = kmax;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t a = 0xFFFFFFFFu, b = 0u;
+        for (int w2 = 0; w2 < TOPK_THREADS / 32; ++w2) {
+            a = min(a, merged[w2]);
+            b = max(b, merged[32 + w2]);
+        }
+        cta_counts[2] = a;
+        cta_counts[3] = b;
+    }
+    cl_sync<CL>();                               // every CTA's min / max published
+    if (tid == 0) {
+        uint32_t a = 0xFFFFFFFFu, b = 0u;
+        for (int r = 0; r < CL; ++r) {
+            const uint32_t base = CL > 1 ? mapa_shared(smem_u32(cta_counts), (uint32_t)r) : smem_u32(cta_counts);
+            a = min(a, CL > 1 ? ld_cluster_u32(base + 8) : cta_counts[2]);
+            b = max(b, CL > 1 ? ld_cluster_u32(base + 12) : cta_counts[3]);
+        }
+        shared_res[4] = a;
+        shared_res[5] = b;
+    }
+    __syncthreads();
+    uint32_t lo_key = shared_res[4], hi_key = shared_res[5], remaining = (uint32_t)k;
+#pragma unroll 1
+    for (int pass = 0; pass < 4 && lo_key != hi_key; ++pass) {
+        const uint32_t width = hi_key - lo_key;
+        const int s_bits = 32 - __clz(width) - 11;        // (width >> s) < NBINS
+        const int sh = s_bits > 0 ? s_bits : 0;
+        for (int i = tid; i < NBINS; i += TOPK_THREADS) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < cnt; i += TOPK_THREADS) {
+            const uint32_t key = keys[i];
+            if (key >= lo_key && key <= hi_key) atomicAdd(&hist[(key - lo_key) >> sh], 1u);
+        }
+        __syncthreads();
+        // cluster-wide histogram: thread t owns bins 2t and 2t+1
+        uint32_t h0, h1;
+        if (CL > 1) {
+            const int buf = pass & 1;            // rank 0 zeroes a buffer after it has been read
+            const uint32_t lead = mapa_shared(smem_u32(cl_hist + buf * NBINS + 2 * tid), 0u);
+            if (hist[2 * tid]) red_cluster_add(lead, hist[2 * tid]);
+            if (hist[2 * tid + 1]) red_cluster_add(lead + 4, hist[2 * tid + 1]);
+            cl_sync<CL>();                       // all additions landed
+            const uint2 v = ld_cluster_v2(lead);
+            h0 = v.x;
+            h1 = v.y;
+        } else {
+            h0 = hist[2 * tid];
+            h1 = hist[2 * tid + 1];
+        }
+        // keys in bins above each thread's pair: scan over reversed thread order
+        uint32_t tot;
+        merged[TOPK_THREADS - 1 - tid] = h0 + h1;
+        __syncthreads();
+        const uint32_t rev = merged[tid];
+        __syncthreads();
+        const uint32_t above_rev = block_excl_scan(rev, warp_sums, &tot);
+        merged[TOPK_THREADS - 1 - tid] = above_rev;
+        __syncthreads();
+        const uint32_t above = merged[tid];
+        if (above < remaining && above + h1 >= remaining) {
+            shared_res[0] = 2u * tid + 1u;
+            shared_res[1] = above;
+        } else if (above + h1 < remaining && above + h1 + h0 >= remaining) {
+            shared_res[0] = 2u * tid;
+            shared_res[1] = above + h1;
+        }
+        __syncthreads();
+        const uint32_t bin = shared_res[0];
+        remaining -= shared_res[1];
+        const uint32_t new_lo = lo_key + (bin << sh);
+        const uint32_t span = sh == 0 ? 0u : ((1u << sh) - 1u);
+        hi_key = (hi_key - new_lo > span) ? new_lo + span : hi_key;
+        lo_key = new_lo;
+        if (CL > 1) {
+            cl_sync<CL>();                       // everyone has read this pass's cluster histogram
+            if (rank == 0)
+                for (int i = tid; i < NBINS; i += TOPK_THREADS) cl_hist[(pass & 1) * NBINS + i] = 0u;
+        } else {
+            __syncthreads();
+        }
+    }
+    const uint32_t T = lo_key;                   // the k-th largest key; `remaining` keys == T to take
 
     // ---- 2. ordered compaction ----
-    const int seg = (n + TOPK_THREADS - 1) / TOPK_THREADS;
-    const int lo = min(n, tid * seg), hi = min(n, lo + seg);
-    uint32_t gt = 0, eq = 0;
-    for (int i = lo; i < hi; ++i) {
-        uint32_t key = score_key(__ldg(x + i));
-        gt += key > T;
-        eq += key == T;
+    // Warp w owns a contiguous run of the slice and walks it 32 keys at a
+    // time (consecutive lanes on consecutive keys: no bank conflicts,
+    // coalesced index writes); ballots give each selected key its rank.
+    const int warp = tid >> 5, lane = tid & 31;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const int chunk = (((cnt + 31) / 32) + 31) / 32 * 32;           // keys per warp, multiple of 32
+    const int wlo = min(cnt, warp * chunk), whi = min(cnt, wlo + chunk);
+    uint32_t gt_w = 0, eq_w = 0;
+    for (int base = wlo; base < whi; base += 32) {
+        const int i = base + lane;
+        const uint32_t key = i < whi ? keys[i] : 0u;
+        gt_w += __popc(__ballot_sync(0xffffffffu, i < whi && key > T));
+        eq_w += __popc(__ballot_sync(0xffffffffu, i < whi && key == T));
     }
-    uint32_t tot;
-    const uint32_t eq_before = block_excl_scan(eq, warp_sums, &tot);
-    const uint32_t take_eq = eq_before >= remaining ? 0u : min(eq, remaining - eq_before);
-    const uint32_t off = block_excl_scan(gt + take_eq, warp_sums, &tot);
-    uint32_t j = off, e = 0;
-    for (int i = lo; i < hi; ++i) {
-        uint32_t key = score_key(__ldg(x + i));
-        if (key > T) {
-            out[j++] = i;
-        } else if (key == T) {
-            if (e < take_eq) out[j++] = i;
-            ++e;
+    uint32_t* wgt = merged;                      // per-warp counts and offsets (scratch)
+    uint32_t* weq = merged + 32;
+    uint32_t* wout = merged + 64;
+    uint32_t* wtake = merged + 96;
+    if (lane == 0) {
+        wgt[warp] = gt_w;
+        weq[warp] = eq_w;
+    }
+    __syncthreads();
+    // CTA totals, and the counts of the cluster's lower-ranked CTAs
+    uint32_t eq_before_cta = 0, out_before_cta = 0;
+    if (CL > 1) {
+        if (warp == 0) {
+            uint32_t g = wgt[lane], e = weq[lane];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                g += __shfl_xor_sync(0xffffffffu, g, o);
+                e += __shfl_xor_sync(0xffffffffu, e, o);
+            }
+            if (lane == 0) {
+                cta_counts[0] = g;
+                cta_counts[1] = e;
+            }
         }
+        cl_sync<CL>();
+        if (tid == 0) {
+            uint32_t eqb = 0, outb = 0;
+            for (uint32_t r = 0; r < rank; ++r) {
+                const uint32_t base = mapa_shared(smem_u32(cta_counts), r);
+                const uint32_t g = ld_cluster_u32(base), e = ld_cluster_u32(base + 4);
+                const uint32_t take = eqb >= remaining ? 0u : min(e, remaining - eqb);
+                outb += g + take;
+                eqb += e;
+            }
+            shared_res[2] = eqb;
+            shared_res[3] = outb;
+        }
+        __syncthreads();
+        eq_before_cta = shared_res[2];
+        out_before_cta = shared_res[3];
     }
+    if (warp == 0) {
+        // exclusive scans over the 32 warps (in position order)
+        const uint32_t e = weq[lane], g = wgt[lane];
+        uint32_t eq_incl = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, eq_incl, o);
+            if (lane >= o) eq_incl += y;
+        }
+        const uint32_t eqb = eq_before_cta + eq_incl - e;
+        const uint32_t take = eqb >= remaining ? 0u : min(e, remaining - eqb);
+        const uint32_t sel = g + take;
+        uint32_t sel_incl = sel;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, sel_incl, o);
+            if (lane >= o) sel_incl += y;
+        }
+        wout[lane] = out_before_cta + sel_incl - sel;
+        wtake[lane] = take;
+    }
+    __syncthreads();
+    uint32_t j = wout[warp], eq_seen = 0;
+    const uint32_t take = wtake[warp];
+    for (int base = wlo; base < whi; base += 32) {
+        const int i = base + lane;
+        const bool ok = i < whi;
+        const uint32_t key = ok ? keys[i] : 0u;
+        const bool is_gt = ok && key > T, is_eq = ok && key == T;
+        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+        const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < take);
+        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[j + __popc(selm & lt_mask)] = lo + i;
+        j += __popc(selm);
+        eq_seen += __popc(eqm);
+    }
+    if (CL > 1) cl_sync<CL>();                   // peers are done reading our counts
 }
+
+namespace {
+
+// Smallest cluster whose CTAs can hold a row in shared memory: a row that
+// fits one SM is selected by one CTA (no cross-CTA traffic at all).
+int choose_cluster(int /*rows*/, int ctx_len) {
+    const int need = (ctx_len + SLICE_CAP - 1) / SLICE_CAP;
+    int cl = 1;
+    while (cl < need && cl < 8) cl <<= 1;
+    return cl;
+}
+
+template <int CL>
+cudaError_t launch_cl(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows, int ctx_len,
+                      int k, int32_t* idx) {
+    const int per = ((ctx_len + CL - 1) / CL + 3) & ~3;
+    const size_t smem = 128 + SMEM_FIXED + (size_t)per * 4;
+    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)rows * CL);
+    cfg.blockDim = dim3(TOPK_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<CL>, logits, ld, row_pos, ctx_len, k, idx);
+    count_launch();
+    return e;
+}
+
+}  // namespace
+
+bool topk_supported(int ctx_len) { return ctx_len <= 8 * SLICE_CAP; }
 
 cudaError_t launch_topk(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows,
                         int ctx_len, int k, int32_t* idx, void* /*workspace*/, size_t /*ws_bytes*/) {
     if (rows == 0) return cudaSuccess;
-    topk_radix_kernel<<<rows, TOPK_THREADS, 0, L.stream>>>(logits, ld, row_pos, ctx_len, k, idx);
-    count_launch();
-    return cudaGetLastError();
+    switch (choose_cluster(rows, ctx_len)) {
+    case 1: return launch_cl<1>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    case 2: return launch_cl<2>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    case 4: return launch_cl<4>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    default: return launch_cl<8>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    }
 }
 
 size_t topk_workspace_bytes(int /*rows*/, int /*ctx_len*/, int /*k*/) { return 0; }
