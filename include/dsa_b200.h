@@ -154,9 +154,12 @@ DSA_API size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d
  *
  *   q          [rows, n_heads, d_qk] of dtype (DSA_BF16 or DSA_FP32)
  *   kv         contiguous cache [batch, ctx_len, d_qk] when page_table is NULL;
- *              paged cache [n_pages, page_size, d_qk] otherwise, with
+ *              paged cache [num_pages, page_size, d_qk] otherwise, with
  *              c_s = kv[page_table[b, s / page_size], s % page_size, :]
- *   page_table [batch, ctx_len / page_size] int32 physical page ids, or NULL
+ *   page_table [batch, ctx_len / page_size] int32 physical page ids in
+ *              [0, num_pages), or NULL (then page_size and num_pages are ignored);
+ *              an id outside the range is skipped and reported by
+ *              dsa_get_device_error
  *   row_batch  [rows] int32
  *   idx        [rows, k] int32 key positions in [0, ctx_len); -1 = unused
  *              slot (skipped).  Order within a row does not matter.
@@ -167,7 +170,7 @@ DSA_API size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d
  * d_qk, d_v <= 64 multiples of 32 in fp32 or bf16 with n_heads a multiple of 8.
  */
 DSA_API dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype,
-                            const int32_t* page_table, int page_size,
+                            const int32_t* page_table, int page_size, int num_pages,
                             const int32_t* row_batch, const int32_t* idx, int k,
                             int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
                             float scale, void* out, float* lse,

@@ -48,8 +48,8 @@ _SIGS = {
     "dsa_topk_workspace_size": (_sz, [_i32, _i32, _i32]),
     "dsa_topk": (_i32, [_vp, _i64, _vp, _i32, _i32, _i32, _vp, _vp, _sz, _vp]),
     "dsa_sparse_mla_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
-    "dsa_sparse_mla": (_i32, [_vp, _vp, _i32, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32,
-                              _vp, _vp, _vp, _sz, _vp]),
+    "dsa_sparse_mla": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                              _f32, _vp, _vp, _vp, _sz, _vp]),
     "dsa_get_device_error": (_i32, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -182,10 +182,10 @@ def sparse_mla(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: 
     k = idx.shape[1]
     if page_table is not None:
         B = page_table.shape[0]
-        page_size = kv.shape[1]
+        num_pages, page_size = kv.shape[0], kv.shape[1]
     else:
         B = kv.shape[0]
-        page_size = 0
+        num_pages, page_size = 0, 0
         if kv.shape[1] != ctx_len:
             raise ValueError("kv.shape[1] != ctx_len")
     if out is None:
@@ -197,7 +197,7 @@ def sparse_mla(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: 
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
-        _check(_lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, _ptr(row_batch),
+        _check(_lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages, _ptr(row_batch),
                                    _ptr(idx), k, rows, B, ctx_len, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
                                    _ptr(workspace), wsb, _stream(dev)), "dsa_sparse_mla")
     return out, lse

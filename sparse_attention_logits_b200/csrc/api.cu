@@ -152,7 +152,7 @@ size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int
 }
 
 dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
-                            int page_size, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                            int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
                             int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream) {
     if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 1 || n_heads <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk)
@@ -163,6 +163,7 @@ dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, co
     if (page_table) {
         if (page_size <= 0 || ctx_len % page_size)
             return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: ctx_len must be a multiple of page_size");
+        if (num_pages <= 0) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: num_pages must be positive with a page table");
     }
     if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: scale must be positive and finite");
     const bool tc = dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v);
@@ -177,11 +178,11 @@ dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, co
         const size_t need = dsa::mla_tc_workspace_bytes(rows, k, L.num_sms);
         if (need && (!workspace || workspace_bytes < need))
             return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: workspace of %zu bytes needed", need);
-        return cuda_status(dsa::launch_mla_tc(L, q, kv, page_table, page_size, row_batch, idx, k, rows, batch,
-                                              ctx_len, scale, out, lse, workspace, workspace_bytes),
+        return cuda_status(dsa::launch_mla_tc(L, q, kv, page_table, page_size, num_pages, row_batch, idx, k, rows,
+                                              batch, ctx_len, scale, out, lse, workspace, workspace_bytes),
                            "dsa_sparse_mla (tensor-core) launch");
     }
-    return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, row_batch, idx, k, rows, batch,
+    return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows, batch,
                                             ctx_len, n_heads, d_qk, d_v, scale, out, lse),
                        "dsa_sparse_mla launch");
 }

@@ -26,14 +26,15 @@ bool topk_supported(int ctx_len);
 
 bool mla_simt_supported(int d_qk, int d_v, int n_heads);
 cudaError_t launch_mla_simt(const Launch& L, const void* q, const void* kv, dsa_dtype_t dtype,
-                            const int32_t* page_table, int page_size, const int32_t* row_batch, const int32_t* idx,
+                            const int32_t* page_table, int page_size, int num_pages, const int32_t* row_batch,
+                            const int32_t* idx,
                             int k, int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v, float scale,
                             void* out, float* lse);
 
 bool mla_tc_supported(dsa_dtype_t dtype, int n_heads, int d_qk, int d_v);
 size_t mla_tc_workspace_bytes(int rows, int k, int num_sms);
 cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
-                          const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch, int ctx_len,
-                          float scale, void* out, float* lse, void* workspace, size_t ws_bytes);
+                          int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                          int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes);
 
 }  // namespace dsa

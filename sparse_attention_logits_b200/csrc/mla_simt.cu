@@ -22,7 +22,7 @@ constexpr float LN2 = 0.6931471805599453f;
 template <typename T, int QPL, int VPL>
 __global__ void __launch_bounds__(256) mla_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ kv, const int32_t* __restrict__ page_table, int page_size,
-    int pages_per_seq, const int32_t* __restrict__ row_batch, const int32_t* __restrict__ idx, int k,
+    int pages_per_seq, int num_pages, const int32_t* __restrict__ row_batch, const int32_t* __restrict__ idx, int k,
     int batch, int ctx_len, int n_heads, float scale, T* __restrict__ out, float* __restrict__ lse, unsigned* err) {
     constexpr int DK = QPL * 32, DV = VPL * 32;
     __shared__ float tile[MLA_SIMT_TILE][DK];
@@ -55,9 +55,16 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
             bool ok = row_ok && s >= 0 && s < ctx_len;
             if (s >= ctx_len) record_error(err, DEV_ERR_BAD_INDEX);
             int64_t row = 0;
-            if (ok) {
-                row = page_table ? (int64_t)page_table[(int64_t)b * pages_per_seq + s / page_size] * page_size + s % page_size
-                                 : (int64_t)b * ctx_len + s;
+            if (ok && page_table) {
+                const int pg = page_table[(int64_t)b * pages_per_seq + s / page_size];
+                if (pg < 0 || pg >= num_pages) {
+                    record_error(err, DEV_ERR_BAD_INDEX);
+                    ok = false;
+                } else {
+                    row = (int64_t)pg * page_size + s % page_size;
+                }
+            } else if (ok) {
+                row = (int64_t)b * ctx_len + s;
             }
             for (int d = lane; d < DK; d += 32) tile[r][d] = ok ? to_f32(kv[row * DK + d]) : 0.f;
             if (lane == 0) valid[r] = ok;
@@ -89,10 +96,10 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
 
 template <typename T, int QPL, int VPL>
 static cudaError_t launch_t(const Launch& L, const void* q, const void* kv, const int32_t* pt, int page_size,
-                            int pages_per_seq, const int32_t* rb, const int32_t* idx, int k, int rows, int batch,
+                            int pages_per_seq, int num_pages, const int32_t* rb, const int32_t* idx, int k, int rows, int batch,
                             int ctx, int H, float scale, void* out, float* lse) {
     dim3 grid(rows, H / MLA_SIMT_HEADS);
-    mla_simt_kernel<T, QPL, VPL><<<grid, 256, 0, L.stream>>>((const T*)q, (const T*)kv, pt, page_size, pages_per_seq,
+    mla_simt_kernel<T, QPL, VPL><<<grid, 256, 0, L.stream>>>((const T*)q, (const T*)kv, pt, page_size, pages_per_seq, num_pages,
                                                              rb, idx, k, batch, ctx, H, scale, (T*)out, lse, L.err);
     count_launch();
     return cudaGetLastError();
@@ -100,12 +107,12 @@ static cudaError_t launch_t(const Launch& L, const void* q, const void* kv, cons
 
 template <typename T>
 static cudaError_t launch_dims(const Launch& L, const void* q, const void* kv, const int32_t* pt, int page_size,
-                               int pps, const int32_t* rb, const int32_t* idx, int k, int rows, int batch, int ctx,
+                               int pps, int npages, const int32_t* rb, const int32_t* idx, int k, int rows, int batch, int ctx,
                                int H, int dqk, int dv, float scale, void* out, float* lse) {
-    if (dqk == 32 && dv == 32) return launch_t<T, 1, 1>(L, q, kv, pt, page_size, pps, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 64 && dv == 64) return launch_t<T, 2, 2>(L, q, kv, pt, page_size, pps, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 64 && dv == 32) return launch_t<T, 2, 1>(L, q, kv, pt, page_size, pps, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 576 && dv == 512) return launch_t<T, 18, 16>(L, q, kv, pt, page_size, pps, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
+    if (dqk == 32 && dv == 32) return launch_t<T, 1, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
+    if (dqk == 64 && dv == 64) return launch_t<T, 2, 2>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
+    if (dqk == 64 && dv == 32) return launch_t<T, 2, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
+    if (dqk == 576 && dv == 512) return launch_t<T, 18, 16>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
     return cudaErrorInvalidValue;
 }
 
@@ -115,14 +122,14 @@ bool mla_simt_supported(int d_qk, int d_v, int n_heads) {
 }
 
 cudaError_t launch_mla_simt(const Launch& L, const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
-                            int page_size, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                            int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
                             int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse) {
     if (rows == 0) return cudaSuccess;
     const int pps = page_table ? ctx_len / page_size : 0;
     if (dtype == DSA_FP32)
-        return launch_dims<float>(L, q, kv, page_table, page_size, pps, row_batch, idx, k, rows, batch, ctx_len,
+        return launch_dims<float>(L, q, kv, page_table, page_size, pps, num_pages, row_batch, idx, k, rows, batch, ctx_len,
                                   n_heads, d_qk, d_v, scale, out, lse);
-    return launch_dims<__nv_bfloat16>(L, q, kv, page_table, page_size, pps, row_batch, idx, k, rows, batch,
+    return launch_dims<__nv_bfloat16>(L, q, kv, page_table, page_size, pps, num_pages, row_batch, idx, k, rows, batch,
                                       ctx_len, n_heads, d_qk, d_v, scale, out, lse);
 }
 

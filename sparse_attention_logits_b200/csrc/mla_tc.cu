@@ -28,9 +28,14 @@
 //                       over several clusters, normalised fp32 partials that
 //                       dsa_mla_combine merges.
 //
-// Warps (both CTAs): 0-7 gather producers, 8-11 softmax (score CTA) or
-// rescale + epilogue (value CTA), one thread per head / TMEM lane, 12 MMA
-// issuer and TMEM owner.  Every wait is bounded; the two CTAs only exchange
+// The selected rows are gathered by TMA (tile::gather4, 4 rows per
+// instruction) one 8 KB dim block (64 rows x 64 dims) at a time; a block is
+// refilled for chunk c+2 as soon as the MMA of chunk c is done with it, and
+// the MMA of a chunk starts on its first block.
+//
+// Warps (both CTAs): 0 TMA gather producer (1-3 spare); 4-11 softmax (score
+// CTA: two threads per head, 32 keys each) or 4-7 rescale + epilogue (value
+// CTA, one thread per head / TMEM lane); 12 MMA issuer and TMEM owner.  Every wait is bounded; the two CTAs only exchange
 // data through bulk copies and mbarrier arrivals that the receiver waits on.
 #include "common.cuh"
 #include "launchers.h"
@@ -46,15 +51,15 @@ constexpr int H = 128;              // query heads = MMA M
 constexpr int DK = 576;             // latent + rope
 constexpr int DV = 512;             // value dims
 constexpr int NK = 64;              // keys per chunk
-constexpr int PWARPS = 8;           // gather producer warps (each keeps its own copies in flight)
-constexpr int ROWS_PER_PW = NK / PWARPS;
-constexpr int SWARP0 = PWARPS;      // first of the 4 softmax / rescale-epilogue warps
-constexpr int MWARP = PWARPS + 4;   // MMA issuer, TMEM owner
-constexpr int THREADS = 32 * (PWARPS + 5);
+constexpr int PWARPS = 4;           // warp 0 issues the TMA row gathers; warps 1-3 are spare
+constexpr int SWARP0 = PWARPS;      // first of the 8 softmax warps (score CTA) / 4 rescale-epilogue warps (value CTA)
+constexpr int MWARP = PWARPS + 8;   // MMA issuer, TMEM owner
+constexpr int THREADS = 32 * (PWARPS + 9);
+constexpr int KBLK = DK / 64;       // 9 dim blocks of 64 (128 B per row) per gathered row
+constexpr int VBLK = DV / 64;       // the value CTA gathers the first 8
 constexpr int KSTAGE = NK * DK * 2; // 73728 B
-constexpr int VSTAGE = NK * DV * 2; // 65536 B
 constexpr int STAGES = 2;
-constexpr int REGION = (STAGES * KSTAGE > STAGES * VSTAGE) ? STAGES * KSTAGE : STAGES * VSTAGE;
+constexpr int REGION = STAGES * KSTAGE;  // [stage][dim block][64 rows x 128 B]
 constexpr int PBYTES = H * NK * 2;  // 16384: P [128 heads x 64 keys] bf16
 constexpr int PSLOTS = 4;           // P ring depth (score CTA may run this many chunks ahead)
 constexpr int ABYTES = H * 4;       // rescale factor per head
@@ -65,8 +70,11 @@ constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between 
 constexpr float LN2 = 0.6931471805599453f;
 
 struct Bars {                       // same offset in both CTAs of a cluster
-    uint64_t kfull[2], kempty[2], sfull[2], sempty[2], pready[PSLOTS], pempty[PSLOTS], qready, statready, statack;
-    uint64_t vfull[2], vempty[2], pfull[PSLOTS], ready[PSLOTS], odone, statfull;
+    uint64_t bfull[2][KBLK];        // a dim block of a stage has landed (cp.async arrivals)
+    uint64_t bempty[2][KBLK];       // the MMA is done reading a dim block of a stage
+    uint64_t sfull[2], sempty[2], pready[PSLOTS], pempty[PSLOTS], qready, statready, statack;
+    uint64_t pfull[PSLOTS], ready[PSLOTS], odone, statfull;
+    uint64_t mx[4];                 // score CTA: the two softmax warps of a lane quarter exchange maxima
     uint32_t tmem;
     int abort;
 };
@@ -82,7 +90,7 @@ struct MlaParams {
     float* part_o;                  // [rows, splits, H, DV] when splits > 1
     float* part_lse;                // [rows, splits, H]
     unsigned* err;
-    int page_size, pages_per_seq;
+    int page_size, pages_per_seq, num_pages;
     int k, rows, batch, ctx, splits, per_split;
     float scale_log2;
 };
@@ -116,6 +124,10 @@ __device__ __forceinline__ int64_t key_row(const MlaParams& p, const Work& w, in
     }
     if (p.page_table) {
         const int pg = __ldg(p.page_table + (int64_t)w.b * p.pages_per_seq + s / p.page_size);
+        if (pg < 0 || pg >= p.num_pages) {
+            record_error(p.err, DEV_ERR_BAD_INDEX);
+            return -1;
+        }
         return (int64_t)pg * p.page_size + s % p.page_size;
     }
     return (int64_t)w.b * p.ctx + s;
@@ -137,41 +149,50 @@ __device__ __forceinline__ int slot_index(const MlaParams& p, const Work& w, int
 // Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-template <int RC>   // 16-byte pieces per gathered row
-__device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, int stage_bytes,
-                                            uint64_t* full, uint64_t* empty, int warp, int lane,
-                                            volatile int* abort_flag) {
-    const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
-    int64_t next_row = key_row(p, w, w.slot0 + my_slot);
-    for (int c = 0; c < w.nchunks; ++c) {
-        const int st = c & 1;
-        if (!mbar_wait(&empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
-        const int myrow_lo = (int)(next_row >= 0 ? next_row : -1);  // row indices fit in 31 bits
-        uint8_t* base = gbuf + (size_t)st * stage_bytes;
-#pragma unroll 4
-        for (int i = lane; i < ROWS_PER_PW * RC; i += 32) {
-            const int rl = i / RC, ci = i - rl * RC;
-            const int row = __shfl_sync(0xffffffffu, myrow_lo, rl);
-            const int r = warp * ROWS_PER_PW + rl;
-            const __nv_bfloat16* src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8 : p.kv;
-            cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
+// Gather of the selected rows with TMA row gathers (tile::gather4), one 8 KB
+// dim block (64 rows x 64 dims) at a time: lane g of the producer warp owns
+// rows 4g..4g+3 of every chunk and issues one 4-row gather per dim block,
+// which lands in the 128-B-swizzled layout the MMA reads.  A block of stage
+// st is refilled as soon as the MMA has finished reading it; unused slots
+// gather row -1, which the TMA fills with zeros.
+template <int NB>   // dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
+__device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, const CUtensorMap* map, uint8_t* gbuf,
+                                            Bars* bars, int lane, volatile int* abort_flag) {
+    const int g = lane & 15;
+    int nrow[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) nrow[q] = (int)key_row(p, w, w.slot0 + 4 * g + q);   // rows fit in 31 bits
+    bool ok = true;
+    for (int c = 0; c < w.nchunks && ok; ++c) {
+        const int st = c & 1, par = ((c >> 1) & 1) ^ 1;
+        const int r0 = nrow[0], r1 = nrow[1], r2 = nrow[2], r3 = nrow[3];
+        uint8_t* base = gbuf + (size_t)st * KSTAGE;
+        for (int b = 0; b < NB; ++b) {
+            if (!mbar_wait(&bars->bempty[st][b], par, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) { ok = false; break; }
+            if (lane == 0) mbar_arrive_expect_tx(&bars->bfull[st][b], NK * 128);
+            __syncwarp();
+            if (lane < 16) tma_gather4(base + b * (NK * 128) + g * 512, map, b * 64, r0, r1, r2, r3, &bars->bfull[st][b]);
         }
-        cp_async_arrive_noinc(&full[st]);
-        // look up the next chunk's row while this chunk's copies are in flight
-        if (c + 1 < w.nchunks) next_row = key_row(p, w, w.slot0 + (c + 1) * NK + my_slot);
+        // look up the next chunk's rows while this chunk's gathers are in flight
+        if (c + 1 < w.nchunks) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) nrow[q] = (int)key_row(p, w, w.slot0 + (c + 1) * NK + 4 * g + q);
+        }
     }
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
+__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map,
+                                                          const MlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
     uint8_t* pbuf = gbuf + REGION;                          // [PSLOTS][PBYTES]
     float* abuf = (float*)(pbuf + PSLOTS * PBYTES);         // [PSLOTS][H]
     float* sbuf = abuf + PSLOTS * H;                        // [2*H]: running max, running sum
-    Bars* bars = (Bars*)(sbuf + 2 * H);
+    float* xbuf = sbuf + 2 * H;                             // [2][2][H]: partial maxima / sums of the two halves
+    Bars* bars = (Bars*)(xbuf + 4 * H);
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,25 +201,27 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars->kfull[i], PWARPS * 32);
-            mbar_init(&bars->kempty[i], 1);
+            for (int b = 0; b < KBLK; ++b) {
+                mbar_init(&bars->bfull[i][b], 1);
+                mbar_init(&bars->bempty[i][b], 1);
+            }
             mbar_init(&bars->sfull[i], 1);
-            mbar_init(&bars->sempty[i], 4);
-            mbar_init(&bars->vfull[i], PWARPS * 32);
-            mbar_init(&bars->vempty[i], 1);
+            mbar_init(&bars->sempty[i], 8);
         }
         for (int i = 0; i < PSLOTS; ++i) {
-            mbar_init(&bars->pready[i], 4);
+            mbar_init(&bars->pready[i], 8);
             mbar_init(&bars->pempty[i], 1);
             mbar_init(&bars->pfull[i], 1);
             mbar_init(&bars->ready[i], 4);
         }
-        mbar_init(&bars->qready, 4);
-        mbar_init(&bars->statready, 4);
+        mbar_init(&bars->qready, 8);
+        mbar_init(&bars->statready, 8);
+        for (int i = 0; i < 4; ++i) mbar_init(&bars->mx[i], 2);
         mbar_init(&bars->statack, 4);
         mbar_init(&bars->odone, 1);
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
+        tma_prefetch_desc(&kv_map);
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
         if (rank == 1) {
             // arm the first phase of each P slot and the final-statistics slot
@@ -218,34 +241,44 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
     const uint32_t peer = rank ^ 1u;
 
     if (warp < PWARPS) {
-        // ------------------------------------------------ gather producers ----
+        // ------------------------------------------------- gather producer ----
         // Warp w owns rows [8w, 8w+8) of every chunk: lane l resolves one of
         // them once per chunk (one index load per lane, all in flight
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (rank == 0) gather_rows<DK / 8>(p, w, gbuf, KSTAGE, bars->kfull, bars->kempty, warp, lane, abort_flag);
-        else gather_rows<DV / 8>(p, w, gbuf, VSTAGE, bars->vfull, bars->vempty, warp, lane, abort_flag);
-    } else if (warp < SWARP0 + 4 && rank == 0) {
+        if (warp == 0) {
+            if (rank == 0) gather_rows<KBLK>(p, w, &kv_map, gbuf, bars, lane, abort_flag);
+            else gather_rows<VBLK>(p, w, &kv_map, gbuf, bars, lane, abort_flag);
+        }
+    } else if (warp < SWARP0 + 8 && rank == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
-        const int h = (warp - SWARP0) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)((warp - SWARP0) * 32) << 16;
-        {   // Q row of head h -> TMEM lane h, columns [0, 288) (bf16 pairs)
-            const uint4* qrow = (const uint4*)(p.q + ((int64_t)w.t * H + h) * DK);
+        // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
+        // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
+        // of every chunk; the two halves of a head exchange their partial
+        // maxima each chunk, so both take the same rescaling decision.
+        const int sw = warp - SWARP0, half = sw >> 2, quarter = sw & 3;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        {   // Q row of head h -> TMEM lane h; this half writes columns [144*half, 144*half + 144)
+            const uint4* qrow = (const uint4*)(p.q + ((int64_t)w.t * H + h) * DK) + half * 36;
 #pragma unroll 1
-            for (int m0 = 0; m0 < DK / 32; m0 += 6) {          // 3 batches, 24 loads in flight each
-                uint4 x[24];
+            for (int m0 = 0; m0 < 9; m0 += 5) {                 // 16-column groups, loads batched
+                uint4 x[20];
 #pragma unroll
-                for (int v = 0; v < 24; ++v) x[v] = __ldg(qrow + m0 * 4 + v);
+                for (int v = 0; v < 20; ++v)
+                    if (m0 * 4 + v < 36) x[v] = __ldg(qrow + m0 * 4 + v);
 #pragma unroll
-                for (int m = 0; m < 6; ++m) {
-                    uint32_t words[16];
+                for (int m = 0; m < 5; ++m) {
+                    if (m0 + m < 9) {
+                        uint32_t words[16];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        words[4 * v] = x[4 * m + v].x; words[4 * v + 1] = x[4 * m + v].y;
-                        words[4 * v + 2] = x[4 * m + v].z; words[4 * v + 3] = x[4 * m + v].w;
+                        for (int v = 0; v < 4; ++v) {
+                            words[4 * v] = x[4 * m + v].x; words[4 * v + 1] = x[4 * m + v].y;
+                            words[4 * v + 2] = x[4 * m + v].z; words[4 * v + 3] = x[4 * m + v].w;
+                        }
+                        tmem_st16(tmem + lane_base + half * 144 + (m0 + m) * 16, words);
                     }
-                    tmem_st16(tmem + lane_base + (m0 + m) * 16, words);
                 }
             }
             tmem_st_wait();
@@ -253,44 +286,42 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->qready);
         }
-        float m_run = -INFINITY, l_run = 0.f;
+        float m_run = -INFINITY, l_run = 0.f;                   // l_run: this half's keys
         const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
         bool ok = true;
-        // which of the 64 keys of a chunk are real: the raw indices are loaded
+        // whether this lane's key of a chunk is real: the raw index is loaded
         // one chunk ahead and only inspected in the next iteration
-        int sa_next = slot_index(p, w, w.slot0 + lane), sb_next = slot_index(p, w, w.slot0 + 32 + lane);
+        int s_next = slot_index(p, w, w.slot0 + 32 * half + lane);
         for (int c = 0; c < w.nchunks && ok; ++c) {
             const int sb = c & 1;
-            const uint32_t mlo = __ballot_sync(0xffffffffu, w.b_ok && sa_next >= 0 && sa_next < p.ctx);
-            const uint32_t mhi = __ballot_sync(0xffffffffu, w.b_ok && sb_next >= 0 && sb_next < p.ctx);
-            if (c + 1 < w.nchunks) {
-                sa_next = slot_index(p, w, w.slot0 + (c + 1) * NK + lane);
-                sb_next = slot_index(p, w, w.slot0 + (c + 1) * NK + 32 + lane);
-            }
+            const uint32_t vmask = __ballot_sync(0xffffffffu, w.b_ok && s_next >= 0 && s_next < p.ctx);
+            if (c + 1 < w.nchunks) s_next = slot_index(p, w, w.slot0 + (c + 1) * NK + 32 * half + lane);
             ok = mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
             if (!ok) break;
             tc_fence_after();
-            float s0[32], s1[32];
-            tmem_ld32(tmem + lane_base + S_COL + sb * NK, s0);
-            tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32, s1);
+            float sv[32];
+            tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32 * half, sv);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->sempty[sb]);
             float mx[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                s0[j] = ((mlo >> j) & 1u) ? s0[j] * p.scale_log2 : -INFINITY;
-                s1[j] = ((mhi >> j) & 1u) ? s1[j] * p.scale_log2 : -INFINITY;
-            }
+            for (int j = 0; j < 32; ++j) sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(fmaxf(s0[2 * j], s0[2 * j + 1]), fmaxf(s1[2 * j], s1[2 * j + 1]));
+            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(sv[2 * j], sv[2 * j + 1]);
 #pragma unroll
             for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
                 for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-            const float mc = mx[0];
+            float* xb = xbuf + (c & 1) * 2 * H;
+            xb[half * H + h] = mx[0];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->mx[quarter]);
+            ok = mbar_wait(&bars->mx[quarter], c & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (!ok) break;
+            const float mc = fmaxf(mx[0], xb[(half ^ 1) * H + h]);
             float alpha = 1.f;
             if (mc > -INFINITY) {
                 if (m_run == -INFINITY) {
@@ -301,21 +332,21 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                     m_run = mc;
                 }
             }
-            uint32_t pk[32];
-            float ls[16];
-            // exp2 of (score - running max): arguments are <= 2^3 above 0 at most
-            // (lazy rescale) and -inf for unused keys, which ex2 maps to +0.
+            uint32_t pk[16];
+            float ls[8];
+            // exp2 of (score - running max): at most 2^8 (lazy rescale); -inf for
+            // unused keys, which ex2 maps to +0
             const float mr = m_run == -INFINITY ? 0.f : m_run;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const __nv_bfloat162 pa = __floats2bfloat162_rn(fast_exp2(s0[2 * j] - mr), fast_exp2(s0[2 * j + 1] - mr));
-                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(fast_exp2(s1[2 * j] - mr), fast_exp2(s1[2 * j + 1] - mr));
+            for (int j = 0; j < 8; ++j) {
+                const __nv_bfloat162 pa = __floats2bfloat162_rn(fast_exp2(sv[4 * j] - mr), fast_exp2(sv[4 * j + 1] - mr));
+                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(fast_exp2(sv[4 * j + 2] - mr), fast_exp2(sv[4 * j + 3] - mr));
                 ls[j] = (__low2float(pa) + __high2float(pa)) + (__low2float(pb2) + __high2float(pb2));
-                pk[j] = *(const uint32_t*)&pa;
-                pk[16 + j] = *(const uint32_t*)&pb2;
+                pk[2 * j] = *(const uint32_t*)&pa;
+                pk[2 * j + 1] = *(const uint32_t*)&pb2;
             }
 #pragma unroll
-            for (int w2 = 8; w2 >= 1; w2 >>= 1)
+            for (int w2 = 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
                 for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
             l_run += ls[0];
@@ -324,9 +355,10 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             if (!ok) break;
             uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *(uint4*)(prow + sw128(h & 7, j)) = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-            abuf[pb * H + h] = alpha;
+            for (int jj = 0; jj < 4; ++jj)
+                *(uint4*)(prow + sw128(h & 7, 4 * half + jj)) =
+                    make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+            if (half == 0) abuf[pb * H + h] = alpha;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->pready[pb]);
@@ -340,9 +372,20 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
         }
-        // final statistics -> value CTA
-        sbuf[h] = m_run;
-        sbuf[H + h] = l_run;
+        // final statistics -> value CTA: running max (same in both halves) and
+        // the sum of the two halves' running sums
+        if (ok) {
+            const int c = w.nchunks;
+            float* xb = xbuf + (c & 1) * 2 * H;
+            xb[half * H + h] = l_run;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->mx[quarter]);
+            ok = mbar_wait(&bars->mx[quarter], c & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (ok && half == 0) {
+                sbuf[h] = m_run;
+                sbuf[H + h] = l_run + xb[H + h];
+            }
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->statready);
@@ -441,42 +484,49 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 bool ok = mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 tc_fence_after();
                 for (int c = 0; c < w.nchunks && ok; ++c) {
-                    const int st = c & 1, sb = c & 1;
-                    ok = mbar_wait(&bars->kfull[st], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
-                         mbar_wait(&bars->sempty[sb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-                    if (!ok) break;
-                    fence_proxy_async_smem();
-                    tc_fence_after();
+                    const int st = c & 1, sb = c & 1, par = (c >> 1) & 1;
+                    ok = mbar_wait(&bars->sempty[sb], par ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    for (int b = 0; b < KBLK && ok; ++b) {
+                        ok = mbar_wait(&bars->bfull[st][b], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                        if (!ok) break;
+                        fence_proxy_async_smem();
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t boff = (uint32_t)(st * KSTAGE + (kk >> 2) * (NK * 128) + (kk & 3) * 32);
-                        mma_ts(tmem + S_COL + sb * NK, tmem + kk * 8, desc_sw128(kbase + boff, 1024), idesc, kk > 0);
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const int kk = b * 4 + k4;
+                            const uint32_t boff = (uint32_t)(st * KSTAGE + b * (NK * 128) + k4 * 32);
+                            mma_ts(tmem + S_COL + sb * NK, tmem + kk * 8, desc_sw128(kbase + boff, 1024), idesc, kk > 0);
+                        }
+                        mma_commit(&bars->bempty[st][b]);
                     }
-                    mma_commit(&bars->kempty[st]);
-                    mma_commit(&bars->sfull[sb]);
+                    if (ok) mma_commit(&bars->sfull[sb]);
                 }
             } else {
                 constexpr uint32_t idesc = idesc_bf16_f32(H, 256, 0, 1);
                 const uint32_t vbase = smem_u32(gbuf), pbase = smem_u32(pbuf);
                 bool ok = true;
+                constexpr uint32_t idesc128 = idesc_bf16_f32(H, 128, 0, 1);
                 for (int c = 0; c < w.nchunks && ok; ++c) {
-                    const int st = c & 1, pb = c % PSLOTS;
-                    ok = mbar_wait(&bars->vfull[st], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
-                         mbar_wait(&bars->ready[pb], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-                    if (!ok) break;
-                    fence_proxy_async_smem();
-                    tc_fence_after();
+                    const int st = c & 1, pb = c % PSLOTS, par = (c >> 1) & 1;
+                    ok = mbar_wait(&bars->ready[pb], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    // O[:, 128j:128j+128] += P . V[:, 128j:128j+128] as dim-block pairs land
+                    for (int j = 0; j < VBLK / 2 && ok; ++j) {
+                        ok = mbar_wait(&bars->bfull[st][2 * j], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
+                             mbar_wait(&bars->bfull[st][2 * j + 1], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                        if (!ok) break;
+                        fence_proxy_async_smem();
+                        tc_fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < NK / 16; ++kk) {
-                        const uint64_t adesc = desc_sw128(pbase + pb * PBYTES + kk * 32, 1024);
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            const uint32_t boff = (uint32_t)(st * VSTAGE + half * 4 * (NK * 128) + kk * 16 * 128);
-                            mma_ss(tmem + half * 256, adesc, desc_sw128_mn(vbase + boff, NK * 128, 1024), idesc,
+                        for (int kk = 0; kk < NK / 16; ++kk) {
+                            const uint64_t adesc = desc_sw128(pbase + pb * PBYTES + kk * 32, 1024);
+                            const uint32_t boff = (uint32_t)(st * KSTAGE + 2 * j * (NK * 128) + kk * 16 * 128);
+                            mma_ss(tmem + j * 128, adesc, desc_sw128_mn(vbase + boff, NK * 128, 1024), idesc128,
                                    (c > 0 || kk > 0) ? 1u : 0u);
                         }
+                        mma_commit(&bars->bempty[st][2 * j]);
+                        mma_commit(&bars->bempty[st][2 * j + 1]);
                     }
-                    mma_commit(&bars->vempty[st]);
+                    if (!ok) break;
                     mma_commit_multicast(&bars->pempty[pb], (uint16_t)0x3);
                     mma_commit(&bars->odone);
                 }
@@ -526,8 +576,8 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restric
 
 namespace {
 
-constexpr size_t MLA_SMEM = 1024 + REGION + PSLOTS * (PBYTES + ABYTES) + SBYTES + 512;
-static_assert(sizeof(Bars) <= 512, "barrier block");
+constexpr size_t MLA_SMEM = 1024 + REGION + PSLOTS * (PBYTES + ABYTES) + SBYTES + 4 * H * 4 + 1024;
+static_assert(sizeof(Bars) <= 1024, "barrier block");
 
 int choose_splits(int rows, int k, int num_sms) {
     const int clusters = num_sms / 2;
@@ -549,9 +599,34 @@ size_t mla_tc_workspace_bytes(int rows, int k, int num_sms) {
     return (size_t)rows * s * H * (DV + 1) * sizeof(float);
 }
 
+typedef CUresult (*EncodeTiledFnM)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2-D view [total_rows, 576] bf16 of the latent cache, box 64 columns x 1 row
+// (the box shape of a 4-row gather), 128-byte swizzle.
+static bool make_kv_map(CUtensorMap* m, const void* kv, uint64_t total_rows) {
+    static EncodeTiledFnM fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &qr) != cudaSuccess ||
+            qr != cudaDriverEntryPointSuccess)
+            return false;
+        fn = (EncodeTiledFnM)f;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)DK, total_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)DK * 2};
+    cuuint32_t box[2] = {64, 1};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
-                          const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch, int ctx_len,
-                          float scale, void* out, float* lse, void* workspace, size_t ws_bytes) {
+                          int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                          int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes) {
     if (rows == 0) return cudaSuccess;
     MlaParams p;
     p.q = (const __nv_bfloat16*)q;
@@ -564,6 +639,10 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.err = L.err;
     p.page_size = page_table ? page_size : 1;
     p.pages_per_seq = page_table ? ctx_len / page_size : 0;
+    p.num_pages = page_table ? num_pages : 0;
+    CUtensorMap kv_map;
+    const uint64_t total_rows = page_table ? (uint64_t)num_pages * page_size : (uint64_t)batch * ctx_len;
+    if (total_rows >= (1ull << 31) || !make_kv_map(&kv_map, kv, total_rows)) return cudaErrorInvalidValue;
     p.k = k;
     p.rows = rows;
     p.batch = batch;
@@ -595,7 +674,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, kv_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1) {

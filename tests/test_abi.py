@@ -74,13 +74,16 @@ def test_invalid_arguments_rejected_before_launch(lib):
     # indexer: unsupported head dim
     assert lib.dsa_indexer_logits(fake, 1, fake, fake, 1, None, fake, fake, 4, 4, 128, 64, 96, fake, 128, None) == 2
     # sparse MLA: null output
-    lib.dsa_sparse_mla.argtypes = [vp, vp, ctypes.c_int, vp, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
+    lib.dsa_sparse_mla.argtypes = [vp, vp, ctypes.c_int, vp, ctypes.c_int, ctypes.c_int, vp, vp, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
-    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, fake, fake, 2048, 4, 4, 4096, 128, 576, 512, 0.04, None,
+    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, 0, fake, fake, 2048, 4, 4, 4096, 128, 576, 512, 0.04, None,
                               fake, None, 0, None) == 1
     # sparse MLA: unbuilt head geometry
-    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, fake, fake, 2048, 4, 4, 4096, 100, 576, 512, 0.04, fake,
+    assert lib.dsa_sparse_mla(fake, fake, 1, None, 0, 0, fake, fake, 2048, 4, 4, 4096, 100, 576, 512, 0.04, fake,
                               fake, None, 0, None) == 2
+    # paged cache without a page count
+    assert lib.dsa_sparse_mla(fake, fake, 1, fake, 64, 0, fake, fake, 2048, 4, 4, 4096, 128, 576, 512, 0.04, fake,
+                              fake, None, 0, None) == 1
     # zero rows is a no-op success without touching the device
     assert lib.dsa_topk(fake, 100, fake, 0, 100, 5, fake, None, 0, None) == 0
