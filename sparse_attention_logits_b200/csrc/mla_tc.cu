@@ -28,14 +28,10 @@
 //                       over several clusters, normalised fp32 partials that
 //                       dsa_mla_combine merges.
 //
-// The selected rows are gathered by TMA (tile::gather4, 4 rows per
-// instruction) one 8 KB dim block (64 rows x 64 dims) at a time; a block is
-// refilled for chunk c+2 as soon as the MMA of chunk c is done with it, and
-// the MMA of a chunk starts on its first block.
-//
-// Warps (both CTAs): 0 TMA gather producer (1-3 spare); 4-11 softmax (score
-// CTA: two threads per head, 32 keys each) or 4-7 rescale + epilogue (value
-// CTA, one thread per head / TMEM lane); 12 MMA issuer and TMEM owner.  Every wait is bounded; the two CTAs only exchange
+// Warps (both CTAs): 0-15 gather producers (cp.async, 4 rows each); 16-23
+// softmax (score CTA: two threads per head, 32 keys each) or 16-19 rescale +
+// epilogue (value CTA, one thread per head / TMEM lane); 24 MMA issuer and
+// TMEM owner.  Every wait is bounded; the two CTAs only exchange
 // data through bulk copies and mbarrier arrivals that the receiver waits on.
 #include "common.cuh"
 #include "launchers.h"
@@ -51,10 +47,16 @@ constexpr int H = 128;              // query heads = MMA M
 constexpr int DK = 576;             // latent + rope
 constexpr int DV = 512;             // value dims
 constexpr int NK = 64;              // keys per chunk
-constexpr int PWARPS = 4;           // warp 0 issues the TMA row gathers; warps 1-3 are spare
+constexpr int PWARPS = 16;          // gather producer warps: cp.async throughput grows with the copies in flight
+constexpr int ROWS_PER_PW = NK / PWARPS;
 constexpr int SWARP0 = PWARPS;      // first of the 8 softmax warps (score CTA) / 4 rescale-epilogue warps (value CTA)
-constexpr int MWARP = PWARPS + 8;   // MMA issuer, TMEM owner
-constexpr int THREADS = 32 * (PWARPS + 9);
+constexpr int MWARP = PWARPS + 8;   // MMA issuer, TMEM owner (its warpgroup's other 3 warps are spare)
+constexpr int THREADS = 32 * (PWARPS + 12);     // 7 warpgroups
+// Register split (per thread) after launch at THREADS x 72: producer and MMA
+// warpgroups give registers back, the softmax warpgroups take them.
+constexpr int REGS_LOW = 56, REGS_SOFTMAX = 104, REGS_LAUNCH = 72;
+static_assert(PWARPS * 32 * REGS_LOW + 8 * 32 * REGS_SOFTMAX + 4 * 32 * REGS_LAUNCH <= REGS_LAUNCH * THREADS,
+              "register split exceeds launch");
 constexpr int KBLK = DK / 64;       // 9 dim blocks of 64 (128 B per row) per gathered row
 constexpr int VBLK = DV / 64;       // the value CTA gathers the first 8
 constexpr int KSTAGE = NK * DK * 2; // 73728 B
@@ -70,8 +72,8 @@ constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between 
 constexpr float LN2 = 0.6931471805599453f;
 
 struct Bars {                       // same offset in both CTAs of a cluster
-    uint64_t bfull[2][KBLK];        // a dim block of a stage has landed (cp.async arrivals)
-    uint64_t bempty[2][KBLK];       // the MMA is done reading a dim block of a stage
+    uint64_t full[2];               // a stage's gathered rows have landed (cp.async arrivals)
+    uint64_t empty[2];              // the MMA is done reading a stage
     uint64_t sfull[2], sempty[2], pready[PSLOTS], pempty[PSLOTS], qready, statready, statack;
     uint64_t pfull[PSLOTS], ready[PSLOTS], odone, statfull;
     uint64_t mx[4];                 // score CTA: the two softmax warps of a lane quarter exchange maxima
@@ -149,42 +151,40 @@ __device__ __forceinline__ int slot_index(const MlaParams& p, const Work& w, int
 // Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// Gather of the selected rows with TMA row gathers (tile::gather4), one 8 KB
-// dim block (64 rows x 64 dims) at a time: lane g of the producer warp owns
-// rows 4g..4g+3 of every chunk and issues one 4-row gather per dim block,
-// which lands in the 128-B-swizzled layout the MMA reads.  A block of stage
-// st is refilled as soon as the MMA has finished reading it; unused slots
-// gather row -1, which the TMA fills with zeros.
+// Gather of the selected rows with cp.async, 16 bytes per copy: warp w owns
+// rows [4w, 4w+4) of every chunk (one index lookup per lane, resolved one
+// chunk ahead) and its lanes walk those rows with consecutive lanes on
+// consecutive 16-byte pieces.  Many producer warps are used because the copy
+// throughput of an SM grows with the number of copies its threads keep in
+// flight.
 template <int NB>   // dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
-__device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, const CUtensorMap* map, uint8_t* gbuf,
-                                            Bars* bars, int lane, volatile int* abort_flag) {
-    const int g = lane & 15;
-    int nrow[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) nrow[q] = (int)key_row(p, w, w.slot0 + 4 * g + q);   // rows fit in 31 bits
-    bool ok = true;
-    for (int c = 0; c < w.nchunks && ok; ++c) {
-        const int st = c & 1, par = ((c >> 1) & 1) ^ 1;
-        const int r0 = nrow[0], r1 = nrow[1], r2 = nrow[2], r3 = nrow[3];
+__device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, Bars* bars, int warp,
+                                            int lane, volatile int* abort_flag) {
+    constexpr int RC = NB * 8;                           // 16-byte pieces per row
+    const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
+    int64_t next_row = key_row(p, w, w.slot0 + my_slot);
+    for (int c = 0; c < w.nchunks; ++c) {
+        const int st = c & 1;
+        if (!mbar_wait(&bars->empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+        const int myrow_lo = (int)(next_row >= 0 ? next_row : -1);  // row indices fit in 31 bits
         uint8_t* base = gbuf + (size_t)st * KSTAGE;
-        for (int b = 0; b < NB; ++b) {
-            if (!mbar_wait(&bars->bempty[st][b], par, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) { ok = false; break; }
-            if (lane == 0) mbar_arrive_expect_tx(&bars->bfull[st][b], NK * 128);
-            __syncwarp();
-            if (lane < 16) tma_gather4(base + b * (NK * 128) + g * 512, map, b * 64, r0, r1, r2, r3, &bars->bfull[st][b]);
-        }
-        // look up the next chunk's rows while this chunk's gathers are in flight
-        if (c + 1 < w.nchunks) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) nrow[q] = (int)key_row(p, w, w.slot0 + (c + 1) * NK + 4 * g + q);
+        for (int i = lane; i < ROWS_PER_PW * RC; i += 32) {
+            const int rl = i / RC, ci = i - rl * RC;
+            const int row = __shfl_sync(0xffffffffu, myrow_lo, rl);
+            const int r = warp * ROWS_PER_PW + rl;
+            const __nv_bfloat16* src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8 : p.kv;
+            cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
         }
+        cp_async_arrive_noinc(&bars->full[st]);
+        // look up the next chunk's row while this chunk's copies are in flight
+        if (c + 1 < w.nchunks) next_row = key_row(p, w, w.slot0 + (c + 1) * NK + my_slot);
     }
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap kv_map,
-                                                          const MlaParams p) {
+__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
@@ -201,10 +201,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            for (int b = 0; b < KBLK; ++b) {
-                mbar_init(&bars->bfull[i][b], 1);
-                mbar_init(&bars->bempty[i][b], 1);
-            }
+            mbar_init(&bars->full[i], PWARPS * 32);
+            mbar_init(&bars->empty[i], 1);
             mbar_init(&bars->sfull[i], 1);
             mbar_init(&bars->sempty[i], 8);
         }
@@ -221,7 +219,6 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         mbar_init(&bars->odone, 1);
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
-        tma_prefetch_desc(&kv_map);
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
         if (rank == 1) {
             // arm the first phase of each P slot and the final-statistics slot
@@ -241,17 +238,18 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     const uint32_t peer = rank ^ 1u;
 
     if (warp < PWARPS) {
-        // ------------------------------------------------- gather producer ----
+        // ------------------------------------------------ gather producers ----
+        regs_dec<REGS_LOW>();
         // Warp w owns rows [8w, 8w+8) of every chunk: lane l resolves one of
         // them once per chunk (one index load per lane, all in flight
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (warp == 0) {
-            if (rank == 0) gather_rows<KBLK>(p, w, &kv_map, gbuf, bars, lane, abort_flag);
-            else gather_rows<VBLK>(p, w, &kv_map, gbuf, bars, lane, abort_flag);
-        }
-    } else if (warp < SWARP0 + 8 && rank == 0) {
+        if (rank == 0) gather_rows<KBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
+        else gather_rows<VBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
+    } else if (warp < SWARP0 + 8) {
+      regs_inc<REGS_SOFTMAX>();
+      if (rank == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
         // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
         // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
@@ -399,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         mbar_wait(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         for (int c = max(0, w.nchunks - PSLOTS); c < w.nchunks; ++c)
             mbar_wait(&bars->pempty[c % PSLOTS], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-    } else if (warp < SWARP0 + 4) {
+      } else if (warp < SWARP0 + 4) {
         // ------------------------- value CTA: rescale of O, then epilogue ----
         const int h = (warp - SWARP0) * 32 + lane;
         const uint32_t lane_base = (uint32_t)((warp - SWARP0) * 32) << 16;
@@ -475,7 +473,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                 p.part_lse[pr] = lse;
             }
         }
-    } else if (warp == MWARP) {
+      }
+    } else {
+      if (warp == MWARP) {
         // ----------------------------------------------------- MMA issuer ----
         if (elect_one()) {
             if (rank == 0) {
@@ -485,53 +485,49 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                 tc_fence_after();
                 for (int c = 0; c < w.nchunks && ok; ++c) {
                     const int st = c & 1, sb = c & 1, par = (c >> 1) & 1;
-                    ok = mbar_wait(&bars->sempty[sb], par ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-                    for (int b = 0; b < KBLK && ok; ++b) {
-                        ok = mbar_wait(&bars->bfull[st][b], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
-                        if (!ok) break;
-                        fence_proxy_async_smem();
-                        tc_fence_after();
+                    ok = mbar_wait(&bars->sempty[sb], par ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag) &&
+                         mbar_wait(&bars->full[st], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                    if (!ok) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
 #pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const int kk = b * 4 + k4;
-                            const uint32_t boff = (uint32_t)(st * KSTAGE + b * (NK * 128) + k4 * 32);
-                            mma_ts(tmem + S_COL + sb * NK, tmem + kk * 8, desc_sw128(kbase + boff, 1024), idesc, kk > 0);
-                        }
-                        mma_commit(&bars->bempty[st][b]);
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t boff = (uint32_t)(st * KSTAGE + (kk >> 2) * (NK * 128) + (kk & 3) * 32);
+                        mma_ts(tmem + S_COL + sb * NK, tmem + kk * 8, desc_sw128(kbase + boff, 1024), idesc, kk > 0);
                     }
+                    mma_commit(&bars->empty[st]);
                     if (ok) mma_commit(&bars->sfull[sb]);
                 }
             } else {
                 constexpr uint32_t idesc = idesc_bf16_f32(H, 256, 0, 1);
                 const uint32_t vbase = smem_u32(gbuf), pbase = smem_u32(pbuf);
                 bool ok = true;
-                constexpr uint32_t idesc128 = idesc_bf16_f32(H, 128, 0, 1);
                 for (int c = 0; c < w.nchunks && ok; ++c) {
                     const int st = c & 1, pb = c % PSLOTS, par = (c >> 1) & 1;
                     ok = mbar_wait(&bars->ready[pb], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-                    // O[:, 128j:128j+128] += P . V[:, 128j:128j+128] as dim-block pairs land
-                    for (int j = 0; j < VBLK / 2 && ok; ++j) {
-                        ok = mbar_wait(&bars->bfull[st][2 * j], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag) &&
-                             mbar_wait(&bars->bfull[st][2 * j + 1], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
-                        if (!ok) break;
-                        fence_proxy_async_smem();
-                        tc_fence_after();
+                    ok = ok && mbar_wait(&bars->full[st], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                    if (!ok) break;
+                    fence_proxy_async_smem();
+                    tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < NK / 16; ++kk) {
-                            const uint64_t adesc = desc_sw128(pbase + pb * PBYTES + kk * 32, 1024);
-                            const uint32_t boff = (uint32_t)(st * KSTAGE + 2 * j * (NK * 128) + kk * 16 * 128);
-                            mma_ss(tmem + j * 128, adesc, desc_sw128_mn(vbase + boff, NK * 128, 1024), idesc128,
+                    for (int kk = 0; kk < NK / 16; ++kk) {
+                        const uint64_t adesc = desc_sw128(pbase + pb * PBYTES + kk * 32, 1024);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            const uint32_t boff = (uint32_t)(st * KSTAGE + half * 4 * (NK * 128) + kk * 16 * 128);
+                            mma_ss(tmem + half * 256, adesc, desc_sw128_mn(vbase + boff, NK * 128, 1024), idesc,
                                    (c > 0 || kk > 0) ? 1u : 0u);
                         }
-                        mma_commit(&bars->bempty[st][2 * j]);
-                        mma_commit(&bars->bempty[st][2 * j + 1]);
                     }
+                    mma_commit(&bars->empty[st]);
                     if (!ok) break;
                     mma_commit_multicast(&bars->pempty[pb], (uint16_t)0x3);
                     mma_commit(&bars->odone);
                 }
             }
         }
+    }
+
     }
 
     tc_fence_before();
@@ -599,31 +595,6 @@ size_t mla_tc_workspace_bytes(int rows, int k, int num_sms) {
     return (size_t)rows * s * H * (DV + 1) * sizeof(float);
 }
 
-typedef CUresult (*EncodeTiledFnM)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// 2-D view [total_rows, 576] bf16 of the latent cache, box 64 columns x 1 row
-// (the box shape of a 4-row gather), 128-byte swizzle.
-static bool make_kv_map(CUtensorMap* m, const void* kv, uint64_t total_rows) {
-    static EncodeTiledFnM fn = nullptr;
-    if (!fn) {
-        void* f = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &qr) != cudaSuccess ||
-            qr != cudaDriverEntryPointSuccess)
-            return false;
-        fn = (EncodeTiledFnM)f;
-    }
-    cuuint64_t dims[2] = {(cuuint64_t)DK, total_rows};
-    cuuint64_t strides[1] = {(cuuint64_t)DK * 2};
-    cuuint32_t box[2] = {64, 1};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(kv), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
                           int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
                           int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes) {
@@ -640,9 +611,6 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.page_size = page_table ? page_size : 1;
     p.pages_per_seq = page_table ? ctx_len / page_size : 0;
     p.num_pages = page_table ? num_pages : 0;
-    CUtensorMap kv_map;
-    const uint64_t total_rows = page_table ? (uint64_t)num_pages * page_size : (uint64_t)batch * ctx_len;
-    if (total_rows >= (1ull << 31) || !make_kv_map(&kv_map, kv, total_rows)) return cudaErrorInvalidValue;
     p.k = k;
     p.rows = rows;
     p.batch = batch;
@@ -674,7 +642,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, kv_map, p);
+    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1) {
