@@ -12,7 +12,8 @@
  *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
  *     never allocates or frees device memory; scratch space, where a step
  *     needs some, is a caller-provided workspace whose size the matching
- *     *_workspace_size() function returns.
+ *     *_workspace_size() function returns (dsa_sparse_mla_noalloc instead
+ *     uses a fixed scratch array in the library's own device memory).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call only enqueues work on that stream and returns; it
  *     never synchronizes, except dsa_get_device_error().
@@ -175,6 +176,35 @@ DSA_API dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t d
                             int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
                             float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the fixed device scratch that dsa_sparse_mla_noalloc uses. */
+#define DSA_MLA_NOALLOC_SCRATCH_BYTES ((size_t)20 << 20)
+
+/*
+ * dsa_sparse_mla_noalloc -- dsa_sparse_mla without a workspace argument; it
+ * allocates nothing, by any route.  The method itself has no counterpart:
+ * this is an interface for callers that may not allocate device memory
+ * while they run a step, such as a serving engine that hands nearly all of
+ * HBM to its paged KV cache up front and keeps cudaMalloc/cudaFree (which
+ * can block and synchronize the device) out of its decode loop, or a plain C
+ * caller with no device allocator of its own.
+ *
+ * Arguments, layouts, results and errors are those of dsa_sparse_mla.  The
+ * partial results of a split key list go to a static scratch array of
+ * DSA_MLA_NOALLOC_SCRATCH_BYTES in the library's device memory (one copy per
+ * device), whose address is looked up on the first call on each device: make
+ * that first call before any stream capture.  Sizes whose partials do not
+ * fit return DSA_ERR_INVALID_ARG with the byte counts in dsa_last_error()
+ * and enqueue nothing (on a 148-SM B200 every size fits).  No part of the
+ * scratch needs clearing between calls.  Calls that overlap in time on one
+ * device -- from two streams or two threads -- race on the scratch and give
+ * undefined results; calls in order on one stream are safe.
+ */
+DSA_API dsa_status_t dsa_sparse_mla_noalloc(const void* q, const void* kv, dsa_dtype_t dtype,
+                            const int32_t* page_table, int page_size, int num_pages,
+                            const int32_t* row_batch, const int32_t* idx, int k,
+                            int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
+                            float scale, void* out, float* lse, void* stream);
 
 /*
  * dsa_get_device_error -- synchronizes `stream`, then reads and clears the

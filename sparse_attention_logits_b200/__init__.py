@@ -50,6 +50,8 @@ _SIGS = {
     "dsa_sparse_mla_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "dsa_sparse_mla": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                               _f32, _vp, _vp, _vp, _sz, _vp]),
+    "dsa_sparse_mla_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                      _i32, _f32, _vp, _vp, _vp]),
     "dsa_get_device_error": (_i32, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -200,6 +202,30 @@ def sparse_mla(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: 
         _check(_lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages, _ptr(row_batch),
                                    _ptr(idx), k, rows, B, ctx_len, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
                                    _ptr(workspace), wsb, _stream(dev)), "dsa_sparse_mla")
+    return out, lse
+
+
+def sparse_mla_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: torch.Tensor, scale: float,
+                       d_v: int, ctx_len: int, out: torch.Tensor, lse: torch.Tensor,
+                       page_table: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """sparse_mla through the entry point that allocates nothing: the caller
+    passes out [rows, H, d_v] and lse [rows, H]; split partials go to the
+    library's fixed device scratch (calls overlapping on one device race)."""
+    dev = _dev(q, kv, idx, row_batch, page_table, out, lse)
+    rows, H, DK = q.shape
+    k = idx.shape[1]
+    if page_table is not None:
+        B = page_table.shape[0]
+        num_pages, page_size = kv.shape[0], kv.shape[1]
+    else:
+        B = kv.shape[0]
+        num_pages, page_size = 0, 0
+        if kv.shape[1] != ctx_len:
+            raise ValueError("kv.shape[1] != ctx_len")
+    with torch.cuda.device(dev):
+        _check(_lib.dsa_sparse_mla_noalloc(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages,
+                                           _ptr(row_batch), _ptr(idx), k, rows, B, ctx_len, H, DK, d_v, float(scale),
+                                           _ptr(out), _ptr(lse), _stream(dev)), "dsa_sparse_mla_noalloc")
     return out, lse
 
 

@@ -4,6 +4,8 @@
 #include <stdio.h>
 #include <stdarg.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "launchers.h"
 
@@ -50,6 +52,39 @@ dsa_status_t make_launch(void* stream, dsa::Launch* L) {
     L->stream = (cudaStream_t)stream;
     L->err = g_err_ptr[dev];
     L->num_sms = g_num_sms[dev];
+    return DSA_OK;
+}
+
+// Fixed scratch of dsa_sparse_mla_noalloc: the fp32 partial outputs and
+// log-sum-exps of a key list split over several clusters.  A (row, split)
+// pair takes 128 heads x 513 floats = 262,656 bytes, and the split count is
+// chosen so that rows x splits <= SMs / 2, so 20 MiB covers every size on a
+// GPU of up to 159 SMs.  No byte of it has to start at zero: each cluster
+// writes its whole partial block before the merge kernel, launched after it
+// on the same stream, reads it.  One copy per device: calls that overlap on
+// one device (two streams, two threads) race on it.
+constexpr size_t kMlaScratchBytes = DSA_MLA_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_mla_scratch[kMlaScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_mla_scratch on the current device, looked up once per
+// device (cudaGetSymbolAddress may load the module, so the first call must
+// not happen inside a stream capture).
+dsa_status_t mla_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mla_scratch);
+        if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(sparse MLA scratch)");
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
     return DSA_OK;
 }
 
@@ -185,6 +220,29 @@ dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, co
     return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows, batch,
                                             ctx_len, n_heads, d_qk, d_v, scale, out, lse),
                        "dsa_sparse_mla launch");
+}
+
+dsa_status_t dsa_sparse_mla_noalloc(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
+                                    int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k,
+                                    int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v, float scale,
+                                    void* out, float* lse, void* stream) {
+    void* scratch = nullptr;
+    if (rows > 0 && k >= 1 && dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v)) {
+        dsa::Launch L;
+        dsa_status_t st = make_launch(stream, &L);
+        if (st != DSA_OK) return st;
+        const size_t need = dsa::mla_tc_workspace_bytes(rows, k, L.num_sms);
+        if (need > kMlaScratchBytes)
+            return fail(DSA_ERR_INVALID_ARG,
+                        "dsa_sparse_mla_noalloc: %d rows x k=%d need %zu bytes of scratch, more than its fixed %zu",
+                        rows, k, need, kMlaScratchBytes);
+        if (need) {
+            st = mla_scratch(&scratch);
+            if (st != DSA_OK) return st;
+        }
+    }
+    return dsa_sparse_mla(q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows, batch, ctx_len,
+                          n_heads, d_qk, d_v, scale, out, lse, scratch, scratch ? kMlaScratchBytes : 0, stream);
 }
 
 dsa_status_t dsa_get_device_error(void* stream) {
