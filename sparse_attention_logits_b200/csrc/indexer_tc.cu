@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "sm100.cuh"
+#include "tensor_map.h"
 
 namespace dsa {
 
@@ -399,44 +400,14 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
 
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = (EncodeTiledFn)p;
-    }
-    return fn;
-}
-
-// 2-D row-major tensor [rows, cols] with 128-byte-swizzled boxes.
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
-              uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int NQ, bool FP8>
 cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Params& p) {
     using C = Cfg<NQ, FP8>;
     CUtensorMap mk, mq;
     const uint64_t krows = (uint64_t)p.batch * p.ctx;
-    bool ok = FP8 ? make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
-                  : make_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, DI, krows, 64, KT);
-    ok = ok && make_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DI, (uint64_t)p.rows * HI, 64, NQ * HI);
+    bool ok = FP8 ? make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
+                  : make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, DI, krows, 64, KT);
+    ok = ok && make_map_sw128(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DI, (uint64_t)p.rows * HI, 64, NQ * HI);
     if (!ok) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<NQ, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM);

@@ -36,6 +36,7 @@
 #include "common.cuh"
 #include "launchers.h"
 #include "sm100.cuh"
+#include "tensor_map.h"
 
 namespace dsa {
 
@@ -49,7 +50,7 @@ constexpr int DV = 512;             // value dims
 constexpr int NK = 64;              // keys per chunk
 constexpr int PWARPS = 16;          // gather producer warps: cp.async throughput grows with the copies in flight
 constexpr int ROWS_PER_PW = NK / PWARPS;
-constexpr int SWARP0 = PWARPS;      // first of the 8 softmax warps (score CTA) / 4 rescale-epilogue warps (value CTA)
+constexpr int SWARP0 = PWARPS;      // first of the 8 softmax warps (score CTA) / 8 rescale-epilogue warps (value CTA)
 constexpr int MWARP = PWARPS + 8;   // MMA issuer, TMEM owner (its warpgroup's other 3 warps are spare)
 constexpr int THREADS = 32 * (PWARPS + 12);     // 7 warpgroups
 // Register split (per thread) after launch at THREADS x 72: producer and MMA
@@ -62,6 +63,9 @@ constexpr int VBLK = DV / 64;       // the value CTA gathers the first 8
 constexpr int KSTAGE = NK * DK * 2; // 73728 B
 constexpr int STAGES = 2;
 constexpr int REGION = STAGES * KSTAGE;  // [stage][dim block][64 rows x 128 B]
+constexpr int QBYTES = H * DK * 2;  // 147456: the Q tile, staged through the same region before the gather starts
+static_assert(QBYTES == REGION, "Q staging uses the gather region");
+constexpr int EPI_BUF = 4096;       // epilogue: per-warp output staging tile (32 heads x 128 B), two per warp
 constexpr int PBYTES = H * NK * 2;  // 16384: P [128 heads x 64 keys] bf16
 constexpr int PSLOTS = 4;           // P ring depth (score CTA may run this many chunks ahead)
 constexpr int ABYTES = H * 4;       // rescale factor per head
@@ -74,9 +78,12 @@ constexpr float LN2 = 0.6931471805599453f;
 struct Bars {                       // same offset in both CTAs of a cluster
     uint64_t full[2];               // a stage's gathered rows have landed (cp.async arrivals)
     uint64_t empty[2];              // the MMA is done reading a stage
-    uint64_t sfull[2], sempty[2], pready[PSLOTS], pempty[PSLOTS], qready, statready, statack;
-    uint64_t pfull[PSLOTS], ready[PSLOTS], odone, statfull;
-    uint64_t mx[4];                 // score CTA: the two softmax warps of a lane quarter exchange maxima
+    uint64_t sfull[2], sempty[2], pempty[PSLOTS], qready, statready, statack;
+    // value CTA: P slot landed / rescaled, PV of chunk c done (ring of PSLOTS, so
+    // that a parity wait never aliases), all PV done, final statistics landed
+    uint64_t pfull[PSLOTS], ready[PSLOTS], odone[PSLOTS], ofinal, statfull;
+    uint64_t qfull;                 // score CTA: the Q tile has landed in shared memory
+    int flag[2][2][8];              // score CTA: per softmax warp "still ok" at the two pair barriers of a chunk
     uint32_t tmem;
     int abort;
 };
@@ -163,6 +170,8 @@ __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, u
     constexpr int RC = NB * 8;                           // 16-byte pieces per row
     const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
     int64_t next_row = key_row(p, w, w.slot0 + my_slot);
+    // score CTA: the region holds the Q tile until it has been moved to TMEM
+    if (NB == KBLK && !mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)) return;
     for (int c = 0; c < w.nchunks; ++c) {
         const int st = c & 1;
         if (!mbar_wait(&bars->empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
@@ -184,7 +193,9 @@ __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, u
 
 }  // namespace
 
-__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
+__global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap q_map,
+                                                          const __grid_constant__ CUtensorMap o_map,
+                                                          const MlaParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
@@ -192,6 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
     float* abuf = (float*)(pbuf + PSLOTS * PBYTES);         // [PSLOTS][H]
     float* sbuf = abuf + PSLOTS * H;                        // [2*H]: running max, running sum
     float* xbuf = sbuf + 2 * H;                             // [2][2][H]: partial maxima / sums of the two halves
+                                                            // of a head (score CTA)
     Bars* bars = (Bars*)(xbuf + 4 * H);
     volatile int* abort_flag = &bars->abort;
 
@@ -207,16 +219,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             mbar_init(&bars->sempty[i], 8);
         }
         for (int i = 0; i < PSLOTS; ++i) {
-            mbar_init(&bars->pready[i], 8);
             mbar_init(&bars->pempty[i], 1);
             mbar_init(&bars->pfull[i], 1);
             mbar_init(&bars->ready[i], 4);
+            mbar_init(&bars->odone[i], 1);
         }
         mbar_init(&bars->qready, 8);
+        mbar_init(&bars->qfull, 1);
         mbar_init(&bars->statready, 8);
-        for (int i = 0; i < 4; ++i) mbar_init(&bars->mx[i], 2);
         mbar_init(&bars->statack, 4);
-        mbar_init(&bars->odone, 1);
+        mbar_init(&bars->ofinal, 1);
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
@@ -226,6 +238,15 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             mbar_arrive_expect_tx(&bars->statfull, SBYTES);
         }
         fence_mbar_init();
+        if (rank == 0) {
+            // Q [128 heads x 576] of this row: 9 boxes of 128 rows x 64 dims,
+            // 128-byte swizzled, into the (still unused) gather region
+            tma_prefetch_desc(&q_map);
+            mbar_arrive_expect_tx(&bars->qfull, QBYTES);
+            for (int b = 0; b < KBLK; ++b) tma_load_2d(gbuf + b * (H * 128), &q_map, b * 64, w.t * H, &bars->qfull);
+        } else {
+            tma_prefetch_desc(&o_map);
+        }
     }
     if (warp == MWARP) {
         tmem_alloc(&bars->tmem, TMEM_COLS);
@@ -253,57 +274,61 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         // ------------------------------------- score CTA: Q load + softmax ----
         // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
         // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
-        // of every chunk; the two halves of a head exchange their partial
-        // maxima each chunk, so both take the same rescaling decision.
+        // of every chunk.  The two warps of a quarter (a "pair") meet at a
+        // named barrier twice per chunk: to combine their partial maxima, so
+        // both take the same rescaling decision, and once both halves of the
+        // quarter's P rows are in shared memory, after which one of them sends
+        // those rows and the quarter's rescale factors to the value CTA.  Each
+        // warp posts whether it is still ok at both meetings, so that the two
+        // always leave the loop together (a named barrier has no time limit).
         const int sw = warp - SWARP0, half = sw >> 2, quarter = sw & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        {   // Q row of head h -> TMEM lane h; this half writes columns [144*half, 144*half + 144)
-            const uint4* qrow = (const uint4*)(p.q + ((int64_t)w.t * H + h) * DK) + half * 36;
+        const int pair_bar = 1 + quarter;
+        volatile int* flag = &bars->flag[0][0][0];
+        bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->qfull, 0, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag));
+        if (ok) {   // Q row h -> TMEM lane h; this half writes the 16-column groups [9*half, 9*half + 9)
 #pragma unroll 1
-            for (int m0 = 0; m0 < 9; m0 += 5) {                 // 16-column groups, loads batched
-                uint4 x[20];
+            for (int g = 9 * half; g < 9 * half + 9; ++g) {
+                const uint8_t* row = gbuf + (g >> 1) * (H * 128) + h * 128;
+                uint32_t words[16];
 #pragma unroll
-                for (int v = 0; v < 20; ++v)
-                    if (m0 * 4 + v < 36) x[v] = __ldg(qrow + m0 * 4 + v);
-#pragma unroll
-                for (int m = 0; m < 5; ++m) {
-                    if (m0 + m < 9) {
-                        uint32_t words[16];
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            words[4 * v] = x[4 * m + v].x; words[4 * v + 1] = x[4 * m + v].y;
-                            words[4 * v + 2] = x[4 * m + v].z; words[4 * v + 3] = x[4 * m + v].w;
-                        }
-                        tmem_st16(tmem + lane_base + half * 144 + (m0 + m) * 16, words);
-                    }
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 x = ld_shared_v4(row + ((((g & 1) * 4 + v) ^ (h & 7)) << 4));
+                    words[4 * v] = x.x; words[4 * v + 1] = x.y; words[4 * v + 2] = x.z; words[4 * v + 3] = x.w;
                 }
+                tmem_st16(tmem + lane_base + g * 16, words);
             }
             tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->qready);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->qready);
         float m_run = -INFINITY, l_run = 0.f;                   // l_run: this half's keys
         const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
-        bool ok = true;
         // whether this lane's key of a chunk is real: the raw index is loaded
         // one chunk ahead and only inspected in the next iteration
         int s_next = slot_index(p, w, w.slot0 + 32 * half + lane);
-        for (int c = 0; c < w.nchunks && ok; ++c) {
-            const int sb = c & 1;
+        for (int c = 0; c < w.nchunks; ++c) {
+            const int sb = c & 1, par = c & 1;
             const uint32_t vmask = __ballot_sync(0xffffffffu, w.b_ok && s_next >= 0 && s_next < p.ctx);
             if (c + 1 < w.nchunks) s_next = slot_index(p, w, w.slot0 + (c + 1) * NK + 32 * half + lane);
-            ok = mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
-            if (!ok) break;
-            tc_fence_after();
             float sv[32];
-            tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32 * half, sv);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+            if (ok)
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32 * half, sv);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+            }
             float mx[16];
 #pragma unroll
             for (int j = 0; j < 32; ++j) sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
@@ -313,11 +338,11 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
                 for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-            float* xb = xbuf + (c & 1) * 2 * H;
+            float* xb = xbuf + par * 2 * H;
             xb[half * H + h] = mx[0];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->mx[quarter]);
-            ok = mbar_wait(&bars->mx[quarter], c & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+            if (lane == 0) flag[(0 * 2 + par) * 8 + sw] = ok ? 1 : 0;
+            named_bar_sync(pair_bar, 64);
+            ok = ok && flag[(0 * 2 + par) * 8 + (sw ^ 4)] != 0;        // the same in both warps of the pair
             if (!ok) break;
             const float mc = fmaxf(mx[0], xb[(half ^ 1) * H + h]);
             float alpha = 1.f;
@@ -349,37 +374,37 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                 for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
             l_run += ls[0];
             const int pb = c % PSLOTS, pu = c / PSLOTS;
-            ok = mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-            if (!ok) break;
-            uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
+            // the slot's previous P has been consumed by the value CTA's MMA
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
+            if (ok) {
+                uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                *(uint4*)(prow + sw128(h & 7, 4 * half + jj)) =
-                    make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-            if (half == 0) abuf[pb * H + h] = alpha;
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->pready[pb]);
-            if (warp == SWARP0 && lane == 0) {
-                ok = mbar_wait(&bars->pready[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-                if (ok) {
-                    const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
-                    bulk_copy_s2cluster(peer_pbuf + pb * PBYTES, pbuf + pb * PBYTES, PBYTES, rbar);
-                    bulk_copy_s2cluster(peer_abuf + pb * ABYTES, abuf + pb * H, ABYTES, rbar);
-                }
+                for (int jj = 0; jj < 4; ++jj)
+                    st_shared_v4(prow + sw128(h & 7, 4 * half + jj), pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2],
+                                 pk[4 * jj + 3]);
+                if (half == 0) abuf[pb * H + h] = alpha;
+                fence_proxy_async_smem();
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+            if (lane == 0) flag[(1 * 2 + par) * 8 + sw] = ok ? 1 : 0;
+            named_bar_sync(pair_bar, 64);
+            ok = ok && flag[(1 * 2 + par) * 8 + (sw ^ 4)] != 0;
+            if (!ok) break;
+            if (half == 0 && lane == 0) {
+                // this quarter's 32 P rows (4 KB, contiguous) and 32 rescale factors
+                const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
+                const uint32_t poff = (uint32_t)(pb * PBYTES + quarter * 4096);
+                bulk_copy_s2cluster(peer_pbuf + poff, pbuf + poff, 4096, rbar);
+                bulk_copy_s2cluster(peer_abuf + pb * ABYTES + quarter * 128, abuf + pb * H + quarter * 32, 128, rbar);
+            }
         }
         // final statistics -> value CTA: running max (same in both halves) and
         // the sum of the two halves' running sums
         if (ok) {
-            const int c = w.nchunks;
-            float* xb = xbuf + (c & 1) * 2 * H;
+            float* xb = xbuf + (w.nchunks & 1) * 2 * H;
             xb[half * H + h] = l_run;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->mx[quarter]);
-            ok = mbar_wait(&bars->mx[quarter], c & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-            if (ok && half == 0) {
+            named_bar_sync(pair_bar, 64);
+            if (half == 0) {
                 sbuf[h] = m_run;
                 sbuf[H + h] = l_run + xb[H + h];
             }
@@ -397,38 +422,50 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
         mbar_wait(&bars->statack, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         for (int c = max(0, w.nchunks - PSLOTS); c < w.nchunks; ++c)
             mbar_wait(&bars->pempty[c % PSLOTS], (c / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-      } else if (warp < SWARP0 + 4) {
-        // ------------------------- value CTA: rescale of O, then epilogue ----
-        const int h = (warp - SWARP0) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)((warp - SWARP0) * 32) << 16;
+      } else {
+        // --------------------------- value CTA: rescale of O, then epilogue ----
+        // Warps SWARP0..SWARP0+3 (one thread per head / TMEM lane) apply the
+        // per-chunk rescale factors to O before its next PV MMA.  At the end
+        // all 8 warps write O / l: warp SWARP0 + 4*colhalf + quarter takes
+        // heads [32*quarter, +32) and columns [256*colhalf, +256), in tiles of
+        // 32 heads x 128 B staged in 128-byte-swizzled shared memory (the
+        // drained gather region) and stored with TMA.
+        const int sw = warp - SWARP0, quarter = sw & 3, colhalf = sw >> 2;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
-        for (int c = 0; c < w.nchunks && ok; ++c) {
-            const int pb = c % PSLOTS, pu = c / PSLOTS;
-            ok = mbar_wait(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
-            if (!ok) break;
-            if (warp == SWARP0 && lane == 0 && c + PSLOTS < w.nchunks)
-                mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
-            const float alpha = abuf[pb * H + h];
-            if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                ok = mbar_wait(&bars->odone, (c - 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+        if (colhalf == 0) {
+            for (int c = 0; c < w.nchunks && ok; ++c) {
+                const int pb = c % PSLOTS, pu = c / PSLOTS;
+                ok = mbar_wait(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 if (!ok) break;
-                tc_fence_after();
+                if (warp == SWARP0 && lane == 0 && c + PSLOTS < w.nchunks)
+                    mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
+                const float alpha = abuf[pb * H + h];
+                if (c > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    // O must hold all of chunk c-1 (P of chunk c arriving means
+                    // the PV MMA of chunk c-4 is done, so this parity is unambiguous)
+                    const int pc = c - 1;
+                    ok = mbar_wait(&bars->odone[pc % PSLOTS], (pc / PSLOTS) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
 #pragma unroll 1
-                for (int j = 0; j < DV / 32; ++j) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + j * 32, v);
-                    tmem_ld_wait();
+                    for (int j = 0; j < DV / 32; ++j) {
+                        float v[32];
+                        tmem_ld32(tmem + lane_base + j * 32, v);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] *= alpha;
-                    tmem_st32(tmem + lane_base + j * 32, v);
+                        for (int e = 0; e < 32; ++e) v[e] *= alpha;
+                        tmem_st32(tmem + lane_base + j * 32, v);
+                    }
+                    tmem_st_wait();
                 }
-                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->ready[pb]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->ready[pb]);
         }
-        if (ok) ok = mbar_wait(&bars->odone, (w.nchunks - 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+        if (ok) ok = mbar_wait(&bars->ofinal, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
         if (ok) ok = mbar_wait(&bars->statfull, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         float m = -INFINITY, l = 0.f;
         if (ok) {
@@ -436,42 +473,78 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
             l = sbuf[H + h];
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->statack), peer));
+        if (colhalf == 0 && lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->statack), peer));
+        ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const float lse = l > 0.f ? (m + log2f(l)) * LN2 : -INFINITY;
+            uint8_t* stage = gbuf + sw * 2 * EPI_BUF;
+            uint8_t* srow = stage + lane * 128;
             if (p.splits == 1) {
-                uint4* orow = (uint4*)(p.out + ((int64_t)w.t * H + h) * DV);
+                // bf16 tiles of 32 heads x 64 columns
+                const int row0 = w.t * H + quarter * 32;
 #pragma unroll 1
-                for (int j = 0; j < DV / 32; ++j) {
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + j * 32, v);
+                for (int j = 0; j < 4; ++j) {
+                    const int col = colhalf * 256 + j * 64;
+                    float v[32], u[32];
+                    tmem_ld32(tmem + lane_base + col, v);
+                    tmem_ld32(tmem + lane_base + col + 32, u);
                     tmem_ld_wait();
-                    uint32_t o[16];
+                    if (j >= 2) {                       // the store that read this buffer two tiles ago is done
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                    }
+                    uint8_t* buf = srow + (j & 1) * EPI_BUF;
+                    uint32_t o[32];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const __nv_bfloat162 x = __floats2bfloat162_rn(v[2 * e] * inv, v[2 * e + 1] * inv);
+                        const __nv_bfloat162 y = __floats2bfloat162_rn(u[2 * e] * inv, u[2 * e + 1] * inv);
                         o[e] = *(const uint32_t*)&x;
+                        o[16 + e] = *(const uint32_t*)&y;
                     }
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) orow[j * 4 + e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+                    for (int ci = 0; ci < 8; ++ci)
+                        st_shared_v4(buf + ((ci ^ (lane & 7)) << 4), o[4 * ci], o[4 * ci + 1], o[4 * ci + 2], o[4 * ci + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&o_map, stage + (j & 1) * EPI_BUF, col, row0);
+                        bulk_commit_group();
+                    }
                 }
-                p.lse[(int64_t)w.t * H + h] = lse;
+                if (colhalf == 0) p.lse[(int64_t)w.t * H + h] = lse;
             } else {
-                const int64_t pr = ((int64_t)w.t * p.splits + w.split) * H + h;
-                float4* orow = (float4*)(p.part_o + pr * DV);
+                // fp32 partial tiles of 32 heads x 32 columns
+                const int row0 = (w.t * p.splits + w.split) * H + quarter * 32;
 #pragma unroll 1
-                for (int j = 0; j < DV / 32; ++j) {
+                for (int j = 0; j < 8; ++j) {
+                    const int col = colhalf * 256 + j * 32;
                     float v[32];
-                    tmem_ld32(tmem + lane_base + j * 32, v);
+                    tmem_ld32(tmem + lane_base + col, v);
                     tmem_ld_wait();
+                    if (j >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                    }
+                    uint8_t* buf = srow + (j & 1) * EPI_BUF;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        orow[j * 8 + e] = make_float4(v[4 * e] * inv, v[4 * e + 1] * inv, v[4 * e + 2] * inv, v[4 * e + 3] * inv);
+                    for (int ci = 0; ci < 8; ++ci)
+                        st_shared_v4(buf + ((ci ^ (lane & 7)) << 4), __float_as_uint(v[4 * ci] * inv),
+                                     __float_as_uint(v[4 * ci + 1] * inv), __float_as_uint(v[4 * ci + 2] * inv),
+                                     __float_as_uint(v[4 * ci + 3] * inv));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&o_map, stage + (j & 1) * EPI_BUF, col, row0);
+                        bulk_commit_group();
+                    }
                 }
-                p.part_lse[pr] = lse;
+                if (colhalf == 0) p.part_lse[((int64_t)w.t * p.splits + w.split) * H + h] = lse;
             }
+            if (lane == 0) bulk_wait_group<0>();
+            __syncwarp();
         }
       }
     } else {
@@ -520,10 +593,10 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const MlaParams p) {
                         }
                     }
                     mma_commit(&bars->empty[st]);
-                    if (!ok) break;
                     mma_commit_multicast(&bars->pempty[pb], (uint16_t)0x3);
-                    mma_commit(&bars->odone);
+                    mma_commit(&bars->odone[pb]);
                 }
+                if (ok) mma_commit(&bars->ofinal);
             }
         }
     }
@@ -624,10 +697,21 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.part_lse = nullptr;
     if (p.splits > 1) {
         const size_t need = (size_t)rows * p.splits * H * (DV + 1) * sizeof(float);
-        if (!workspace || ws_bytes < need) return cudaErrorInvalidValue;
+        if (!workspace || ws_bytes < need || (uintptr_t)workspace % 16) return cudaErrorInvalidValue;
         p.part_o = (float*)workspace;
         p.part_lse = p.part_o + (size_t)rows * p.splits * H * DV;
     }
+    // Q as [rows*128, 576] bf16 in boxes of 128 heads x 64 dims; the output as
+    // [rows*128, 512] bf16 in boxes of 32 heads x 64 columns, or the partials
+    // as [rows*splits*128, 512] fp32 in boxes of 32 heads x 32 columns
+    CUtensorMap q_map, o_map;
+    bool ok = make_map_sw128(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DK, (uint64_t)rows * H, 64, H);
+    if (p.splits == 1)
+        ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, DV, (uint64_t)rows * H, 64, 32);
+    else
+        ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.part_o, DV,
+                                  (uint64_t)rows * p.splits * H, 32, 32);
+    if (!ok) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -642,7 +726,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, q_map, o_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1) {
