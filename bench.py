@@ -33,7 +33,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-INDEXER_SRC = "indexer_simt.cu"   # source of the kernel that runs the bf16 indexer
+INDEXER_SRC = "indexer_tc.cu"     # source of the kernel that runs the bf16 indexer
 METRIC = "DSA decode queries/s @32K ctx & prefill tok/s; fraction of HBM/tensor roofline"
 
 
