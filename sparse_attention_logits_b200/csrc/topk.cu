@@ -359,12 +359,15 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
 
 namespace {
 
-// Smallest cluster whose CTAs can hold a row in shared memory: a row that
-// fits one SM is selected by one CTA (no cross-CTA traffic at all).
-int choose_cluster(int /*rows*/, int ctx_len) {
+// Cluster size: at least enough CTAs to hold a row in shared memory, and,
+// when there are few rows, as many more (up to 8) as keep every SM busy --
+// a decode batch of 32 rows would otherwise leave most SMs idle.  Many rows
+// that fit one SM each are selected one CTA per row (no cross-CTA traffic).
+int choose_cluster(int rows, int ctx_len, int num_sms) {
     const int need = (ctx_len + SLICE_CAP - 1) / SLICE_CAP;
     int cl = 1;
     while (cl < need && cl < 8) cl <<= 1;
+    while (cl < 8 && (int64_t)rows * cl * 2 <= num_sms && ctx_len / (cl * 2) >= 4096) cl <<= 1;
     return cl;
 }
 
@@ -399,7 +402,7 @@ bool topk_supported(int ctx_len) { return ctx_len <= 8 * SLICE_CAP; }
 cudaError_t launch_topk(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows,
                         int ctx_len, int k, int32_t* idx, void* /*workspace*/, size_t /*ws_bytes*/) {
     if (rows == 0) return cudaSuccess;
-    switch (choose_cluster(rows, ctx_len)) {
+    switch (choose_cluster(rows, ctx_len, L.num_sms)) {
     case 1: return launch_cl<1>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
     case 2: return launch_cl<2>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
     case 4: return launch_cl<4>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
