@@ -30,7 +30,9 @@ namespace {
 constexpr int TOPK_THREADS = 1024;
 constexpr int NBINS = 2048;                    // 11-bit digits
 constexpr int SLICE_CAP = 40960;               // keys per CTA kept in shared memory (160 KB)
-constexpr int SMEM_FIXED = 4 * NBINS * 4 + 64 * 4 + 8 * 16;   // hist, 3 per-pass merged histograms, scratch
+constexpr int MAX_PASSES = 4;
+// hist, merged (scan scratch), one cluster-wide histogram per pass, scratch
+constexpr int SMEM_FIXED = (2 + MAX_PASSES) * NBINS * 4 + 64 * 4 + 8 * 16;
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -100,8 +102,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* tk_smem = (uint32_t*)(((uintptr_t)tk_smem_raw + 127) & ~(uintptr_t)127);
     uint32_t* hist = tk_smem;                    // [NBINS]   this CTA's histogram
     uint32_t* merged = hist + NBINS;             // [NBINS]   scratch for the suffix scan
-    uint32_t* cl_hist = merged + NBINS;          // [2][NBINS] cluster-wide histograms (rank 0 holds them)
-    uint32_t* warp_sums = cl_hist + 2 * NBINS;   // [33]
+    uint32_t* cl_hist = merged + NBINS;          // [MAX_PASSES][NBINS] cluster-wide histograms (rank 0 holds them)
+    uint32_t* warp_sums = cl_hist + MAX_PASSES * NBINS;   // [33]
     uint32_t* shared_res = warp_sums + 40;       // digit, count above
     uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers)
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         }
     }
     if (CL > 1)
-        for (int i = tid; i < 2 * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
+        for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
     cl_sync<CL>();                               // cluster histograms are zero before anyone adds
 
     // ---- 1. select the exact k-th largest key ----
@@ -163,11 +165,16 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     // range's width), finds the bucket that holds the remaining-th largest
     // candidate and shrinks [lo, hi] to it.  Bucketing by the actual range
     // spreads keys over the bins even when all scores share one exponent.
+    // the slice is padded with copies of its first key up to a multiple of 4
+    // (cnt4), so that every walk below reads 16 bytes per lane
+    const int cnt4 = (cnt + 3) & ~3;
+    for (int i = cnt + tid; i < cnt4; i += TOPK_THREADS) keys[i] = keys[0];
+    __syncthreads();
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i = tid; i < cnt; i += TOPK_THREADS) {
-        const uint32_t key = keys[i];
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
+    for (int i = 4 * tid; i < cnt4; i += 4 * TOPK_THREADS) {
+        const uint4 q = *(const uint4*)(keys + i);
+        kmin = min(min(kmin, min(q.x, q.y)), min(q.z, q.w));
+        kmax = max(max(kmax, max(q.x, q.y)), max(q.z, q.w));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -202,22 +209,26 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     __syncthreads();
     uint32_t lo_key = shared_res[4], hi_key = shared_res[5], remaining = (uint32_t)k;
 #pragma unroll 1
-    for (int pass = 0; pass < 4 && lo_key != hi_key; ++pass) {
+    for (int pass = 0; pass < MAX_PASSES && lo_key != hi_key; ++pass) {
         const uint32_t width = hi_key - lo_key;
         const int s_bits = 32 - __clz(width) - 11;        // (width >> s) < NBINS
         const int sh = s_bits > 0 ? s_bits : 0;
         for (int i = tid; i < NBINS; i += TOPK_THREADS) hist[i] = 0u;
         __syncthreads();
-        for (int i = tid; i < cnt; i += TOPK_THREADS) {
-            const uint32_t key = keys[i];
-            if (key >= lo_key && key <= hi_key) atomicAdd(&hist[(key - lo_key) >> sh], 1u);
+        for (int i = 4 * tid; i < cnt; i += 4 * TOPK_THREADS) {
+            const uint4 q = *(const uint4*)(keys + i);
+            const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i + u < cnt && kq[u] >= lo_key && kq[u] <= hi_key) atomicAdd(&hist[(kq[u] - lo_key) >> sh], 1u);
         }
         __syncthreads();
         // cluster-wide histogram: thread t owns bins 2t and 2t+1
         uint32_t h0, h1;
         if (CL > 1) {
-            const int buf = pass & 1;            // rank 0 zeroes a buffer after it has been read
-            const uint32_t lead = mapa_shared(smem_u32(cl_hist + buf * NBINS + 2 * tid), 0u);
+            // a fresh, zeroed buffer per pass: no CTA can add into a buffer
+            // another is still reading
+            const uint32_t lead = mapa_shared(smem_u32(cl_hist + pass * NBINS + 2 * tid), 0u);
             if (hist[2 * tid]) red_cluster_add(lead, hist[2 * tid]);
             if (hist[2 * tid + 1]) red_cluster_add(lead + 4, hist[2 * tid + 1]);
             cl_sync<CL>();                       // all additions landed
@@ -252,30 +263,37 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         const uint32_t span = sh == 0 ? 0u : ((1u << sh) - 1u);
         hi_key = (hi_key - new_lo > span) ? new_lo + span : hi_key;
         lo_key = new_lo;
-        if (CL > 1) {
-            cl_sync<CL>();                       // everyone has read this pass's cluster histogram
-            if (rank == 0)
-                for (int i = tid; i < NBINS; i += TOPK_THREADS) cl_hist[(pass & 1) * NBINS + i] = 0u;
-        } else {
-            __syncthreads();
-        }
+        __syncthreads();                         // shared_res / merged are reused by the next pass
     }
     const uint32_t T = lo_key;                   // the k-th largest key; `remaining` keys == T to take
 
     // ---- 2. ordered compaction ----
-    // Warp w owns a contiguous run of the slice and walks it 32 keys at a
-    // time (consecutive lanes on consecutive keys: no bank conflicts,
-    // coalesced index writes); ballots give each selected key its rank.
+    // Warp w owns a contiguous run of the slice and walks it 128 keys at a
+    // time, lane l on the 4 consecutive keys 4l..4l+3 of each step (16-byte
+    // loads); warp scans of the lanes' counts give every selected key its rank.
     const int warp = tid >> 5, lane = tid & 31;
-    const uint32_t lt_mask = (1u << lane) - 1u;
-    const int chunk = (((cnt + 31) / 32) + 31) / 32 * 32;           // keys per warp, multiple of 32
+    const int chunk = (((cnt + 127) / 128) + 31) / 32 * 128;        // keys per warp, multiple of 128
     const int wlo = min(cnt, warp * chunk), whi = min(cnt, wlo + chunk);
     uint32_t gt_w = 0, eq_w = 0;
-    for (int base = wlo; base < whi; base += 32) {
-        const int i = base + lane;
-        const uint32_t key = i < whi ? keys[i] : 0u;
-        gt_w += __popc(__ballot_sync(0xffffffffu, i < whi && key > T));
-        eq_w += __popc(__ballot_sync(0xffffffffu, i < whi && key == T));
+    for (int base = wlo; base < whi; base += 128) {
+        const int i = base + 4 * lane;
+        uint32_t g = 0, e = 0;
+        if (i < whi) {
+            const uint4 q = *(const uint4*)(keys + i);
+            const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                g += (i + u < whi && kq[u] > T) ? 1u : 0u;
+                e += (i + u < whi && kq[u] == T) ? 1u : 0u;
+            }
+        }
+        gt_w += g;
+        eq_w += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        gt_w += __shfl_xor_sync(0xffffffffu, gt_w, o);
+        eq_w += __shfl_xor_sync(0xffffffffu, eq_w, o);
     }
     uint32_t* wgt = merged;                      // per-warp counts and offsets (scratch)
     uint32_t* weq = merged + 32;
@@ -342,17 +360,46 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     __syncthreads();
     uint32_t j = wout[warp], eq_seen = 0;
     const uint32_t take = wtake[warp];
-    for (int base = wlo; base < whi; base += 32) {
-        const int i = base + lane;
-        const bool ok = i < whi;
-        const uint32_t key = ok ? keys[i] : 0u;
-        const bool is_gt = ok && key > T, is_eq = ok && key == T;
-        const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
-        const bool sel = is_gt || (is_eq && eq_seen + __popc(eqm & lt_mask) < take);
-        const uint32_t selm = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[j + __popc(selm & lt_mask)] = lo + i;
-        j += __popc(selm);
-        eq_seen += __popc(eqm);
+    for (int base = wlo; base < whi; base += 128) {
+        const int i = base + 4 * lane;
+        uint32_t kq[4] = {0u, 0u, 0u, 0u};
+        if (i < whi) {
+            const uint4 q = *(const uint4*)(keys + i);
+            kq[0] = q.x; kq[1] = q.y; kq[2] = q.z; kq[3] = q.w;
+        }
+        uint32_t gm = 0, em = 0;                 // per-lane bit masks of its 4 keys
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            gm |= (i + u < whi && kq[u] > T) ? (1u << u) : 0u;
+            em |= (i + u < whi && kq[u] == T) ? (1u << u) : 0u;
+        }
+        // equal keys before this lane (in position order), then the lane's own
+        uint32_t e_incl = __popc(em);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, e_incl, o);
+            if (lane >= o) e_incl += y;
+        }
+        uint32_t e_before = eq_seen + e_incl - __popc(em);
+        uint32_t sm = gm;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if ((em >> u) & 1u) {
+                if (e_before < take) sm |= 1u << u;
+                ++e_before;
+            }
+        uint32_t s_incl = __popc(sm);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, s_incl, o);
+            if (lane >= o) s_incl += y;
+        }
+        uint32_t o_at = j + s_incl - __popc(sm);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if ((sm >> u) & 1u) out[o_at++] = lo + i + u;
+        j += __shfl_sync(0xffffffffu, s_incl, 31);
+        eq_seen += __shfl_sync(0xffffffffu, e_incl, 31);
     }
     if (CL > 1) cl_sync<CL>();                   // peers are done reading our counts
 }
