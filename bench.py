@@ -13,9 +13,13 @@ Multi-GPU (launched by torchrun, one process per GPU): every rank runs its
 own independent batch (replicas, weak scaling, no collective on the data
 path); the step time is the max over ranks.
 
-Timing: CUDA events on the launching stream around each step; a 256 MB
-buffer is written between steps to flush L2 (outside the events); per-kernel
-times come from events between the kernels of the same steps.
+Timing: the step is captured in a CUDA graph and each replay is bracketed by
+CUDA events on the launching stream.  Decode: the inputs exceed L2 (268 MB of
+indexer keys, 1.2 GB of latent cache), so nothing is flushed between replays
+(a written flush would leave dirty lines whose write-back lands in the next
+step).  Prefill: a 256 MB buffer is written between replays (its 1 GB score
+matrix also evicts L2 every step).  Per-kernel times come from graphs holding
+one library call each.
 """
 from __future__ import annotations
 
@@ -245,15 +249,20 @@ def _graph(fn):
     return g
 
 
-def time_graph(g, steps, device, flush):
-    """Replay `g` `steps` times with an L2 flush before each replay (outside
-    the events); returns the mean device time of one replay in ms."""
+def time_graph(g, steps, device, flush=None):
+    """Replay `g` `steps` times, each bracketed by CUDA events on the current
+    stream; with `flush` (a buffer larger than L2) it is written before each
+    replay, outside the events.  Returns the mean device time of one replay
+    in ms.  Without `flush` the inputs themselves must exceed L2: a written
+    flush leaves L2 full of dirty lines whose write-back would then be
+    charged to the next replay."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(device)
     torch.cuda.synchronize(device)
     for a, b in evs:
-        flush.zero_()
+        if flush is not None:
+            flush.zero_()
         a.record()
         g.replay()
         b.record()
@@ -262,7 +271,7 @@ def time_graph(g, steps, device, flush):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
-def time_steps(step, steps, warmup, device, flush, soak_s=0.0):
+def time_steps(step, steps, warmup, device, flush=None, soak_s=0.0):
     """The step (indexer -> top-k -> sparse MLA) is captured once into a CUDA
     graph and replayed: timings are device time, free of host launch gaps.
     Per-kernel times come from graphs holding one library call each.
@@ -407,8 +416,7 @@ def run_kernel_only(args):
     dsa.get_device_error(device)
     host_ms = a.elapsed_time(b) / args.steps
     g = _graph(launch)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
-    dev_ms = time_graph(g, args.steps, device, flush)
+    dev_ms = time_graph(g, args.steps, device)
     print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": dev_ms, "ms_stream_launches": host_ms}))
 
 
@@ -424,11 +432,10 @@ def run_ours(args):
     wl = workloads.BY_NAME[args.workload]
     inp = workloads.generate(wl, device=device, seed=rank)
     step = DecodeStep(dsa, wl, inp, device)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     peaks = measured_peaks()
 
     with ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
-        ms, kern, launches = time_steps(step, args.steps, args.warmup, device, flush, soak_s=1.5)
+        ms, kern, launches = time_steps(step, args.steps, args.warmup, device, soak_s=1.5)
     dsa.get_device_error(device)
     ms_max = max_over_ranks(ms, device)
     value = wl.rows * world / (ms_max / 1e3)
@@ -451,7 +458,7 @@ def run_ours(args):
         "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "topk": wl.topk,
                    "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "mla": f"{wl.heads}h {wl.d_qk}/{wl.d_v}",
                    "parallelism": f"replicas{world}", "launch": "CUDA graph of the step (device time)",
-                   "l2": "inputs larger than L2 (keys 268 MB, latent cache 1.2 GB); 256 MB write between steps"},
+                   "l2": "inputs larger than L2 (keys 268 MB, latent cache 1.2 GB); no flush between steps"},
         "roofline": roof,
         "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
         "gpu_launches": launches,

@@ -50,13 +50,18 @@ struct Cfg {
     static constexpr int KBYTES = FP8 ? KT * DI : KT * DI * 2;      // one key tile in shared memory
     static constexpr int QBYTES = N * DI * 2;                        // one query tile (bf16)
     static constexpr int ACC_COLS = N;
-    static constexpr int A_COL0 = 2 * ACC_COLS;                     // fp8: bf16 key tiles in TMEM
+    // accumulator ring: decode has 4 (two epilogue groups take alternate
+    // tiles, so the per-tile epilogue never throttles the key stream)
+    static constexpr int NACC = NQ == 1 ? 4 : 2;
+    static constexpr int A_COL0 = NACC * ACC_COLS;                  // fp8: bf16 key tiles in TMEM
     static constexpr int A_COLS = DI / 2;                            // 128 bf16 = 64 columns
-    static constexpr int TMEM_NEED = 2 * ACC_COLS + (FP8 ? 2 * A_COLS : 0);
+    static constexpr int TMEM_NEED = NACC * ACC_COLS + (FP8 ? 2 * A_COLS : 0);
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
-    static constexpr int EPI_WARPS = NQ == 1 ? 4 : 8;
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * KBYTES + 2 * (size_t)QBYTES + 256;
+    static constexpr int EPI_WARPS = 8;     // NQ = 1: two groups of 4 on alternate tiles; NQ = 4: two column halves
+    static constexpr int NBARS = 2 * STAGES + 4 + 2 * NACC + 4;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * KBYTES + 2 * (size_t)QBYTES + NBARS * 8 + 16;
+    static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(TMEM_NEED <= 512, "TMEM budget");
     static_assert(N % 16 == 0 && N <= 256, "MMA N");
 };
@@ -178,9 +183,9 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     uint64_t* kempty = kfull + C::STAGES;         // [STAGES]
     uint64_t* qfull = kempty + C::STAGES;         // [2]
     uint64_t* qempty = qfull + 2;                 // [2]
-    uint64_t* accfull = qempty + 2;               // [2]
-    uint64_t* accempty = accfull + 2;             // [2]
-    uint64_t* afull = accempty + 2;               // [2] (fp8)
+    uint64_t* accfull = qempty + 2;               // [NACC]
+    uint64_t* accempty = accfull + C::NACC;       // [NACC]
+    uint64_t* afull = accempty + C::NACC;         // [2] (fp8)
     uint64_t* aempty = afull + 2;                 // [2] (fp8)
     uint32_t* tmem_slot = (uint32_t*)(aempty + 2);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -195,10 +200,12 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], 1);
-            mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], C::EPI_WARPS);
             mbar_init(&afull[i], 4);
             mbar_init(&aempty[i], 1);
+        }
+        for (int i = 0; i < C::NACC; ++i) {
+            mbar_init(&accfull[i], 1);
+            mbar_init(&accempty[i], NQ == 1 ? 4 : C::EPI_WARPS);   // the warps that read accumulator i
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -268,14 +275,14 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                     ok = mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                     if (!ok) break;
                 }
-                const int st = i % C::STAGES, acc = i & 1;
+                const int st = i % C::STAGES, acc = i % C::NACC, ab = i & 1;
                 if (FP8) {
-                    ok = mbar_wait(&afull[acc], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    ok = mbar_wait(&afull[ab], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 } else {
                     ok = mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                 }
                 if (!ok) break;
-                ok = mbar_wait(&accempty[acc], ((i >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                ok = mbar_wait(&accempty[acc], ((i / C::NACC) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t d = tmem + acc * C::ACC_COLS;
@@ -285,13 +292,13 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                     const uint32_t koff = (uint32_t)((kk >> 2) * (C::N * 128) + (kk & 3) * 32);
                     const uint64_t bdesc = desc_sw128(qaddr + koff, 1024);
                     if (FP8) {
-                        mma_ts(d, tmem + C::A_COL0 + acc * C::A_COLS + kk * 8, bdesc, idesc, kk > 0);
+                        mma_ts(d, tmem + C::A_COL0 + ab * C::A_COLS + kk * 8, bdesc, idesc, kk > 0);
                     } else {
                         const uint32_t aoff = (uint32_t)(st * C::KBYTES + (kk >> 2) * (KT * 128) + (kk & 3) * 32);
                         mma_ss(d, desc_sw128(kbase + aoff, 1024), bdesc, idesc, kk > 0);
                     }
                 }
-                if (FP8) mma_commit(&aempty[acc]);
+                if (FP8) mma_commit(&aempty[ab]);
                 else mma_commit(&kempty[st]);
                 mma_commit(&accfull[acc]);
                 if (un.last) mma_commit(&qempty[qe & 1]);
@@ -342,13 +349,16 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         }
     } else if (warp >= 8 && warp < 8 + C::EPI_WARPS) {
         // --------------------------------------------------- epilogue ----
+        // NQ = 1: warp group eg = (warp - 8) / 4 takes the units i with
+        // i % 2 == eg; NQ = 4: group eg takes query columns [128 eg, +128).
         const int quarter = warp & 3;
-        const int col_half = (warp - 8) >> 2;              // which 128 query columns (NQ = 4)
+        const int eg = (warp - 8) >> 2;
         sch.init(p);
         int i = 0;
         while (sch.next(p, un)) {
-            const int acc = i & 1;
-            if (!mbar_wait(&accfull[acc], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+            if (NQ == 1 && (i & 1) != eg) { ++i; continue; }
+            const int acc = i % C::NACC;
+            if (!mbar_wait(&accfull[acc], (i / C::NACC) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
             const int key = un.tile * KT + quarter * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * C::ACC_COLS;
@@ -356,19 +366,28 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             float score[QPW];
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-                const int qi = col_half * 2 + qq;          // query within the group
+                const int qi = NQ == 1 ? 0 : eg * 2 + qq;  // query within the group
                 float v0[32], v1[32];
                 tmem_ld32(tbase + qi * HI, v0);
                 tmem_ld32(tbase + qi * HI + 32, v1);
-                tmem_ld_wait();
                 const int t = min(un.t0 + qi, p.rows - 1);
-                const float* wr = p.w + (int64_t)t * HI;
-                float s = 0.f;
+                const float4* wr = (const float4*)(p.w + (int64_t)t * HI);
+                tmem_ld_wait();
+                // four independent partial sums (the weights are read as float4)
+                float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int h = 0; h < 32; ++h) s = fmaf(__ldg(wr + h), fmaxf(v0[h], 0.f), s);
-#pragma unroll
-                for (int h = 0; h < 32; ++h) s = fmaf(__ldg(wr + 32 + h), fmaxf(v1[h], 0.f), s);
-                score[qq] = s;
+                for (int h4 = 0; h4 < 8; ++h4) {
+                    const float4 wa = __ldg(wr + h4), wb = __ldg(wr + 8 + h4);
+                    s4[0] = fmaf(wa.x, fmaxf(v0[4 * h4], 0.f), s4[0]);
+                    s4[1] = fmaf(wa.y, fmaxf(v0[4 * h4 + 1], 0.f), s4[1]);
+                    s4[2] = fmaf(wa.z, fmaxf(v0[4 * h4 + 2], 0.f), s4[2]);
+                    s4[3] = fmaf(wa.w, fmaxf(v0[4 * h4 + 3], 0.f), s4[3]);
+                    s4[0] = fmaf(wb.x, fmaxf(v1[4 * h4], 0.f), s4[0]);
+                    s4[1] = fmaf(wb.y, fmaxf(v1[4 * h4 + 1], 0.f), s4[1]);
+                    s4[2] = fmaf(wb.z, fmaxf(v1[4 * h4 + 2], 0.f), s4[2]);
+                    s4[3] = fmaf(wb.w, fmaxf(v1[4 * h4 + 3], 0.f), s4[3]);
+                }
+                score[qq] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
             }
             tc_fence_before();
             __syncwarp();
@@ -380,7 +399,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             if (FP8 && b_ok && key < p.ctx) ks = __ldg(p.k_scale + (int64_t)b * p.ctx + key);
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
-                const int t = un.t0 + col_half * 2 + qq;
+                const int t = un.t0 + (NQ == 1 ? 0 : eg * 2 + qq);
                 if (b_ok && t < p.rows && key <= last_visible(p, t))
                     p.logits[(int64_t)t * p.ld + key] = FP8 ? score[qq] * ks : score[qq];
             }
