@@ -111,7 +111,8 @@ DSA_API dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch,
  *              s <= row_pos[t] are written; entries beyond row_pos[t] are
  *              left untouched (dsa_topk never reads them).
  * Accumulation is fp32.  Supported: head_dim in {32, 64, 128}; q and k of the
- * same floating type, or bf16 q with fp8 k; n_heads <= 128.
+ * same floating type, or bf16 q with fp8 k; n_heads <= 128.  fp8 key codes
+ * must be finite (0x7F and 0xFF, the e4m3 NaNs, are not valid codes).
  */
 DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float* w,
                                 const void* k, dsa_dtype_t k_dtype, const float* k_scale,

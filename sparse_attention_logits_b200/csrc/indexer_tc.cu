@@ -55,11 +55,15 @@ struct Cfg {
     static constexpr int NACC = NQ == 1 ? 4 : 2;
     static constexpr int A_COL0 = NACC * ACC_COLS;                  // fp8: bf16 key tiles in TMEM
     static constexpr int A_COLS = DI / 2;                            // 128 bf16 = 64 columns
-    static constexpr int TMEM_NEED = NACC * ACC_COLS + (FP8 ? 2 * A_COLS : 0);
+    // fp8: ring of widened key tiles in TMEM (as deep as the columns allow,
+    // so that the widening warps can run ahead of the MMA)
+    static constexpr int NA = FP8 ? (512 - NACC * ACC_COLS) / A_COLS < 4 ? (512 - NACC * ACC_COLS) / A_COLS : 4 : 2;
+    static constexpr int TMEM_NEED = NACC * ACC_COLS + (FP8 ? NA * A_COLS : 0);
+    static_assert(!FP8 || NA >= 2, "fp8 needs at least two widened key tiles in TMEM");
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int EPI_WARPS = 8;     // NQ = 1: two groups of 4 on alternate tiles; NQ = 4: two column halves
-    static constexpr int NBARS = 2 * STAGES + 4 + 2 * NACC + 4;
+    static constexpr int NBARS = 2 * STAGES + 4 + 2 * NACC + 2 * NA;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * KBYTES + 2 * (size_t)QBYTES + NBARS * 8 + 16;
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(TMEM_NEED <= 512, "TMEM budget");
@@ -156,7 +160,9 @@ struct Sched {
     }
 };
 
-// e4m3 pair (low byte = first element) -> bf16 pair, exact.
+// e4m3 pair (low byte = first element) -> bf16 pair, exact for every finite
+// code (the hardware e4m3 -> f16 conversion, then f16 -> f32 -> bf16, none of
+// which rounds: an e4m3 value has at most 4 significant bits).
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
@@ -185,9 +191,9 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     uint64_t* qempty = qfull + 2;                 // [2]
     uint64_t* accfull = qempty + 2;               // [NACC]
     uint64_t* accempty = accfull + C::NACC;       // [NACC]
-    uint64_t* afull = accempty + C::NACC;         // [2] (fp8)
-    uint64_t* aempty = afull + 2;                 // [2] (fp8)
-    uint32_t* tmem_slot = (uint32_t*)(aempty + 2);
+    uint64_t* afull = accempty + C::NACC;         // [NA] (fp8)
+    uint64_t* aempty = afull + C::NA;             // [NA] (fp8)
+    uint32_t* tmem_slot = (uint32_t*)(aempty + C::NA);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,6 +206,8 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], 1);
+        }
+        for (int i = 0; i < C::NA; ++i) {
             mbar_init(&afull[i], 4);
             mbar_init(&aempty[i], 1);
         }
@@ -275,9 +283,9 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                     ok = mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                     if (!ok) break;
                 }
-                const int st = i % C::STAGES, acc = i % C::NACC, ab = i & 1;
+                const int st = i % C::STAGES, acc = i % C::NACC, ab = i % C::NA;
                 if (FP8) {
-                    ok = mbar_wait(&afull[ab], (i >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                    ok = mbar_wait(&afull[ab], (i / C::NA) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 } else {
                     ok = mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                 }
@@ -312,9 +320,9 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         sch.init(p);
         int i = 0;
         while (sch.next(p, un)) {
-            const int st = i % C::STAGES, ab = i & 1;
+            const int st = i % C::STAGES, ab = i % C::NA;
             if (!mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
-            if (!mbar_wait(&aempty[ab], ((i >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+            if (!mbar_wait(&aempty[ab], ((i / C::NA) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
             const uint8_t* src = kbuf + (size_t)st * C::KBYTES + r * 128;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + ab * C::A_COLS;
