@@ -30,9 +30,11 @@ namespace {
 constexpr int TOPK_THREADS = 1024;
 constexpr int NBINS = 2048;                    // 11-bit digits
 constexpr int SLICE_CAP = 40960;               // keys per CTA kept in shared memory (160 KB)
-constexpr int MAX_PASSES = 4;
-// hist, merged (scan scratch), one cluster-wide histogram per pass, scratch
-constexpr int SMEM_FIXED = (2 + MAX_PASSES) * NBINS * 4 + 64 * 4 + 8 * 16;
+constexpr int MAX_PASSES = 3;                  // 11 + 10 + 10 bits: the range is exact after three passes
+constexpr int CAND_CAP = 1024;                 // candidates ranked directly after the first pass
+// hist, merged (scan scratch), one cluster-wide histogram per pass, scratch,
+// candidate buffer
+constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + CAND_CAP + 32) * 4;
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -90,6 +92,18 @@ __device__ __forceinline__ void red_cluster_add(uint32_t addr, uint32_t v) {
     asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
+// Atomic add on a shared-memory word of any CTA of the cluster (or of this
+// CTA); returns the old value.
+__device__ __forceinline__ uint32_t atom_add_cluster(uint32_t addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.relaxed.cluster.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(addr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
 }  // namespace
 
 template <int CL>
@@ -106,6 +120,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* warp_sums = cl_hist + MAX_PASSES * NBINS;   // [33]
     uint32_t* shared_res = warp_sums + 40;       // digit, count above
     uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers)
+    uint32_t* cand_n = cta_counts + 8;           // candidate count (rank 0's is used)
+    uint32_t* cand = cta_counts + 16;            // [CAND_CAP] candidate keys (rank 0's is used)
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
 
     const int row = blockIdx.x / CL;
@@ -157,6 +173,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     }
     if (CL > 1)
         for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
+    if (tid == 0) *cand_n = 0u;
     cl_sync<CL>();                               // cluster histograms are zero before anyone adds
 
     // ---- 1. select the exact k-th largest key ----
@@ -252,18 +269,75 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         if (above < remaining && above + h1 >= remaining) {
             shared_res[0] = 2u * tid + 1u;
             shared_res[1] = above;
+            shared_res[6] = h1;
         } else if (above + h1 < remaining && above + h1 + h0 >= remaining) {
             shared_res[0] = 2u * tid;
             shared_res[1] = above + h1;
+            shared_res[6] = h0;
         }
         __syncthreads();
-        const uint32_t bin = shared_res[0];
+        const uint32_t bin = shared_res[0], bin_cnt = shared_res[6];
         remaining -= shared_res[1];
         const uint32_t new_lo = lo_key + (bin << sh);
         const uint32_t span = sh == 0 ? 0u : ((1u << sh) - 1u);
         hi_key = (hi_key - new_lo > span) ? new_lo + span : hi_key;
         lo_key = new_lo;
         __syncthreads();                         // shared_res / merged are reused by the next pass
+        if (pass == 0 && lo_key != hi_key && bin_cnt <= (uint32_t)CAND_CAP) {
+            // Few keys are left in the chosen range (typically tens): gather
+            // them into rank 0's buffer and find the remaining-th largest by
+            // counting, for each candidate, the candidates above it.
+            const uint32_t n_addr = CL > 1 ? mapa_shared(smem_u32(cand_n), 0u) : smem_u32(cand_n);
+            const uint32_t c_addr = CL > 1 ? mapa_shared(smem_u32(cand), 0u) : smem_u32(cand);
+            const int lane = tid & 31, warp = tid >> 5;
+            for (int b0 = warp * 128; b0 < cnt; b0 += 128 * (TOPK_THREADS / 32)) {
+                const int i = b0 + 4 * lane;
+                uint32_t kq[4] = {0u, 0u, 0u, 0u};
+                if (i < cnt) {
+                    const uint4 q = *(const uint4*)(keys + i);
+                    kq[0] = q.x; kq[1] = q.y; kq[2] = q.z; kq[3] = q.w;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const bool c_ok = i + u < cnt && kq[u] >= lo_key && kq[u] <= hi_key;
+                    const uint32_t m = __ballot_sync(0xffffffffu, c_ok);
+                    if (m == 0u) continue;
+                    const int leader = __ffs(m) - 1;
+                    uint32_t base = 0u;
+                    if (lane == leader) base = atom_add_cluster(n_addr, (uint32_t)__popc(m));
+                    base = __shfl_sync(0xffffffffu, base, leader);
+                    if (c_ok) st_cluster_u32(c_addr + 4u * (base + __popc(m & ((1u << lane) - 1u))), kq[u]);
+                }
+            }
+            cl_sync<CL>();                       // every candidate has landed in rank 0's buffer
+            if (rank == 0) {
+                const uint32_t nc = *cand_n;
+                if ((uint32_t)tid < nc) {
+                    const uint32_t key = cand[tid];
+                    uint32_t gt = 0u, ge = 0u;
+                    for (uint32_t j = 0; j < nc; ++j) {
+                        const uint32_t kj = cand[j];
+                        gt += kj > key ? 1u : 0u;
+                        ge += kj >= key ? 1u : 0u;
+                    }
+                    if (gt < remaining && remaining <= ge) {   // every thread holding that key agrees
+                        shared_res[4] = key;
+                        shared_res[5] = remaining - gt;
+                    }
+                }
+            }
+            cl_sync<CL>();
+            if (CL > 1 && rank != 0) {
+                const uint32_t r0 = mapa_shared(smem_u32(shared_res + 4), 0u);
+                lo_key = ld_cluster_u32(r0);
+                remaining = ld_cluster_u32(r0 + 4);
+            } else {
+                lo_key = shared_res[4];
+                remaining = shared_res[5];
+            }
+            hi_key = lo_key;
+            break;
+        }
     }
     const uint32_t T = lo_key;                   // the k-th largest key; `remaining` keys == T to take
 
