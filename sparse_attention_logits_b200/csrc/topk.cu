@@ -144,7 +144,9 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     const int lo = min(n, (int)rank * per), hi = min(n, lo + per);
     const int cnt = hi - lo;
     // 8 independent 16-byte loads in flight per thread (one memory round trip
-    // for a 32K-key slice); scalar path for rows that are not 16-byte aligned
+    // for a 32K-key slice); scalar path for rows that are not 16-byte aligned.
+    // The key range of the slice is taken on the way.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     if ((((uintptr_t)(x + lo)) & 15u) == 0u) {
         const float4* x4 = (const float4*)(x + lo);
         const int n4 = cnt >> 2;
@@ -155,11 +157,20 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                 if (i0 + u * TOPK_THREADS < n4) v[u] = __ldg(x4 + i0 + u * TOPK_THREADS);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (i0 + u * TOPK_THREADS < n4)
-                    *(uint4*)(keys + 4 * (i0 + u * TOPK_THREADS)) =
-                        make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z), score_key(v[u].w));
+                if (i0 + u * TOPK_THREADS < n4) {
+                    const uint4 q = make_uint4(score_key(v[u].x), score_key(v[u].y), score_key(v[u].z),
+                                               score_key(v[u].w));
+                    *(uint4*)(keys + 4 * (i0 + u * TOPK_THREADS)) = q;
+                    kmin = min(min(kmin, min(q.x, q.y)), min(q.z, q.w));
+                    kmax = max(max(kmax, max(q.x, q.y)), max(q.z, q.w));
+                }
         }
-        for (int i = 4 * n4 + tid; i < cnt; i += TOPK_THREADS) keys[i] = score_key(__ldg(x + lo + i));
+        for (int i = 4 * n4 + tid; i < cnt; i += TOPK_THREADS) {
+            const uint32_t key = score_key(__ldg(x + lo + i));
+            keys[i] = key;
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+        }
     } else {
         for (int i0 = tid; i0 < cnt; i0 += 8 * TOPK_THREADS) {
             float v[8];
@@ -168,30 +179,13 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                 if (i0 + u * TOPK_THREADS < cnt) v[u] = __ldg(x + lo + i0 + u * TOPK_THREADS);
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-                if (i0 + u * TOPK_THREADS < cnt) keys[i0 + u * TOPK_THREADS] = score_key(v[u]);
+                if (i0 + u * TOPK_THREADS < cnt) {
+                    const uint32_t key = score_key(v[u]);
+                    keys[i0 + u * TOPK_THREADS] = key;
+                    kmin = min(kmin, key);
+                    kmax = max(kmax, key);
+                }
         }
-    }
-    if (CL > 1)
-        for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
-    if (tid == 0) *cand_n = 0u;
-    cl_sync<CL>();                               // cluster histograms are zero before anyone adds
-
-    // ---- 1. select the exact k-th largest key ----
-    // Adaptive range narrowing: the candidate keys lie in [lo, hi]; each pass
-    // buckets (key - lo) >> s into at most NBINS bins (s chosen from the
-    // range's width), finds the bucket that holds the remaining-th largest
-    // candidate and shrinks [lo, hi] to it.  Bucketing by the actual range
-    // spreads keys over the bins even when all scores share one exponent.
-    // the slice is padded with copies of its first key up to a multiple of 4
-    // (cnt4), so that every walk below reads 16 bytes per lane
-    const int cnt4 = (cnt + 3) & ~3;
-    for (int i = cnt + tid; i < cnt4; i += TOPK_THREADS) keys[i] = keys[0];
-    __syncthreads();
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i = 4 * tid; i < cnt4; i += 4 * TOPK_THREADS) {
-        const uint4 q = *(const uint4*)(keys + i);
-        kmin = min(min(kmin, min(q.x, q.y)), min(q.z, q.w));
-        kmax = max(max(kmax, max(q.x, q.y)), max(q.z, q.w));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -202,7 +196,14 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         merged[tid >> 5] = kmin;
         merged[32 + (tid >> 5)] = kmax;
     }
+    if (CL > 1)
+        for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
+    if (tid == 0) *cand_n = 0u;
     __syncthreads();
+    // the slice is padded with copies of its first key up to a multiple of 4
+    // (cnt4), so that every walk below reads 16 bytes per lane
+    const int cnt4 = (cnt + 3) & ~3;
+    for (int i = cnt + tid; i < cnt4; i += TOPK_THREADS) keys[i] = keys[0];
     if (tid == 0) {
         uint32_t a = 0xFFFFFFFFu, b = 0u;
         for (int w2 = 0; w2 < TOPK_THREADS / 32; ++w2) {
@@ -212,7 +213,15 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         cta_counts[2] = a;
         cta_counts[3] = b;
     }
-    cl_sync<CL>();                               // every CTA's min / max published
+    // every CTA's key range published, its cluster histograms zeroed
+    cl_sync<CL>();
+
+    // ---- 1. select the exact k-th largest key ----
+    // Adaptive range narrowing: the candidate keys lie in [lo, hi]; each pass
+    // buckets (key - lo) >> s into at most NBINS bins (s chosen from the
+    // range's width), finds the bucket that holds the remaining-th largest
+    // candidate and shrinks [lo, hi] to it.  Bucketing by the actual range
+    // spreads keys over the bins even when all scores share one exponent.
     if (tid == 0) {
         uint32_t a = 0xFFFFFFFFu, b = 0u;
         for (int r = 0; r < CL; ++r) {
