@@ -28,6 +28,15 @@
 //                       over several clusters, normalised fp32 partials that
 //                       dsa_mla_combine merges.
 //
+// Two splits per row (decode with few rows): both pairs of a row form one
+// 4-CTA cluster (ranks 0-1 split 0, ranks 2-3 split 1) and their value CTAs
+// merge the splits themselves: each sends the 256 columns that the other
+// finalises (raw fp32, DSMEM stores) as soon as both gather regions are
+// drained, then they swap (max, sum) per head and each writes its half of
+// out = (a O_0 + a' O_1) / (a l_0 + a' l_1).  This replaces the fp32 partials
+// in global memory and the merge launch whenever all rows' 4-CTA clusters fit
+// on the GPU at once.
+//
 // Warps (both CTAs): 0-15 gather producers (cp.async, 4 rows each); 16-23
 // softmax (score CTA: two threads per head, 32 keys each) or 16-19 rescale +
 // epilogue (value CTA, one thread per head / TMEM lane); 24 MMA issuer and
@@ -83,6 +92,8 @@ struct Bars {                       // same offset in both CTAs of a cluster
     // that a parity wait never aliases), all PV done, final statistics landed
     uint64_t pfull[PSLOTS], ready[PSLOTS], odone[PSLOTS], ofinal, statfull;
     uint64_t qfull;                 // score CTA: the Q tile has landed in shared memory
+    uint64_t cfree, cstat, crecv;   // fused two-split merge (value CTAs): the other split's gather region is
+                                    // drained / its statistics / its share of O have landed here
     int flag[2][2][8];              // score CTA: per softmax warp "still ok" at the two pair barriers of a chunk
     uint32_t tmem;
     int abort;
@@ -101,6 +112,7 @@ struct MlaParams {
     unsigned* err;
     int page_size, pages_per_seq, num_pages;
     int k, rows, batch, ctx, splits, per_split;
+    int fuse2;                      // two key splits per row in one 4-CTA cluster, merged in the kernel
     float scale_log2;
 };
 
@@ -153,6 +165,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // Raw key position stored in a slot (-1 past the end of this split's slots).
 __device__ __forceinline__ int slot_index(const MlaParams& p, const Work& w, int slot) {
     return slot < w.slot_end ? __ldg(p.idx + (int64_t)w.t * p.k + slot) : -1;
+}
+
+// Stores into another CTA's shared memory (cluster address from mapa).
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 // Offset of 16-byte chunk `c` of row `r` in a [rows x 128 B] 128-B-swizzled block.
@@ -208,7 +229,10 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
+    // a (query row, key split) is a pair of CTAs: role 0 = score CTA, role 1 =
+    // value CTA; with the fused two-split merge the cluster holds both splits
+    // of a row (ranks 0-1: split 0, ranks 2-3: split 1)
+    const uint32_t role = cluster_ctarank() & 1u;
     const Work w = work_of(p);
 
     if (threadIdx.x == 0) {
@@ -232,13 +256,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
-        if (rank == 1) {
+        mbar_init(&bars->cfree, 1);
+        mbar_init(&bars->cstat, H);
+        mbar_init(&bars->crecv, 8 * 32);
+        if (role == 1) {
             // arm the first phase of each P slot and the final-statistics slot
             for (int i = 0; i < PSLOTS && i < w.nchunks; ++i) mbar_arrive_expect_tx(&bars->pfull[i], PBYTES + ABYTES);
             mbar_arrive_expect_tx(&bars->statfull, SBYTES);
         }
         fence_mbar_init();
-        if (rank == 0) {
+        if (role == 0) {
             // Q [128 heads x 576] of this row: 9 boxes of 128 rows x 64 dims,
             // 128-byte swizzled, into the (still unused) gather region
             tma_prefetch_desc(&q_map);
@@ -256,7 +283,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     cluster_sync_all();                 // both CTAs' barriers exist before any remote traffic
     tc_fence_after();
     const uint32_t tmem = bars->tmem;
-    const uint32_t peer = rank ^ 1u;
+    const uint32_t peer = cluster_ctarank() ^ 1u;
 
     if (warp < PWARPS) {
         // ------------------------------------------------ gather producers ----
@@ -266,11 +293,11 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (rank == 0) gather_rows<KBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
+        if (role == 0) gather_rows<KBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
         else gather_rows<VBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
     } else if (warp < SWARP0 + 8) {
       regs_inc<REGS_SOFTMAX>();
-      if (rank == 0) {
+      if (role == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
         // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
         // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
@@ -466,6 +493,35 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             }
         }
         if (ok) ok = mbar_wait(&bars->ofinal, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+        if (p.fuse2) {
+            // Fused two-split merge, first half: once both value CTAs' gather
+            // regions are drained, each sends the columns that the other split
+            // finalises (split s finalises [256 s, +256)), unscaled, into the
+            // other's region; the weights need the final statistics, which
+            // are swapped afterwards.  Tiles of 32 heads x 32 columns are laid
+            // out [8 pieces][32 lanes][16 B], so that one remote store of a
+            // warp covers 512 contiguous bytes.
+            const uint32_t oth = cluster_ctarank() ^ 2u;
+            if (ok && sw == 0 && lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&bars->cfree), oth));
+            ok = __all_sync(0xffffffffu, ok) &&
+                 __all_sync(0xffffffffu, mbar_wait_cluster(&bars->cfree, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
+            if (ok) {
+                tc_fence_after();
+                const int send0 = (1 - w.split) * 256 + colhalf * 128;
+                const uint32_t rdst =
+                    mapa_shared(smem_u32(gbuf + (quarter * 2 + colhalf) * 4 * 4096 + lane * 16), oth);
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) {
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + send0 + j * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int ci = 0; ci < 8; ++ci)
+                        st_cluster_v4(rdst + j * 4096 + ci * 512, v[4 * ci], v[4 * ci + 1], v[4 * ci + 2], v[4 * ci + 3]);
+                }
+                mbar_arrive_remote(mapa_shared(smem_u32(&bars->crecv), oth));
+            }
+        }
         if (ok) ok = mbar_wait(&bars->statfull, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
         float m = -INFINITY, l = 0.f;
         if (ok) {
@@ -481,7 +537,76 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             const float lse = l > 0.f ? (m + log2f(l)) * LN2 : -INFINITY;
             uint8_t* stage = gbuf + sw * 2 * EPI_BUF;
             uint8_t* srow = stage + lane * 128;
-            if (p.splits == 1) {
+            if (p.fuse2) {
+                // Fused two-split merge, second half: swap the per-head
+                // statistics, then out = (a O_own + a' O_other) / (a l + a' l')
+                // on this split's columns, with a = 2^(m - max(m, m')).
+                const uint32_t oth = cluster_ctarank() ^ 2u;
+                if (colhalf == 0) {
+                    st_cluster_f32(mapa_shared(smem_u32(xbuf + h), oth), m);
+                    st_cluster_f32(mapa_shared(smem_u32(xbuf + H + h), oth), l);
+                    mbar_arrive_remote(mapa_shared(smem_u32(&bars->cstat), oth));
+                }
+                bool got = __all_sync(0xffffffffu,
+                                      mbar_wait_cluster(&bars->cstat, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
+                if (got) {
+                    const float mo = xbuf[h], lo = xbuf[H + h];
+                    const float mm = fmaxf(m, mo);
+                    const float a = m == -INFINITY ? 0.f : exp2f(m - mm);
+                    const float ao = mo == -INFINITY ? 0.f : exp2f(mo - mm);
+                    const float ll = a * l + ao * lo;
+                    const float so = ll > 0.f ? a / ll : 0.f, sr = ll > 0.f ? ao / ll : 0.f;
+                    const int keep0 = w.split * 256 + colhalf * 128;
+                    const int tile0 = (quarter * 2 + colhalf) * 4;     // this warp's 4 received tiles
+                    got = __all_sync(0xffffffffu,
+                                     mbar_wait_cluster(&bars->crecv, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
+                    if (got) {
+#pragma unroll 1
+                        for (int jj = 0; jj < 2; ++jj) {
+                            // bf16 tile of 32 heads x 64 columns, staged in the
+                            // received tile 2jj once the whole warp has read it
+                            uint8_t* tbuf = gbuf + (tile0 + 2 * jj) * 4096;
+#pragma unroll 1
+                            for (int e = 0; e < 2; ++e) {
+                                const int j = 2 * jj + e;
+                                float v[32];
+                                tmem_ld32(tmem + lane_base + keep0 + j * 32, v);
+                                tmem_ld_wait();
+                                const uint8_t* rrow = gbuf + (tile0 + j) * 4096 + lane * 16;
+#pragma unroll
+                                for (int ci = 0; ci < 8; ++ci) {
+                                    const uint4 x = ld_shared_v4(rrow + ci * 512);
+                                    v[4 * ci] = fmaf(v[4 * ci], so, __uint_as_float(x.x) * sr);
+                                    v[4 * ci + 1] = fmaf(v[4 * ci + 1], so, __uint_as_float(x.y) * sr);
+                                    v[4 * ci + 2] = fmaf(v[4 * ci + 2], so, __uint_as_float(x.z) * sr);
+                                    v[4 * ci + 3] = fmaf(v[4 * ci + 3], so, __uint_as_float(x.w) * sr);
+                                }
+                                if (e == 0) __syncwarp();                 // all lanes are done reading tile 2jj
+#pragma unroll
+                                for (int ci = 0; ci < 4; ++ci) {
+                                    uint32_t o[4];
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        const __nv_bfloat162 x =
+                                            __floats2bfloat162_rn(v[8 * ci + 2 * q], v[8 * ci + 2 * q + 1]);
+                                        o[q] = *(const uint32_t*)&x;
+                                    }
+                                    st_shared_v4(tbuf + lane * 128 + (((4 * e + ci) ^ (lane & 7)) << 4), o[0], o[1],
+                                                 o[2], o[3]);
+                                }
+                            }
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(&o_map, tbuf, keep0 + jj * 64, w.t * H + quarter * 32);
+                                bulk_commit_group();
+                            }
+                        }
+                        if (w.split == 0 && colhalf == 0)
+                            p.lse[(int64_t)w.t * H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
+                    }
+                }
+            } else if (p.splits == 1) {
                 // bf16 tiles of 32 heads x 64 columns
                 const int row0 = w.t * H + quarter * 32;
 #pragma unroll 1
@@ -551,7 +676,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
       if (warp == MWARP) {
         // ----------------------------------------------------- MMA issuer ----
         if (elect_one()) {
-            if (rank == 0) {
+            if (role == 0) {
                 constexpr uint32_t idesc = idesc_bf16_f32(H, NK, 0, 0);
                 const uint32_t kbase = smem_u32(gbuf);
                 bool ok = mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
@@ -593,7 +718,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                         }
                     }
                     mma_commit(&bars->empty[st]);
-                    mma_commit_multicast(&bars->pempty[pb], (uint16_t)0x3);
+                    mma_commit_multicast(&bars->pempty[pb], (uint16_t)(0x3u << (cluster_ctarank() & 2u)));
                     mma_commit(&bars->odone[pb]);
                 }
                 if (ok) mma_commit(&bars->ofinal);
@@ -656,6 +781,34 @@ int choose_splits(int rows, int k, int num_sms) {
     return s < 1 ? 1 : s;
 }
 
+// How many 4-CTA clusters of mla_tc_kernel can be resident at once on the
+// current device (0 if the query fails); looked up once per device.
+int max_active_quads() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(4);
+        cfg.blockDim = dim3(THREADS);
+        cfg.dynamicSmemBytes = MLA_SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 4;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev] = n > 0 ? n : -1;
+    }
+    return cache[dev] > 0 ? cache[dev] : 0;
+}
+
 }  // namespace
 
 bool mla_tc_supported(dsa_dtype_t dtype, int n_heads, int d_qk, int d_v) {
@@ -695,7 +848,13 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.part_o = nullptr;
     p.part_lse = nullptr;
-    if (p.splits > 1) {
+    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
+    if (e != cudaSuccess) return e;
+    // Two splits per row: merge them inside a 4-CTA cluster when all rows'
+    // clusters are resident in one wave (no partials in global memory, no
+    // merge launch); otherwise split partials go to the workspace.
+    p.fuse2 = (p.splits == 2 && rows <= max_active_quads()) ? 1 : 0;
+    if (p.splits > 1 && !p.fuse2) {
         const size_t need = (size_t)rows * p.splits * H * (DV + 1) * sizeof(float);
         if (!workspace || ws_bytes < need || (uintptr_t)workspace % 16) return cudaErrorInvalidValue;
         p.part_o = (float*)workspace;
@@ -706,14 +865,12 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     // as [rows*splits*128, 512] fp32 in boxes of 32 heads x 32 columns
     CUtensorMap q_map, o_map;
     bool ok = make_map_sw128(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DK, (uint64_t)rows * H, 64, H);
-    if (p.splits == 1)
+    if (p.splits == 1 || p.fuse2)
         ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, DV, (uint64_t)rows * H, 64, 32);
     else
         ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.part_o, DV,
                                   (uint64_t)rows * p.splits * H, 32, 32);
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
-    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2u * (unsigned)rows * (unsigned)p.splits);
     cfg.blockDim = dim3(THREADS);
@@ -721,7 +878,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.x = p.fuse2 ? 4 : 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -729,7 +886,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, q_map, o_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
-    if (p.splits > 1) {
+    if (p.splits > 1 && !p.fuse2) {
         mla_combine_kernel<<<dim3(rows, H), 128, 0, L.stream>>>(p.part_o, p.part_lse, p.splits,
                                                                (__nv_bfloat16*)out, lse);
         count_launch();

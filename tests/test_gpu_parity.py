@@ -116,6 +116,10 @@ def _random_idx(rows, k, ctx, g, pad=0):
     (workloads.DECODE_32K.with_(batch=3, rows=5, ctx=3000), 0),
     (workloads.DECODE_32K.with_(batch=2, rows=3, ctx=2500), 700),
     (workloads.DECODE_128K_FP8_PAGED.with_(batch=2, rows=2, ctx=4096), 13),
+    # two key splits per row, merged inside one 4-CTA cluster
+    (workloads.DECODE_32K.with_(batch=4, rows=32, ctx=4096), 0),
+    # same, with the second split of every row entirely unused slots
+    (workloads.DECODE_32K.with_(batch=3, rows=26, ctx=3000), 1500),
 ], ids=lambda x: getattr(x, "name", str(x)))
 def test_sparse_mla_on_given_indices(cuda_device, wl, pad):
     inp = workloads.generate(wl, parts=("mla",))
@@ -133,11 +137,13 @@ def test_sparse_mla_on_given_indices(cuda_device, wl, pad):
     assert lerr <= ATOL_LSE[wl.dtype], lerr
 
 
-@pytest.mark.parametrize("order", ["ascending", "descending", "shuffled"])
-def test_sparse_mla_running_max_moves(cuda_device, order):
+@pytest.mark.parametrize("order,rows", [("ascending", 3), ("descending", 3), ("shuffled", 3), ("ascending", 28)])
+def test_sparse_mla_running_max_moves(cuda_device, order, rows):
     """Scores that climb by many e-folds across the key list, so the running
-    maximum moves again and again (the lazy-rescale path of the kernel)."""
-    wl = workloads.DECODE_32K.with_(batch=2, rows=3, ctx=4096)
+    maximum moves again and again (the lazy-rescale path of the kernel).  With
+    28 rows each row's two key splits end with maxima far apart, which the
+    in-cluster merge of the splits must weigh."""
+    wl = workloads.DECODE_32K.with_(batch=2, rows=rows, ctx=4096)
     inp = workloads.generate(wl, parts=("mla",))
     q, kv = inp["q"].float(), inp["kv"].float()
     ramp = torch.arange(wl.ctx, dtype=torch.float32) * 0.02           # rope dims carry the ramp
