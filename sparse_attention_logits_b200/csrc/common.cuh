@@ -61,4 +61,22 @@ __device__ __forceinline__ uint32_t score_key(float f) {
 
 __host__ __device__ constexpr int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch.  The step's kernels are launched with the
+// programmatic-serialisation attribute, so the next kernel of the stream may
+// be scheduled while this one drains.  pdl_wait() blocks until every kernel
+// the grid depends on has completed and its writes are visible (a no-op when
+// launched without the attribute): nothing before it may read or write global
+// memory that another kernel touches.  pdl_launch_dependents() lets the next
+// kernel's CTAs start (they too wait before touching memory).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+inline cudaLaunchAttribute pdl_attr() {
+    cudaLaunchAttribute a;
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+    return a;
+}
+
 }  // namespace dsa

@@ -228,6 +228,8 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();                     // inputs written by earlier kernels are visible from here on
+    pdl_launch_dependents();
 
     Sched<NQ> sch;
     Unit un;
@@ -443,9 +445,17 @@ cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Para
     if (NQ == 1) units = (int64_t)p.rows * ((p.ctx + KT - 1) / KT);
     else units = (p.rows + NQ - 1) / NQ;
     const int grid = (int)(units < L.num_sms ? units : L.num_sms);
-    indexer_tc_kernel<NQ, FP8><<<grid, THREADS, C::SMEM, L.stream>>>(mk, mq, p);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, indexer_tc_kernel<NQ, FP8>, mk, mq, p);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace

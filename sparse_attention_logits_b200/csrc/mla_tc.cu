@@ -217,6 +217,8 @@ __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, u
 __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                                                           const __grid_constant__ CUtensorMap o_map,
                                                           const MlaParams p) {
+    pdl_wait();                     // the indices of the previous kernel are visible from here on
+    pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
@@ -740,6 +742,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
 __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
                                                           const float* __restrict__ part_lse, int splits,
                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    pdl_wait();
     const int t = blockIdx.x, h = blockIdx.y;
     const int d = threadIdx.x * 4;
     float mx = -INFINITY;
@@ -876,22 +879,30 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = MLA_SMEM;
     cfg.stream = L.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = p.fuse2 ? 4 : 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, q_map, o_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1 && !p.fuse2) {
-        mla_combine_kernel<<<dim3(rows, H), 128, 0, L.stream>>>(p.part_o, p.part_lse, p.splits,
-                                                               (__nv_bfloat16*)out, lse);
+        cudaLaunchConfig_t c2 = {};
+        c2.gridDim = dim3(rows, H);
+        c2.blockDim = dim3(128);
+        c2.stream = L.stream;
+        cudaLaunchAttribute a2[1] = {pdl_attr()};
+        c2.attrs = a2;
+        c2.numAttrs = 1;
+        e = cudaLaunchKernelEx(&c2, mla_combine_kernel, (const float*)p.part_o, (const float*)p.part_lse, p.splits,
+                               (__nv_bfloat16*)out, lse);
         count_launch();
     }
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dsa

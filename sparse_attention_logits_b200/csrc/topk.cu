@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* cand = cta_counts + 16;            // [CAND_CAP] candidate keys (rank 0's is used)
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
 
+    pdl_wait();                     // the scores of the previous kernel are visible from here on
+    pdl_launch_dependents();
     const int row = blockIdx.x / CL;
     const uint32_t rank = cl_rank<CL>();
     const int tid = threadIdx.x;
@@ -513,13 +515,14 @@ cudaError_t launch_cl(const Launch& L, const float* logits, int64_t ld, const in
     cfg.blockDim = dim3(TOPK_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = L.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr();
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<CL>, logits, ld, row_pos, ctx_len, k, idx);
     count_launch();
     return e;
