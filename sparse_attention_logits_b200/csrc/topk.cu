@@ -33,8 +33,8 @@ constexpr int SLICE_CAP = 40960;               // keys per CTA kept in shared me
 constexpr int MAX_PASSES = 3;                  // 11 + 10 + 10 bits: the range is exact after three passes
 constexpr int CAND_CAP = 1024;                 // candidates ranked directly after the first pass
 // hist, merged (scan scratch), one cluster-wide histogram per pass, scratch,
-// candidate buffer
-constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + CAND_CAP + 32) * 4;
+// candidate buffer, candidates' source CTAs, per-CTA counts (rank 0)
+constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 32 + 32) * 4;
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -119,9 +119,12 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* cl_hist = merged + NBINS;          // [MAX_PASSES][NBINS] cluster-wide histograms (rank 0 holds them)
     uint32_t* warp_sums = cl_hist + MAX_PASSES * NBINS;   // [33]
     uint32_t* shared_res = warp_sums + 40;       // digit, count above
-    uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers)
+    uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers), key range, and [4..7]: the
+                                                 // threshold, keys equal to it to take, this CTA's offsets (from rank 0)
     uint32_t* cand_n = cta_counts + 8;           // candidate count (rank 0's is used)
     uint32_t* cand = cta_counts + 16;            // [CAND_CAP] candidate keys (rank 0's is used)
+    uint32_t* cand_src = cand + CAND_CAP;        // [CAND_CAP] the CTA each candidate comes from (rank 0's)
+    uint32_t* cta_cnt = cand_src + CAND_CAP;     // [3][8] per-CTA keys above the bin, candidates > T, == T (rank 0's)
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
 
     pdl_wait();                     // the scores of the previous kernel are visible from here on
@@ -201,6 +204,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     if (CL > 1)
         for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
     if (tid == 0) *cand_n = 0u;
+    if (tid < 24) cta_cnt[tid] = 0u;
     __syncthreads();
     // the slice is padded with copies of its first key up to a multiple of 4
     // (cnt4), so that every walk below reads 16 bytes per lane
@@ -236,6 +240,10 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     }
     __syncthreads();
     uint32_t lo_key = shared_res[4], hi_key = shared_res[5], remaining = (uint32_t)k;
+    // candidate path: rank 0 hands every CTA its output offset and its share
+    // of the keys equal to the threshold, so no later cluster exchange is needed
+    bool offsets_known = false;
+    uint32_t eq_before_given = 0u, out_before_given = 0u;
 #pragma unroll 1
     for (int pass = 0; pass < MAX_PASSES && lo_key != hi_key; ++pass) {
         const uint32_t width = hi_key - lo_key;
@@ -300,7 +308,17 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
             // counting, for each candidate, the candidates above it.
             const uint32_t n_addr = CL > 1 ? mapa_shared(smem_u32(cand_n), 0u) : smem_u32(cand_n);
             const uint32_t c_addr = CL > 1 ? mapa_shared(smem_u32(cand), 0u) : smem_u32(cand);
+            const uint32_t s_addr = CL > 1 ? mapa_shared(smem_u32(cand_src), 0u) : smem_u32(cand_src);
             const int lane = tid & 31, warp = tid >> 5;
+            {
+                // this CTA's keys in bins above the chosen one: all of them are taken
+                uint32_t a = (2u * tid > bin ? hist[2 * tid] : 0u) + (2u * tid + 1u > bin ? hist[2 * tid + 1] : 0u);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                const uint32_t ab_addr =
+                    CL > 1 ? mapa_shared(smem_u32(cta_cnt + rank), 0u) : smem_u32(cta_cnt + rank);
+                if (lane == 0 && a) atom_add_cluster(ab_addr, a);
+            }
             for (int b0 = warp * 128; b0 < cnt; b0 += 128 * (TOPK_THREADS / 32)) {
                 const int i = b0 + 4 * lane;
                 uint32_t kq[4] = {0u, 0u, 0u, 0u};
@@ -317,7 +335,11 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                     uint32_t base = 0u;
                     if (lane == leader) base = atom_add_cluster(n_addr, (uint32_t)__popc(m));
                     base = __shfl_sync(0xffffffffu, base, leader);
-                    if (c_ok) st_cluster_u32(c_addr + 4u * (base + __popc(m & ((1u << lane) - 1u))), kq[u]);
+                    if (c_ok) {
+                        const uint32_t pos = 4u * (base + __popc(m & ((1u << lane) - 1u)));
+                        st_cluster_u32(c_addr + pos, kq[u]);
+                        st_cluster_u32(s_addr + pos, rank);
+                    }
                 }
             }
             cl_sync<CL>();                       // every candidate has landed in rank 0's buffer
@@ -336,16 +358,39 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                         shared_res[5] = remaining - gt;
                     }
                 }
+                __syncthreads();
+                // count each CTA's candidates above and equal to the threshold
+                const uint32_t t_key = shared_res[4];
+                if ((uint32_t)tid < nc) {
+                    const uint32_t key = cand[tid], src = cand_src[tid];
+                    if (key > t_key) atomicAdd(&cta_cnt[8 + src], 1u);
+                    else if (key == t_key) atomicAdd(&cta_cnt[16 + src], 1u);
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    // ranks own contiguous slices in position order: CTA r's
+                    // selected keys follow those of ranks < r
+                    const uint32_t rem_eq = shared_res[5];
+                    uint32_t eqb = 0u, outb = 0u;
+                    for (uint32_t r = 0; r < (uint32_t)CL; ++r) {
+                        const uint32_t dst = CL > 1 ? mapa_shared(smem_u32(cta_counts + 4), r) : smem_u32(cta_counts + 4);
+                        st_cluster_u32(dst, t_key);
+                        st_cluster_u32(dst + 4, rem_eq);
+                        st_cluster_u32(dst + 8, eqb);
+                        st_cluster_u32(dst + 12, outb);
+                        const uint32_t e = cta_cnt[16 + r];
+                        const uint32_t take = eqb >= rem_eq ? 0u : min(e, rem_eq - eqb);
+                        outb += cta_cnt[r] + cta_cnt[8 + r] + take;
+                        eqb += e;
+                    }
+                }
             }
-            cl_sync<CL>();
-            if (CL > 1 && rank != 0) {
-                const uint32_t r0 = mapa_shared(smem_u32(shared_res + 4), 0u);
-                lo_key = ld_cluster_u32(r0);
-                remaining = ld_cluster_u32(r0 + 4);
-            } else {
-                lo_key = shared_res[4];
-                remaining = shared_res[5];
-            }
+            cl_sync<CL>();                       // the last remote access of the kernel
+            lo_key = cta_counts[4];
+            remaining = cta_counts[5];
+            eq_before_given = cta_counts[6];
+            out_before_given = cta_counts[7];
+            offsets_known = true;
             hi_key = lo_key;
             break;
         }
@@ -390,8 +435,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     }
     __syncthreads();
     // CTA totals, and the counts of the cluster's lower-ranked CTAs
-    uint32_t eq_before_cta = 0, out_before_cta = 0;
-    if (CL > 1) {
+    uint32_t eq_before_cta = eq_before_given, out_before_cta = out_before_given;
+    if (CL > 1 && !offsets_known) {
         if (warp == 0) {
             uint32_t g = wgt[lane], e = weq[lane];
 #pragma unroll
@@ -486,7 +531,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         j += __shfl_sync(0xffffffffu, s_incl, 31);
         eq_seen += __shfl_sync(0xffffffffu, e_incl, 31);
     }
-    if (CL > 1) cl_sync<CL>();                   // peers are done reading our counts
+    if (CL > 1 && !offsets_known) cl_sync<CL>();   // peers are done reading our counts
 }
 
 namespace {
