@@ -8,6 +8,11 @@
  *   dsa_topk            per query row, the k best-scoring visible keys
  *   dsa_sparse_mla      MQA-mode MLA attention over the selected latent rows
  *
+ * and two variants of the last step for DeepSeek-V4's compressed attention:
+ *
+ *   csa_core_attention  CSA: the selected compressed entries plus a window of raw rows
+ *   hca_attention       HCA: dense attention over every visible heavily compressed entry
+ *
  * Conventions shared by every entry point
  *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
  *     never allocates or frees device memory; scratch space, where a step
@@ -80,13 +85,16 @@ DSA_API uint64_t dsa_launch_count(void);
  * Every m consecutive rows of a cache become one "super entry" (V4 CSA
  * summary: 4 tokens -> 1; "解密DeepSeek-V4 ..." section 4.3: average pooling or
  * a small network -- average pooling is what is built).  Used on both the
- * MLA latent cache (D = 576) and the indexer key cache (D = 128).
+ * MLA latent cache (D = 576) and the indexer key cache (D = 128), and with
+ * m = 128 for HCA ("DeepSeek-V4 技术报告深度解析": m' = 128).
  *
  *   src    [batch, len, dim]   of `dtype` (DSA_BF16 or DSA_FP32)
  *   dst    [batch, len/m, dim] of `dtype`
  * The sum is formed exactly (double precision) and rounded once to the
- * storage type, round-to-nearest-even.  len must be a multiple of m;
- * m in [1, 64]; src and dst must not overlap; both 16-byte aligned.
+ * storage type, round-to-nearest-even (exact as long as the m values of a
+ * column span fewer than about 45 binary orders of magnitude).  len must be
+ * a multiple of m; m in [1, 1024]; src and dst must not overlap; both
+ * 16-byte aligned.
  */
 DSA_API dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch, int len, int dim, int m,
                           void* dst, void* stream);
@@ -174,6 +182,64 @@ DSA_API size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d
 DSA_API dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype,
                             const int32_t* page_table, int page_size, int num_pages,
                             const int32_t* row_batch, const int32_t* idx, int k,
+                            int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
+                            float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * csa_core_attention -- CSA core attention with the window segment
+ * ("DeepSeek V4 发布：1.6T 参数、百万上下文…", section on CSA: the window KV
+ * and the compressed KV are concatenated and attended together; CSA
+ * pipeline "compress -> index selection -> core attention" in
+ * "DeepSeek-V4 技术报告深度解析").  Slot s of query row t holds
+ *   s <  k:            the selected compressed entry idx[t, s] of kv, exactly
+ *                      as in dsa_sparse_mla (-1 = unused slot);
+ *   k <= s < k+window: the raw (uncompressed) cache row
+ *                      p = win_pos[t] - window + 1 + (s - k) of kv_win,
+ *                      unused when p < 0,
+ * and attention runs over all used slots together:
+ *   out[t,h,:] = sum_s softmax_s(scale * q[t,h,:] . c_s[0:d_qk]) * c_s[0:d_v].
+ * A window row is not deduplicated against a compressed entry that covers
+ * it: the two are different vectors.
+ *
+ *   kv_win   [batch, win_len, d_qk] contiguous raw cache of dtype, 16-byte
+ *            aligned (the bf16 tensor-core path)
+ *   win_pos  [rows] int32 raw position of each query (its window ends there);
+ *            win_pos[t] >= win_len is skipped and reported by
+ *            dsa_get_device_error
+ *   window   rows per window, >= 0 (0: plain dsa_sparse_mla); k >= 0 and
+ *            k + window >= 1; idx may be NULL when k = 0
+ * Other arguments, layouts, results and errors are those of dsa_sparse_mla;
+ * the workspace is dsa_sparse_mla_workspace_size(rows, k + window, ...).
+ * The pages name no window size and no attention sink: the caller chooses
+ * the window, and no sink term is added.
+ */
+DSA_API dsa_status_t csa_core_attention(const void* q, const void* kv, dsa_dtype_t dtype,
+                            const int32_t* page_table, int page_size, int num_pages,
+                            const int32_t* row_batch, const int32_t* idx, int k,
+                            int rows, int batch, int ctx_len,
+                            const void* kv_win, const int32_t* win_pos, int win_len, int window,
+                            int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * hca_attention -- HCA, heavily compressed attention ("DeepSeek-V4
+ * 技术报告深度解析": m' = 128, no sparse selection; "DeepSeek V4 发布…": every
+ * query sees all compressed KV, dense attention).  Dense MQA attention over
+ * every visible entry of a compressed latent cache (from csa_compress with
+ * m = 128):
+ *   out[t,h,:] = sum_{s <= row_last[t]} softmax_s(scale * q[t,h,:] . c_s[0:d_qk]) * c_s[0:d_v]
+ * with c_s entry s of cache b = row_batch[t].
+ *
+ *   kv        [batch, ctx_len, d_qk] contiguous compressed cache
+ *   row_last  [rows] int32: last visible entry of each row (ctx_len - 1 in
+ *             decode; -1: none visible, out = 0 and lse = -inf); entries
+ *             past ctx_len - 1 are not read
+ * Other arguments, layouts and errors are those of dsa_sparse_mla; the
+ * workspace is dsa_sparse_mla_workspace_size(rows, ctx_len, ...).
+ */
+DSA_API dsa_status_t hca_attention(const void* q, const void* kv, dsa_dtype_t dtype,
+                            const int32_t* row_batch, const int32_t* row_last,
                             int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
                             float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);

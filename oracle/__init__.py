@@ -7,7 +7,9 @@ it imports nothing from the product.  All arithmetic lives in ``oracle.c``
 arrays and marshals arguments.
 
 Functions and the passages they follow are listed in the header of
-``oracle.c``.
+``oracle.c``.  The two variants of the attention step at the end of this
+module (CSA core attention with its window segment, HCA) are compositions of
+``sparse_mla``: they only rearrange caches and index lists.
 """
 from __future__ import annotations
 
@@ -213,3 +215,46 @@ def sparse_mla(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int,
                             _p(ids, _I32P), n, _p(out, _F64P), _p(lse, _F64P),
                             _p(probs, _F64P) if probs is not None else None)
     return out, lse, probs
+
+
+def csa_core_attention(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int, kv_win, win_pos, window: int,
+                       page_table=None):
+    """CSA core attention with the window segment ("DeepSeek V4 发布：1.6T 参数、
+    百万上下文…", CSA: the window KV and the compressed KV are concatenated and
+    take part in core attention together).  Slots are the selected compressed
+    entries idx[t] of kv followed by the raw rows win_pos[t]-window+1 ..
+    win_pos[t] of kv_win (negative positions unused).
+
+    Written as that concatenation: one cache [B, ctx + win_len, D] holding the
+    (de-paged) compressed cache then the raw cache, and one index list holding
+    the selected entries then ctx + the window positions; attention over it is
+    sparse_mla.  Returns (out [rows,H,D_V] f64, lse [rows,H] f64)."""
+    kva = torch.as_tensor(kv)
+    if page_table is not None:
+        pt = torch.as_tensor(page_table).long()
+        B = pt.shape[0]
+        kva = kva[pt.reshape(-1)].reshape(B, ctx, kva.shape[-1])
+    win = torch.as_tensor(kv_win)
+    assert win.dtype == kva.dtype and win.shape[0] == kva.shape[0]
+    comb = torch.cat([kva, win], dim=1)
+    rows = torch.as_tensor(q).shape[0]
+    pos = torch.as_tensor(win_pos).long().view(rows, 1)
+    wi = pos - window + 1 + torch.arange(window).view(1, -1)
+    wi = torch.where(wi >= 0, wi + ctx, torch.full_like(wi, -1))
+    parts = [] if idx is None else [torch.as_tensor(idx).long()]
+    full = torch.cat(parts + [wi], dim=1).to(torch.int32)
+    out, lse, _ = sparse_mla(q, comb, full, row_batch, scale, d_v, ctx + win.shape[1])
+    return out, lse
+
+
+def hca_attention(q, kv, row_batch, row_last, scale: float, d_v: int):
+    """HCA ("DeepSeek-V4 技术报告深度解析": m' = 128, no top-k selection;
+    "DeepSeek V4 发布…": each query sees all compressed KV): attention of row t
+    over entries 0..row_last[t] of the compressed cache kv [B, L, D], i.e.
+    sparse_mla with the index list 0..row_last[t].  Returns (out, lse)."""
+    L = torch.as_tensor(kv).shape[1]
+    last = torch.as_tensor(row_last).long().view(-1, 1)
+    ar = torch.arange(L).view(1, -1)
+    idx = torch.where(ar <= last, ar, torch.full_like(ar, -1)).to(torch.int32)
+    out, lse, _ = sparse_mla(q, kv, idx, row_batch, scale, d_v, L)
+    return out, lse

@@ -52,6 +52,10 @@ _SIGS = {
                               _f32, _vp, _vp, _vp, _sz, _vp]),
     "dsa_sparse_mla_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                       _i32, _f32, _vp, _vp, _vp]),
+    "csa_core_attention": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32,
+                                  _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+    "hca_attention": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
+                             _vp]),
     "dsa_get_device_error": (_i32, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -202,6 +206,66 @@ def sparse_mla(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: 
         _check(_lib.dsa_sparse_mla(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages, _ptr(row_batch),
                                    _ptr(idx), k, rows, B, ctx_len, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
                                    _ptr(workspace), wsb, _stream(dev)), "dsa_sparse_mla")
+    return out, lse
+
+
+def csa_core_attention(q: torch.Tensor, kv: torch.Tensor, idx: Optional[torch.Tensor], row_batch: torch.Tensor,
+                       scale: float, d_v: int, ctx_len: int, kv_win: torch.Tensor, win_pos: torch.Tensor, window: int,
+                       page_table: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """CSA core attention: the selected compressed entries idx of kv plus the
+    window of `window` raw rows of kv_win [B, win_len, d_qk] ending at
+    win_pos[t] (out [rows, H, d_v], lse [rows, H] fp32)."""
+    dev = _dev(q, kv, idx, row_batch, kv_win, win_pos, page_table, out, lse, workspace)
+    rows, H, DK = q.shape
+    k = 0 if idx is None else idx.shape[1]
+    if page_table is not None:
+        B = page_table.shape[0]
+        num_pages, page_size = kv.shape[0], kv.shape[1]
+    else:
+        B = kv.shape[0]
+        num_pages, page_size = 0, 0
+        if kv.shape[1] != ctx_len:
+            raise ValueError("kv.shape[1] != ctx_len")
+    if kv_win.shape[0] != B or kv_win.dtype != q.dtype:
+        raise ValueError("kv_win must be [B, win_len, d_qk] of q's dtype")
+    if out is None:
+        out = torch.empty((rows, H, d_v), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((rows, H), dtype=torch.float32, device=dev)
+    need = sparse_mla_workspace_size(rows, k + window, H, DK, d_v, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(_lib.csa_core_attention(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages,
+                                       _ptr(row_batch), _ptr(idx), k, rows, B, ctx_len, _ptr(kv_win), _ptr(win_pos),
+                                       kv_win.shape[1], window, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
+                                       _ptr(workspace), wsb, _stream(dev)), "csa_core_attention")
+    return out, lse
+
+
+def hca_attention(q: torch.Tensor, kv: torch.Tensor, row_batch: torch.Tensor, row_last: torch.Tensor, scale: float,
+                  d_v: int, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """HCA: dense attention of each row over entries 0..row_last[t] of the
+    compressed cache kv [B, L, d_qk] (out [rows, H, d_v], lse [rows, H] fp32)."""
+    dev = _dev(q, kv, row_batch, row_last, out, lse, workspace)
+    rows, H, DK = q.shape
+    B, L = kv.shape[0], kv.shape[1]
+    if out is None:
+        out = torch.empty((rows, H, d_v), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((rows, H), dtype=torch.float32, device=dev)
+    need = sparse_mla_workspace_size(rows, L, H, DK, d_v, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(_lib.hca_attention(_ptr(q), _ptr(kv), _dt(q), _ptr(row_batch), _ptr(row_last), rows, B, L, H, DK, d_v,
+                                  float(scale), _ptr(out), _ptr(lse), _ptr(workspace), wsb, _stream(dev)),
+               "hca_attention")
     return out, lse
 
 

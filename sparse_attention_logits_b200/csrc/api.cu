@@ -109,7 +109,7 @@ const char* dsa_last_error(void) { return g_last_error; }
 dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch, int len, int dim, int m, void* dst,
                           void* stream) {
     if (!src || !dst) return fail(DSA_ERR_INVALID_ARG, "csa_compress: null pointer");
-    if (batch < 0 || len < 0 || dim <= 0 || m < 1 || m > 64)
+    if (batch < 0 || len < 0 || dim <= 0 || m < 1 || m > 1024)
         return fail(DSA_ERR_INVALID_ARG, "csa_compress: bad sizes (batch=%d len=%d dim=%d m=%d)", batch, len, dim, m);
     if (len % m) return fail(DSA_ERR_INVALID_ARG, "csa_compress: len=%d not a multiple of m=%d", len, m);
     if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "csa_compress: dtype must be bf16 or fp32");
@@ -186,40 +186,97 @@ size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int
     return dsa::mla_tc_workspace_bytes(rows, k, sms);
 }
 
-dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
-                            int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
-                            int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
-                            void* workspace, size_t workspace_bytes, void* stream) {
-    if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 1 || n_heads <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk)
-        return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: bad sizes");
+}  // extern "C"
+
+namespace {
+
+// Shared body of dsa_sparse_mla, csa_core_attention and hca_attention: the
+// selected (or, with idx NULL, every visible) keys of kv, plus an optional
+// window segment of raw rows (x).
+dsa_status_t sparse_attention(const char* name, const void* q, const void* kv, dsa_dtype_t dtype,
+                              const int32_t* page_table, int page_size, int num_pages, const int32_t* row_batch,
+                              const int32_t* idx, int k, int rows, int batch, int ctx_len, int n_heads, int d_qk,
+                              int d_v, float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                              void* stream, const dsa::KvExtra& x) {
+    const int window = x.kv2 ? x.window : 0;
+    if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 0 || window < 0 || k + window < 1 || n_heads <= 0 ||
+        d_qk <= 0 || d_v <= 0 || d_v > d_qk)
+        return fail(DSA_ERR_INVALID_ARG, "%s: bad sizes", name);
+    if ((int64_t)batch * ctx_len >= ((int64_t)1 << 31) - 2 ||
+        (window > 0 && (int64_t)batch * x.len2 >= ((int64_t)1 << 31) - 2))
+        return fail(DSA_ERR_UNSUPPORTED, "%s: a cache holds more than 2^31 - 2 rows", name);
     if (rows == 0) return DSA_OK;
-    if (!q || !kv || !row_batch || !idx || !out || !lse) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: null pointer");
-    if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "dsa_sparse_mla: dtype must be bf16 or fp32");
+    if (!q || !kv || !row_batch || !out || !lse || (k > 0 && !idx && !x.row_last))
+        return fail(DSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (window > 0 && (!x.pos2 || x.len2 <= 0)) return fail(DSA_ERR_INVALID_ARG, "%s: window needs win_pos and win_len", name);
+    if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "%s: dtype must be bf16 or fp32", name);
     if (page_table) {
         if (page_size <= 0 || ctx_len % page_size)
-            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: ctx_len must be a multiple of page_size");
-        if (num_pages <= 0) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: num_pages must be positive with a page table");
+            return fail(DSA_ERR_INVALID_ARG, "%s: ctx_len must be a multiple of page_size", name);
+        if (num_pages <= 0) return fail(DSA_ERR_INVALID_ARG, "%s: num_pages must be positive with a page table", name);
     }
-    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: scale must be positive and finite");
+    if (!(scale > 0.f) || !(scale < 1e30f)) return fail(DSA_ERR_INVALID_ARG, "%s: scale must be positive and finite", name);
     const bool tc = dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v);
     if (!tc && !dsa::mla_simt_supported(d_qk, d_v, n_heads))
-        return fail(DSA_ERR_UNSUPPORTED, "dsa_sparse_mla: no kernel for d_qk=%d d_v=%d n_heads=%d", d_qk, d_v, n_heads);
+        return fail(DSA_ERR_UNSUPPORTED, "%s: no kernel for d_qk=%d d_v=%d n_heads=%d", name, d_qk, d_v, n_heads);
     dsa::Launch L;
     dsa_status_t st = make_launch(stream, &L);
     if (st != DSA_OK) return st;
     if (tc) {
-        if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16))
-            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: q, kv and out must be 16-byte aligned");
-        const size_t need = dsa::mla_tc_workspace_bytes(rows, k, L.num_sms);
+        if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || (window > 0 && !aligned(x.kv2, 16)))
+            return fail(DSA_ERR_INVALID_ARG, "%s: q, kv, the window cache and out must be 16-byte aligned", name);
+        const size_t need = dsa::mla_tc_workspace_bytes(rows, k + window, L.num_sms);
         if (need && (!workspace || workspace_bytes < need))
-            return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: workspace of %zu bytes needed", need);
+            return fail(DSA_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed", name, need);
         return cuda_status(dsa::launch_mla_tc(L, q, kv, page_table, page_size, num_pages, row_batch, idx, k, rows,
-                                              batch, ctx_len, scale, out, lse, workspace, workspace_bytes),
-                           "dsa_sparse_mla (tensor-core) launch");
+                                              batch, ctx_len, scale, out, lse, workspace, workspace_bytes, x),
+                           "sparse attention (tensor-core) launch");
     }
-    return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows, batch,
-                                            ctx_len, n_heads, d_qk, d_v, scale, out, lse),
-                       "dsa_sparse_mla launch");
+    return cuda_status(dsa::launch_mla_simt(L, q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows,
+                                            batch, ctx_len, n_heads, d_qk, d_v, scale, out, lse, x),
+                       "sparse attention launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
+                            int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
+                            int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    if (k < 1) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: bad sizes (k=%d)", k);
+    if (rows > 0 && !idx) return fail(DSA_ERR_INVALID_ARG, "dsa_sparse_mla: null pointer");
+    return sparse_attention("dsa_sparse_mla", q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k, rows,
+                            batch, ctx_len, n_heads, d_qk, d_v, scale, out, lse, workspace, workspace_bytes, stream,
+                            dsa::KvExtra());
+}
+
+dsa_status_t csa_core_attention(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
+                                int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k,
+                                int rows, int batch, int ctx_len, const void* kv_win, const int32_t* win_pos,
+                                int win_len, int window, int n_heads, int d_qk, int d_v, float scale, void* out,
+                                float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    if (window < 0 || (window > 0 && !kv_win)) return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: bad window");
+    if (rows > 0 && k > 0 && !idx) return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: null pointer");
+    dsa::KvExtra x;
+    x.kv2 = kv_win;
+    x.pos2 = win_pos;
+    x.len2 = win_len;
+    x.window = window;
+    return sparse_attention("csa_core_attention", q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k,
+                            rows, batch, ctx_len, n_heads, d_qk, d_v, scale, out, lse, workspace, workspace_bytes,
+                            stream, x);
+}
+
+dsa_status_t hca_attention(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* row_batch,
+                           const int32_t* row_last, int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
+                           float scale, void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    if (rows > 0 && !row_last) return fail(DSA_ERR_INVALID_ARG, "hca_attention: null pointer");
+    dsa::KvExtra x;
+    x.row_last = row_last;
+    return sparse_attention("hca_attention", q, kv, dtype, nullptr, 0, 0, row_batch, nullptr, ctx_len, rows, batch,
+                            ctx_len, n_heads, d_qk, d_v, scale, out, lse, workspace, workspace_bytes, stream, x);
 }
 
 dsa_status_t dsa_sparse_mla_noalloc(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,

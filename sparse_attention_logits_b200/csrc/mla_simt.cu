@@ -23,7 +23,10 @@ template <typename T, int QPL, int VPL>
 __global__ void __launch_bounds__(256) mla_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ kv, const int32_t* __restrict__ page_table, int page_size,
     int pages_per_seq, int num_pages, const int32_t* __restrict__ row_batch, const int32_t* __restrict__ idx, int k,
-    int batch, int ctx_len, int n_heads, float scale, T* __restrict__ out, float* __restrict__ lse, unsigned* err) {
+    int batch, int ctx_len, int n_heads, float scale, T* __restrict__ out, float* __restrict__ lse, unsigned* err,
+    const T* __restrict__ kv2, const int32_t* __restrict__ pos2, int len2, int window,
+    const int32_t* __restrict__ row_last) {
+    pdl_wait();
     constexpr int DK = QPL * 32, DV = VPL * 32;
     __shared__ float tile[MLA_SIMT_TILE][DK];
     __shared__ int valid[MLA_SIMT_TILE];
@@ -46,12 +49,26 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
     for (int i = 0; i < VPL; ++i) acc[i] = 0.f;
     float m = -INFINITY, l = 0.f;
 
-    const int32_t* sel = idx + (int64_t)t * k;
-    for (int j0 = 0; j0 < k; j0 += MLA_SIMT_TILE) {
+    const int32_t* sel = idx ? idx + (int64_t)t * k : nullptr;
+    const int last = idx ? 0 : row_last[t];
+    const int wpos = window > 0 ? pos2[t] : 0;
+    const int ktot = k + window;
+    for (int j0 = 0; j0 < ktot; j0 += MLA_SIMT_TILE) {
         __syncthreads();
-        // gather up to 16 selected rows (warp w loads rows w and w+8)
+        // gather up to 16 slots (warp w loads slots w and w+8): selected keys
+        // (or every visible key in dense mode), then the window rows
         for (int r = warp; r < MLA_SIMT_TILE; r += 8) {
-            int s = j0 + r < k ? sel[j0 + r] : -1;
+            const int j = j0 + r;
+            if (j >= k && j < ktot) {
+                const int s = wpos - window + 1 + (j - k);
+                const bool ok = row_ok && s >= 0 && s < len2;
+                if (s >= len2) record_error(err, DEV_ERR_BAD_INDEX);
+                const int64_t row = (int64_t)b * len2 + s;
+                for (int d = lane; d < DK; d += 32) tile[r][d] = ok ? to_f32(kv2[row * DK + d]) : 0.f;
+                if (lane == 0) valid[r] = ok;
+                continue;
+            }
+            int s = j < k ? (sel ? sel[j] : (j <= last ? j : -1)) : -1;
             bool ok = row_ok && s >= 0 && s < ctx_len;
             if (s >= ctx_len) record_error(err, DEV_ERR_BAD_INDEX);
             int64_t row = 0;
@@ -97,22 +114,29 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
 template <typename T, int QPL, int VPL>
 static cudaError_t launch_t(const Launch& L, const void* q, const void* kv, const int32_t* pt, int page_size,
                             int pages_per_seq, int num_pages, const int32_t* rb, const int32_t* idx, int k, int rows, int batch,
-                            int ctx, int H, float scale, void* out, float* lse) {
-    dim3 grid(rows, H / MLA_SIMT_HEADS);
-    mla_simt_kernel<T, QPL, VPL><<<grid, 256, 0, L.stream>>>((const T*)q, (const T*)kv, pt, page_size, pages_per_seq, num_pages,
-                                                             rb, idx, k, batch, ctx, H, scale, (T*)out, lse, L.err);
+                            int ctx, int H, float scale, void* out, float* lse, const KvExtra& x) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows, H / MLA_SIMT_HEADS);
+    cfg.blockDim = dim3(256);
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_simt_kernel<T, QPL, VPL>, (const T*)q, (const T*)kv, pt, page_size,
+                                             pages_per_seq, num_pages, rb, idx, k, batch, ctx, H, scale, (T*)out, lse,
+                                             L.err, (const T*)x.kv2, x.pos2, x.len2, x.kv2 ? x.window : 0, x.row_last);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 template <typename T>
 static cudaError_t launch_dims(const Launch& L, const void* q, const void* kv, const int32_t* pt, int page_size,
                                int pps, int npages, const int32_t* rb, const int32_t* idx, int k, int rows, int batch, int ctx,
-                               int H, int dqk, int dv, float scale, void* out, float* lse) {
-    if (dqk == 32 && dv == 32) return launch_t<T, 1, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 64 && dv == 64) return launch_t<T, 2, 2>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 64 && dv == 32) return launch_t<T, 2, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
-    if (dqk == 576 && dv == 512) return launch_t<T, 18, 16>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse);
+                               int H, int dqk, int dv, float scale, void* out, float* lse, const KvExtra& x) {
+    if (dqk == 32 && dv == 32) return launch_t<T, 1, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse, x);
+    if (dqk == 64 && dv == 64) return launch_t<T, 2, 2>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse, x);
+    if (dqk == 64 && dv == 32) return launch_t<T, 2, 1>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse, x);
+    if (dqk == 576 && dv == 512) return launch_t<T, 18, 16>(L, q, kv, pt, page_size, pps, npages, rb, idx, k, rows, batch, ctx, H, scale, out, lse, x);
     return cudaErrorInvalidValue;
 }
 
@@ -123,14 +147,15 @@ bool mla_simt_supported(int d_qk, int d_v, int n_heads) {
 
 cudaError_t launch_mla_simt(const Launch& L, const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
                             int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
-                            int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse) {
+                            int ctx_len, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
+                            const KvExtra& x) {
     if (rows == 0) return cudaSuccess;
     const int pps = page_table ? ctx_len / page_size : 0;
     if (dtype == DSA_FP32)
         return launch_dims<float>(L, q, kv, page_table, page_size, pps, num_pages, row_batch, idx, k, rows, batch, ctx_len,
-                                  n_heads, d_qk, d_v, scale, out, lse);
+                                  n_heads, d_qk, d_v, scale, out, lse, x);
     return launch_dims<__nv_bfloat16>(L, q, kv, page_table, page_size, pps, num_pages, row_batch, idx, k, rows, batch,
-                                      ctx_len, n_heads, d_qk, d_v, scale, out, lse);
+                                      ctx_len, n_heads, d_qk, d_v, scale, out, lse, x);
 }
 
 }  // namespace dsa

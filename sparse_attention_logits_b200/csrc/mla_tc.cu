@@ -104,14 +104,18 @@ struct MlaParams {
     const __nv_bfloat16* kv;
     const int32_t* page_table;
     const int32_t* row_batch;
-    const int32_t* idx;
+    const int32_t* idx;             // [rows, k]; NULL: dense mode (slot s is key s up to row_last[t])
+    const int32_t* row_last;
+    const __nv_bfloat16* kv2;       // window segment: raw cache [batch, len2, DK]
+    const int32_t* pos2;            // [rows] raw position of each query
+    int len2, window;
     __nv_bfloat16* out;
     float* lse;
     float* part_o;                  // [rows, splits, H, DV] when splits > 1
     float* part_lse;                // [rows, splits, H]
     unsigned* err;
     int page_size, pages_per_seq, num_pages;
-    int k, rows, batch, ctx, splits, per_split;
+    int k, ktot, rows, batch, ctx, splits, per_split;   // ktot = k + window slots per row
     int fuse2;                      // two key splits per row in one 4-CTA cluster, merged in the kernel
     float scale_log2;
 };
@@ -127,18 +131,43 @@ __device__ __forceinline__ Work work_of(const MlaParams& p) {
     w.t = item / p.splits;
     w.split = item - w.t * p.splits;
     w.slot0 = w.split * p.per_split;
-    w.slot_end = min(p.k, w.slot0 + p.per_split);
+    w.slot_end = min(p.ktot, w.slot0 + p.per_split);
     w.nchunks = (w.slot_end - w.slot0 + NK - 1) / NK;
     w.b = __ldg(p.row_batch + w.t);
     w.b_ok = w.b >= 0 && w.b < p.batch;
     return w;
 }
 
-// Cache row of key position s (or -1 if the slot is unused / invalid).
+// Key position held by slot `slot` of this row (-1: unused), before range
+// checks: selected (or, in dense mode, every visible) key for slot < k, raw
+// window position for k <= slot < ktot.
+// EXT = false compiles the plain selected-rows path (no window, no dense
+// mode) exactly as lean as it was before those existed.
+template <bool EXT>
+__device__ __forceinline__ int slot_key(const MlaParams& p, const Work& w, int slot) {
+    if (!EXT) return __ldg(p.idx + (int64_t)w.t * p.k + slot);
+    if (slot < p.k) {
+        if (p.idx) return __ldg(p.idx + (int64_t)w.t * p.k + slot);
+        return slot <= __ldg(p.row_last + w.t) ? slot : -1;
+    }
+    const int s = __ldg(p.pos2 + w.t) - p.window + 1 + (slot - p.k);
+    return s < 0 ? -1 : s;
+}
+
+// Row to gather for a slot: >= 0 a row of kv, <= -2 the row -2 - r of the
+// window cache kv2, -1 nothing (unused or invalid slot; the copy writes zeros).
+template <bool EXT>
 __device__ __forceinline__ int64_t key_row(const MlaParams& p, const Work& w, int slot) {
     if (!w.b_ok || slot >= w.slot_end) return -1;
-    const int s = __ldg(p.idx + (int64_t)w.t * p.k + slot);
+    const int s = slot_key<EXT>(p, w, slot);
     if (s < 0) return -1;
+    if (EXT && slot >= p.k) {
+        if (s >= p.len2) {
+            record_error(p.err, DEV_ERR_BAD_INDEX);
+            return -1;
+        }
+        return -2 - ((int64_t)w.b * p.len2 + s);
+    }
     if (s >= p.ctx) {
         record_error(p.err, DEV_ERR_BAD_INDEX);
         return -1;
@@ -162,9 +191,19 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-// Raw key position stored in a slot (-1 past the end of this split's slots).
+// Key position of a slot for the softmax's validity mask (-1 past the end of
+// this split's slots).  It is loaded one chunk ahead and only compared (with
+// slot_limit) in the next iteration, so the load latency stays hidden.
+template <bool EXT>
 __device__ __forceinline__ int slot_index(const MlaParams& p, const Work& w, int slot) {
-    return slot < w.slot_end ? __ldg(p.idx + (int64_t)w.t * p.k + slot) : -1;
+    return slot < w.slot_end ? slot_key<EXT>(p, w, slot) : -1;
+}
+
+// Exclusive bound of valid key positions for a slot: the same decision as
+// key_row, without its error reports and page lookups.
+template <bool EXT>
+__device__ __forceinline__ int slot_limit(const MlaParams& p, int slot) {
+    return !EXT || slot < p.k ? p.ctx : p.len2;
 }
 
 // Stores into another CTA's shared memory (cluster address from mapa).
@@ -185,35 +224,41 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 
 // consecutive 16-byte pieces.  Many producer warps are used because the copy
 // throughput of an SM grows with the number of copies its threads keep in
 // flight.
-template <int NB>   // dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
+template <int NB, bool EXT>   // NB: dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
 __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, Bars* bars, int warp,
                                             int lane, volatile int* abort_flag) {
     constexpr int RC = NB * 8;                           // 16-byte pieces per row
     const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
-    int64_t next_row = key_row(p, w, w.slot0 + my_slot);
+    int64_t next_row = key_row<EXT>(p, w, w.slot0 + my_slot);
     // score CTA: the region holds the Q tile until it has been moved to TMEM
     if (NB == KBLK && !mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)) return;
     for (int c = 0; c < w.nchunks; ++c) {
         const int st = c & 1;
         if (!mbar_wait(&bars->empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
-        const int myrow_lo = (int)(next_row >= 0 ? next_row : -1);  // row indices fit in 31 bits
+        const int myrow_lo = (int)next_row;     // row indices (and the window encoding) fit in 31 bits
         uint8_t* base = gbuf + (size_t)st * KSTAGE;
 #pragma unroll
         for (int i = lane; i < ROWS_PER_PW * RC; i += 32) {
             const int rl = i / RC, ci = i - rl * RC;
             const int row = __shfl_sync(0xffffffffu, myrow_lo, rl);
             const int r = warp * ROWS_PER_PW + rl;
-            const __nv_bfloat16* src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8 : p.kv;
-            cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row >= 0 ? 16u : 0u);
+            const __nv_bfloat16* src;
+            if (EXT)
+                src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8
+                    : row <= -2 ? p.kv2 + (int64_t)(-2 - row) * DK + ci * 8 : p.kv;
+            else
+                src = row >= 0 ? p.kv + (int64_t)row * DK + ci * 8 : p.kv;
+            cp_async_16(base + (ci >> 3) * (NK * 128) + sw128(r, ci & 7), src, row != -1 ? 16u : 0u);
         }
         cp_async_arrive_noinc(&bars->full[st]);
         // look up the next chunk's row while this chunk's copies are in flight
-        if (c + 1 < w.nchunks) next_row = key_row(p, w, w.slot0 + (c + 1) * NK + my_slot);
+        if (c + 1 < w.nchunks) next_row = key_row<EXT>(p, w, w.slot0 + (c + 1) * NK + my_slot);
     }
 }
 
 }  // namespace
 
+template <bool EXT>
 __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                                                           const __grid_constant__ CUtensorMap o_map,
                                                           const MlaParams p) {
@@ -295,8 +340,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (role == 0) gather_rows<KBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
-        else gather_rows<VBLK>(p, w, gbuf, bars, warp, lane, abort_flag);
+        if (role == 0) gather_rows<KBLK, EXT>(p, w, gbuf, bars, warp, lane, abort_flag);
+        else gather_rows<VBLK, EXT>(p, w, gbuf, bars, warp, lane, abort_flag);
     } else if (warp < SWARP0 + 8) {
       regs_inc<REGS_SOFTMAX>();
       if (role == 0) {
@@ -338,11 +383,13 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
         // whether this lane's key of a chunk is real: the raw index is loaded
         // one chunk ahead and only inspected in the next iteration
-        int s_next = slot_index(p, w, w.slot0 + 32 * half + lane);
+        int s_next = slot_index<EXT>(p, w, w.slot0 + 32 * half + lane);
         for (int c = 0; c < w.nchunks; ++c) {
             const int sb = c & 1, par = c & 1;
-            const uint32_t vmask = __ballot_sync(0xffffffffu, w.b_ok && s_next >= 0 && s_next < p.ctx);
-            if (c + 1 < w.nchunks) s_next = slot_index(p, w, w.slot0 + (c + 1) * NK + 32 * half + lane);
+            const uint32_t vmask = __ballot_sync(
+                0xffffffffu,
+                w.b_ok && s_next >= 0 && s_next < slot_limit<EXT>(p, w.slot0 + c * NK + 32 * half + lane));
+            if (c + 1 < w.nchunks) s_next = slot_index<EXT>(p, w, w.slot0 + (c + 1) * NK + 32 * half + lane);
             float sv[32];
             if (ok)
                 ok = __all_sync(0xffffffffu,
@@ -803,7 +850,10 @@ int max_active_quads() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel, &cfg) != cudaSuccess) {
+        // both kernel variants have the same shape; the attribute must be set on the one queried
+        if (cudaFuncSetAttribute(mla_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<false>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -826,7 +876,8 @@ size_t mla_tc_workspace_bytes(int rows, int k, int num_sms) {
 
 cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
                           int num_pages, const int32_t* row_batch, const int32_t* idx, int k, int rows, int batch,
-                          int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes) {
+                          int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
+                          const KvExtra& x) {
     if (rows == 0) return cudaSuccess;
     MlaParams p;
     p.q = (const __nv_bfloat16*)q;
@@ -834,6 +885,11 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.page_table = page_table;
     p.row_batch = row_batch;
     p.idx = idx;
+    p.row_last = x.row_last;
+    p.kv2 = (const __nv_bfloat16*)x.kv2;
+    p.pos2 = x.pos2;
+    p.len2 = x.len2;
+    p.window = x.kv2 ? x.window : 0;
     p.out = (__nv_bfloat16*)out;
     p.lse = lse;
     p.err = L.err;
@@ -841,17 +897,20 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.pages_per_seq = page_table ? ctx_len / page_size : 0;
     p.num_pages = page_table ? num_pages : 0;
     p.k = k;
+    p.ktot = k + p.window;
     p.rows = rows;
     p.batch = batch;
     p.ctx = ctx_len;
-    p.splits = choose_splits(rows, k, L.num_sms);
-    const int per = (k + p.splits - 1) / p.splits;
+    p.splits = choose_splits(rows, p.ktot, L.num_sms);
+    const int per = (p.ktot + p.splits - 1) / p.splits;
     p.per_split = (per + NK - 1) / NK * NK;
-    p.splits = (k + p.per_split - 1) / p.per_split;            // no empty split
+    p.splits = (p.ktot + p.per_split - 1) / p.per_split;       // no empty split
     p.scale_log2 = scale * 1.4426950408889634f;
     p.part_o = nullptr;
     p.part_lse = nullptr;
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
+    const bool ext = p.window > 0 || !p.idx;
+    auto kern = ext ? mla_tc_kernel<true> : mla_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
     if (e != cudaSuccess) return e;
     // Two splits per row: merge them inside a 4-CTA cluster when all rows'
     // clusters are resident in one wave (no partials in global memory, no
@@ -887,7 +946,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, mla_tc_kernel, q_map, o_map, p);
+    e = cudaLaunchKernelEx(&cfg, kern, q_map, o_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1 && !p.fuse2) {

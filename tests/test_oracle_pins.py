@@ -360,3 +360,81 @@ def test_csa_with_m1_is_dsa():
     a = oracle.index_scores(inp["q_idx"], inp["w"], inp["k_idx"], inp["row_batch"], inp["row_pos"])
     b = oracle.index_scores(inp["q_idx"], inp["w"], k1, inp["row_batch"], inp["row_pos"])
     assert np.array_equal(a, b)
+
+
+# ------------------------------------------- CSA window and HCA (NEXT rows) ----
+
+def _brute_attention(q, vecs, scale, d_v):
+    """softmax(scale * q . c) @ c[:d_v] for one row: q [H, D], vecs [n, D] (n >= 1)."""
+    z = scale * (q @ vecs.T)                                   # [H, n]
+    p = scipy.special.softmax(z, axis=1)
+    return p @ vecs[:, :d_v], scipy.special.logsumexp(z, axis=1)
+
+
+def test_csa_core_attention_is_attention_over_the_concatenated_keys():
+    g = torch.Generator().manual_seed(31)
+    B, Lc, Lr, H, D, dv, k, W = 2, 20, 80, 3, 12, 8, 5, 6
+    q = torch.randn(5, H, D, generator=g)
+    kv = torch.randn(B, Lc, D, generator=g)
+    raw = torch.randn(B, Lr, D, generator=g)
+    rb = torch.tensor([0, 1, 1, 0, 1], dtype=torch.int32)
+    pos = torch.tensor([79, 40, 3, 0, 5], dtype=torch.int32)      # rows 2-4: window clipped at position 0
+    idx = torch.stack([torch.randperm(Lc, generator=g)[:k] for _ in range(5)]).to(torch.int32)
+    idx[1, 2] = -1
+    out, lse = oracle.csa_core_attention(q, kv, idx, rb, 0.4, dv, Lc, raw, pos, W)
+    for t in range(5):
+        b = int(rb[t])
+        sel = [kv[b, int(s)] for s in idx[t] if s >= 0]
+        win = [raw[b, p] for p in range(int(pos[t]) - W + 1, int(pos[t]) + 1) if p >= 0]
+        vecs = torch.stack(sel + win).double().numpy()
+        ro, rl = _brute_attention(q[t].double().numpy(), vecs, 0.4, dv)
+        np.testing.assert_allclose(out[t], ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[t], rl, rtol=0, atol=1e-12)
+    # a window of 0 rows is plain sparse attention; no selected entries leaves the window alone
+    o0, l0 = oracle.csa_core_attention(q, kv, idx, rb, 0.4, dv, Lc, raw, pos, 0)
+    so, sl, _ = oracle.sparse_mla(q, kv, idx, rb, 0.4, dv, Lc)
+    np.testing.assert_allclose(o0, so, rtol=0, atol=0)
+    ow, lw = oracle.csa_core_attention(q, kv, None, rb, 0.4, dv, Lc, raw, pos, W)
+    t = 0
+    ro, rl = _brute_attention(q[t].double().numpy(), raw[0, 74:80].double().numpy(), 0.4, dv)
+    np.testing.assert_allclose(ow[t], ro, rtol=0, atol=1e-12)
+
+
+def test_csa_core_attention_paged_equals_contiguous():
+    g = torch.Generator().manual_seed(32)
+    B, Lc, page, H, D = 2, 16, 4, 2, 8
+    kv = torch.randn(B, Lc, D, generator=g)
+    raw = torch.randn(B, 30, D, generator=g)
+    q = torch.randn(3, H, D, generator=g)
+    rb = torch.tensor([1, 0, 1], dtype=torch.int32)
+    pos = torch.tensor([29, 10, 2], dtype=torch.int32)
+    idx = torch.stack([torch.randperm(Lc, generator=g)[:6] for _ in range(3)]).to(torch.int32)
+    perm = torch.randperm(B * Lc // page, generator=g)
+    pages = torch.empty(B * Lc // page, page, D)
+    pages[perm] = kv.reshape(-1, page, D)
+    table = perm.view(B, Lc // page).to(torch.int32)
+    a, la = oracle.csa_core_attention(q, kv, idx, rb, 0.5, 8, Lc, raw, pos, 4)
+    p, lp = oracle.csa_core_attention(q, pages, idx, rb, 0.5, 8, Lc, raw, pos, 4, page_table=table)
+    np.testing.assert_allclose(p, a, rtol=0, atol=0)
+    np.testing.assert_allclose(lp, la, rtol=0, atol=0)
+
+
+def test_hca_attention_is_dense_attention_over_visible_blocks():
+    g = torch.Generator().manual_seed(33)
+    m, B, Lraw, H, D, dv = 128, 2, 1024, 2, 16, 16
+    raw = torch.randn(B, Lraw, D, generator=g).to(torch.bfloat16)
+    kvc_bits = oracle.csa_compress(raw, m)                      # [B, 8, D] bf16 codes
+    kvc = torch.from_numpy(kvc_bits.view(np.int16)).view(torch.bfloat16)
+    # the pooled entry is the mean of its 128 raw rows, rounded once
+    mean = raw[1, 3 * m:4 * m].double().mean(0)
+    assert torch.equal(kvc[1, 3], mean.to(torch.bfloat16))
+    q = torch.randn(4, H, D, generator=g).to(torch.bfloat16)
+    rb = torch.tensor([0, 1, 1, 0], dtype=torch.int32)
+    last = torch.tensor([7, 7, 2, -1], dtype=torch.int32)       # decode, decode, causal prefix, nothing visible
+    out, lse = oracle.hca_attention(q, kvc, rb, last, 0.25, dv)
+    for t in range(3):
+        vecs = kvc[int(rb[t]), :int(last[t]) + 1].double().numpy()
+        ro, rl = _brute_attention(q[t].double().numpy(), vecs, 0.25, dv)
+        np.testing.assert_allclose(out[t], ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[t], rl, rtol=0, atol=1e-12)
+    assert np.all(out[3] == 0) and np.all(np.isneginf(lse[3]))
