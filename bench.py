@@ -249,20 +249,24 @@ def _graph(fn):
     return g
 
 
-def time_graph(g, steps, device, flush=None):
+def time_graph(g, steps, device, flush=None, flush_read=None):
     """Replay `g` `steps` times, each bracketed by CUDA events on the current
     stream; with `flush` (a buffer larger than L2) it is written before each
     replay, outside the events.  Returns the mean device time of one replay
     in ms.  Without `flush` the inputs themselves must exceed L2: a written
     flush leaves L2 full of dirty lines whose write-back would then be
-    charged to the next replay."""
+    charged to the next replay.  `flush_read` (a buffer larger than L2) is
+    instead read before each replay, which evicts L2 without dirtying it."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(device)
     torch.cuda.synchronize(device)
+    sink = torch.empty((), dtype=torch.float32, device=device)
     for a, b in evs:
         if flush is not None:
             flush.zero_()
+        if flush_read is not None:
+            torch.sum(flush_read, dim=0, out=sink)
         a.record()
         g.replay()
         b.record()
@@ -519,6 +523,8 @@ def run_ours(args):
     }
     if args.prefill:
         result["prefill"] = run_prefill(dsa, workloads, device, peaks, args)
+    if args.v4:
+        result["v4_variants"] = run_v4_variants(dsa, workloads, device, peaks, args)
     if world == 1 and rank == 0 and args.cpu_baseline:
         qps, n, cores, secs = cpu_baseline_decode(wl, inp)
         result["cpu_baseline"] = {"value": round(qps, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
@@ -552,6 +558,109 @@ def run_prefill(dsa, workloads, device, peaks, args):
                          "algorithmic_flops": fl_m},
             "indexer_roofline": {"bound": "tensor", "achieved": round(idx_t, 1), "peak": pk, "unit": "TFLOP/s",
                                  "frac": round(idx_t / pk, 4), "algorithmic_flops": fl_i}}
+
+
+V4_WINDOW = 128       # raw rows in the CSA window (the pages give no size)
+HCA_M = 128           # HCA pooling factor m'
+
+
+def run_v4_variants(dsa, workloads, device, peaks, args):
+    """DeepSeek-V4's two compressed-attention variants at the 1M-token CSA
+    shapes (4 sequences of 1,048,576 raw tokens, one new query each):
+
+    csa_step: pooled indexer keys -> top-1024 pooled entries -> CSA core
+      attention over those entries plus a window of the last 128 raw rows.
+      The pooling itself (csa_compress) runs once per 4 new tokens in a real
+      cache and is not part of the step.
+    hca: dense attention of each query over all 8,192 entries of the 128:1
+      pooled latent cache (pooling again outside the step).
+    Each is captured in a CUDA graph and timed like the main step; the
+    roofline is HBM bytes (what must be read once) over the event time."""
+    import torch
+    rank, world, _ = dist_env()
+    wl = workloads.CSA_DECODE_1M
+    inp = workloads.generate(wl, device=device, seed=200 + rank)
+    raw_kv = inp["kv"]
+    k_c = dsa.csa_compress(inp["k_idx"], wl.compress_m)
+    kv_c = dsa.csa_compress(raw_kv, wl.compress_m)
+    del inp["k_idx"]
+    rows, ctx = wl.rows, wl.ctx
+    logits = torch.empty((rows, ctx), dtype=torch.float32, device=device)
+    idx = torch.empty((rows, wl.topk), dtype=torch.int32, device=device)
+    n = dsa.topk_workspace_size(rows, ctx, wl.topk)
+    tws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    n = dsa.sparse_mla_workspace_size(rows, wl.topk + V4_WINDOW, wl.heads, wl.d_qk, wl.d_v, torch.bfloat16)
+    mws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    out = torch.empty((rows, wl.heads, wl.d_v), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((rows, wl.heads), dtype=torch.float32, device=device)
+    win_pos = torch.full((rows,), wl.raw_ctx - 1, dtype=torch.int32, device=device)
+
+    class Csa:
+        def run_one(self, name):
+            if name == "dsa_indexer_logits":
+                dsa.indexer_logits(inp["q_idx"], inp["w"], k_c, inp["row_batch"], inp["row_pos"], out=logits)
+            elif name == "dsa_topk":
+                dsa.topk(logits, inp["row_pos"], wl.topk, ctx_len=ctx, out=idx, workspace=tws)
+            else:
+                dsa.csa_core_attention(inp["q"], kv_c, idx, inp["row_batch"], wl.softmax_scale, wl.d_v, ctx, raw_kv,
+                                       win_pos, V4_WINDOW, out=out, lse=lse, workspace=mws)
+
+        def run(self):
+            for nm in ("dsa_indexer_logits", "dsa_topk", "csa_core_attention"):
+                self.run_one(nm)
+
+    st = Csa()
+    st.dsa = dsa
+    g = _graph(st.run)
+    for _ in range(3):
+        g.replay()
+    steps = max(5, args.steps)
+    ms = max_over_ranks(time_graph(g, steps, device), device)
+    del g
+    # alone, the gathered rows (5 MB) would stay in L2 between replays: read
+    # a 256 MB buffer before each one
+    evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    ga = _graph(lambda: st.run_one("csa_core_attention"))
+    ga.replay()
+    ms_attn = time_graph(ga, steps, device, flush_read=evict)
+    del ga
+    sel_rows = rows * (wl.topk + V4_WINDOW)
+    step_bytes = (indexer_bytes(wl) + sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2)
+    attn_bytes = sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2
+    csa = {"workload": f"{wl.name}+window{V4_WINDOW}", "value": round(rows * world / (ms / 1e3), 1),
+           "unit": "queries/s", "ms_per_step": round(ms, 4), "core_attention_ms": round(ms_attn, 4),
+           "roofline": {"bound": "hbm", "achieved": round(step_bytes / (ms / 1e3) / 1e9, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "algorithmic_bytes": step_bytes},
+           "core_attention_bytes": attn_bytes,
+           "l2": "step: pooled keys (268 MB) exceed L2, no flush; core attention alone: 256 MB read between replays"}
+    del logits, idx, tws, k_c, kv_c
+    # HCA over the 128:1 pooled cache
+    kv_h = dsa.csa_compress(raw_kv, HCA_M)
+    del raw_kv, inp["kv"]
+    torch.cuda.empty_cache()
+    L_h = kv_h.shape[1]
+    last = torch.full((rows,), L_h - 1, dtype=torch.int32, device=device)
+    n = dsa.sparse_mla_workspace_size(rows, L_h, wl.heads, wl.d_qk, wl.d_v, torch.bfloat16)
+    hws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
+    gh = _graph(lambda: dsa.hca_attention(inp["q"], kv_h, inp["row_batch"], last, wl.softmax_scale, wl.d_v,
+                                          out=out, lse=lse, workspace=hws))
+    for _ in range(3):
+        gh.replay()
+    ms_h = max_over_ranks(time_graph(gh, steps, device, flush_read=evict), device)
+    del gh
+    h_bytes = rows * L_h * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2
+    hca = {"workload": f"hca_decode_bf16_B4_L1048576_m{HCA_M}", "value": round(rows * world / (ms_h / 1e3), 1),
+           "unit": "queries/s", "ms_per_step": round(ms_h, 4),
+           "roofline": {"bound": "hbm", "achieved": round(h_bytes / (ms_h / 1e3) / 1e9, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(h_bytes / (ms_h / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                        "algorithmic_bytes": h_bytes},
+           "l2": "256 MB buffer read between replays (the 38 MB pooled cache would stay in L2)"}
+    del kv_h, inp, out, lse, hws, evict
+    torch.cuda.empty_cache()
+    return {"csa_core_attention_decode": csa, "hca_decode": hca}
 
 
 def _finish():
@@ -604,6 +713,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dsa_decode_bf16_B32_L32768_k2048")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
+    ap.add_argument("--no-v4", dest="v4", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla"], default=None,
                     help="time one kernel of the step alone (for profiler captures)")

@@ -124,3 +124,58 @@ def test_full_size_sampled_rows(cuda_device, wl, sample):
         assert lerr <= ATOL_LSE[wl.dtype], f"row {t}: lse max-abs {lerr:.3g}"
     del dv, k_pooled, kv_pooled, logits, idx, idx2, out2, lse2, mws
     torch.cuda.empty_cache()
+
+
+V4_WINDOW = 128
+
+
+def test_full_size_v4_variants(cuda_device):
+    """The 1M-token CSA shapes (4 sequences of 1,048,576 raw tokens) through
+    the two variants of the attention step, in the bench's launch
+    configuration: CSA core attention over 1024 seeded pooled entries plus a
+    128-row window of raw rows, and HCA over all 8,192 entries of the 128:1
+    pooled cache.  Sampled rows are checked against the oracle, which pools
+    the raw seeded rows itself."""
+    wl = workloads.CSA_DECODE_1M
+    dv = workloads.generate(wl, device=cuda_device, seed=0, parts=("mla",))
+    raw = dv["kv"]                                               # [4, 1048576, 576] bf16
+    B, Lraw = raw.shape[0], raw.shape[1]
+    rows = wl.rows
+    rb = dv["row_batch"]
+    pos = torch.full((rows,), Lraw - 1, dtype=torch.int32, device=cuda_device)
+    # --- CSA core attention: pooled entries + window ---
+    kv_c = dsa.csa_compress(raw, wl.compress_m)
+    g = torch.Generator().manual_seed(5)
+    idx = torch.stack([torch.randperm(wl.ctx, generator=g)[:wl.topk] for _ in range(rows)]).to(torch.int32)
+    out, lse = dsa.csa_core_attention(dv["q"], kv_c, idx.to(cuda_device), rb, wl.softmax_scale, wl.d_v, wl.ctx,
+                                      raw, pos, V4_WINDOW)
+    dsa.get_device_error()
+    for t in (0, rows - 1):
+        b = int(rb[t])
+        sel = idx[t].long().to(cuda_device)
+        raw_ids = (sel[:, None] * wl.compress_m + torch.arange(wl.compress_m, device=cuda_device)[None, :]).reshape(-1)
+        pooled = oracle.csa_compress(raw[b, raw_ids].unsqueeze(0), wl.compress_m)            # [1, 1024, 576]
+        pooled_t = torch.from_numpy(pooled.view(np.int16)).view(torch.bfloat16)
+        win = raw[b, Lraw - V4_WINDOW:].unsqueeze(0).cpu()
+        ro, rl = oracle.csa_core_attention(dv["q"][t:t + 1].cpu(), pooled_t, torch.arange(wl.topk).view(1, -1), [0],
+                                           wl.softmax_scale, wl.d_v, wl.topk, win, [V4_WINDOW - 1], V4_WINDOW)
+        assert np.abs(out[t].float().cpu().numpy() - ro[0]).max() <= ATOL_OUT["bf16"], f"csa row {t}"
+        assert np.abs(lse[t].cpu().numpy() - rl[0]).max() <= ATOL_LSE["bf16"], f"csa row {t} lse"
+    del kv_c, out, lse
+    # --- HCA: every entry of the 128:1 pooled cache ---
+    m_h = 128
+    kv_h = dsa.csa_compress(raw, m_h)                                                       # [4, 8192, 576]
+    last = torch.full((rows,), Lraw // m_h - 1, dtype=torch.int32, device=cuda_device)
+    out, lse = dsa.hca_attention(dv["q"], kv_h, rb, last, wl.softmax_scale, wl.d_v)
+    dsa.get_device_error()
+    for t in (0, rows - 1):
+        b = int(rb[t])
+        pooled = oracle.csa_compress(raw[b:b + 1], m_h)                                    # [1, 8192, 576]
+        assert np.array_equal(oracle._host(kv_h[b:b + 1]), pooled), f"hca pooling, cache {b}"
+        pooled_t = torch.from_numpy(pooled.view(np.int16)).view(torch.bfloat16)
+        ro, rl = oracle.hca_attention(dv["q"][t:t + 1].cpu(), pooled_t, [0], [Lraw // m_h - 1], wl.softmax_scale,
+                                      wl.d_v)
+        assert np.abs(out[t].float().cpu().numpy() - ro[0]).max() <= ATOL_OUT["bf16"], f"hca row {t}"
+        assert np.abs(lse[t].cpu().numpy() - rl[0]).max() <= ATOL_LSE["bf16"], f"hca row {t} lse"
+    del dv, raw, kv_h, out, lse
+    torch.cuda.empty_cache()
