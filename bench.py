@@ -523,6 +523,8 @@ def run_ours(args):
     }
     if args.prefill:
         result["prefill"] = run_prefill(dsa, workloads, device, peaks, args)
+    if args.others:
+        result["other_decodes"] = run_other_decodes(dsa, workloads, device, peaks, args)
     if args.v4:
         result["v4_variants"] = run_v4_variants(dsa, workloads, device, peaks, args)
     if world == 1 and rank == 0 and args.cpu_baseline:
@@ -558,6 +560,36 @@ def run_prefill(dsa, workloads, device, peaks, args):
                          "algorithmic_flops": fl_m},
             "indexer_roofline": {"bound": "tensor", "achieved": round(idx_t, 1), "peak": pk, "unit": "TFLOP/s",
                                  "frac": round(idx_t / pk, 4), "algorithmic_flops": fl_i}}
+
+
+def run_other_decodes(dsa, workloads, device, peaks, args):
+    """The two other decode workloads, each a whole step (indexer -> top-k ->
+    sparse MLA) in a CUDA graph, timed like the main step, against the HBM
+    roofline of its algorithmic bytes: CSA decode over 4 x 262,144 pooled
+    entries of 1,048,576-token caches (pooling is per 4 new tokens, outside
+    the step), and decode over 64 x 131,072 keys with fp8 indexer keys and a
+    paged latent cache."""
+    import torch
+    rank, world, _ = dist_env()
+    res = {}
+    for wl in (workloads.CSA_DECODE_1M, workloads.DECODE_128K_FP8_PAGED):
+        inp = workloads.generate(wl, device=device, seed=300 + rank)
+        step = DecodeStep(dsa, wl, inp, device)
+        ms, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device)
+        ms = max_over_ranks(ms, device)
+        b = indexer_bytes(wl) + mla_bytes(wl)
+        if wl.page_size:
+            b += wl.batch * (wl.ctx // wl.page_size) * 4          # the page table
+        ach = b / (ms / 1e3) / 1e9
+        res[wl.name] = {"value": round(wl.rows * world / (ms / 1e3), 1), "unit": "queries/s",
+                        "ms_per_step": round(ms, 4), "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+                        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                                     "algorithmic_bytes": b},
+                        "l2": "inputs larger than L2; no flush between steps"}
+        del inp, step
+        torch.cuda.empty_cache()
+    return res
 
 
 V4_WINDOW = 128       # raw rows in the CSA window (the pages give no size)
@@ -714,6 +746,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="dsa_decode_bf16_B32_L32768_k2048")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--no-v4", dest="v4", action="store_false")
+    ap.add_argument("--no-other-decodes", dest="others", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla"], default=None,
                     help="time one kernel of the step alone (for profiler captures)")

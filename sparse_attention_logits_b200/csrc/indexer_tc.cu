@@ -15,9 +15,15 @@
 // Warp roles (512 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: key tiles (ring of STAGES), query tiles (x2)
 //   warp 1      MMA issuer (one thread); allocates / frees TMEM
-//   warps 4-7   fp8 only: widen e4m3 key codes to bf16 straight into TMEM
+//   warps 4-7   fp8 only: widen e4m3 key codes to f16 straight into TMEM
 //               (the MMA then reads its A operand from TMEM, which keeps
-//               shared-memory traffic below the HBM rate)
+//               shared-memory traffic below the HBM rate), and convert each
+//               query tile from bf16 to f16 in shared memory once it lands:
+//               the fp8 path multiplies in f16 (one hardware conversion per
+//               two keys instead of four instructions to reach bf16).  Every
+//               e4m3 value is exact in f16; a bf16 query value is exact in f16
+//               when 2^-14 <= |q| <= 65504, and a smaller one is rounded to
+//               f16's subnormal grid (error below 2^-25)
 //   warps 8-11  epilogue for query columns [0, 128)
 //   warps 12-15 epilogue for query columns [128, 256) (NQ = 4 only)
 //
@@ -63,7 +69,7 @@ struct Cfg {
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int EPI_WARPS = 8;     // NQ = 1: two groups of 4 on alternate tiles; NQ = 4: two column halves
-    static constexpr int NBARS = 2 * STAGES + 4 + 2 * NACC + 2 * NA;
+    static constexpr int NBARS = 2 * STAGES + 4 + 2 * NACC + 2 * NA + 2;
     static constexpr size_t SMEM = 1024 + (size_t)STAGES * KBYTES + 2 * (size_t)QBYTES + NBARS * 8 + 16;
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(TMEM_NEED <= 512, "TMEM budget");
@@ -160,17 +166,25 @@ struct Sched {
     }
 };
 
-// e4m3 pair (low byte = first element) -> bf16 pair, exact for every finite
-// code (the hardware e4m3 -> f16 conversion, then f16 -> f32 -> bf16, none of
-// which rounds: an e4m3 value has at most 4 significant bits).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
+// e4m3 pair (low byte = first element) -> f16 pair, exact for every finite
+// code (an e4m3 value has at most 4 significant bits and lies within f16's
+// range).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
     uint32_t h2;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
-    const float lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    const float hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    return h2;
+}
+
+// bf16 pair -> f16 pair (round to nearest even; exact for 2^-14 <= |x| <= 65504).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(v & 0xFFFF0000u)), "f"(__uint_as_float(v << 16)));
     return r;
+}
+
+// Instruction descriptor, kind::f16 with f16 A and B, f32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace
@@ -193,7 +207,8 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     uint64_t* accempty = accfull + C::NACC;       // [NACC]
     uint64_t* afull = accempty + C::NACC;         // [NA] (fp8)
     uint64_t* aempty = afull + C::NA;             // [NA] (fp8)
-    uint32_t* tmem_slot = (uint32_t*)(aempty + C::NA);
+    uint64_t* qconv = aempty + C::NA;             // [2]  (fp8) the query tile is in f16
+    uint32_t* tmem_slot = (uint32_t*)(qconv + 2);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,6 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], 1);
+            mbar_init(&qconv[i], 4);
         }
         for (int i = 0; i < C::NA; ++i) {
             mbar_init(&afull[i], 4);
@@ -275,14 +291,15 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         // ------------------------------------------------- MMA issuer ----
         if (elect_one()) {
             sch.init(p);
-            constexpr uint32_t idesc = idesc_bf16_f32(KT, C::N, 0, 0);
+            constexpr uint32_t idesc = FP8 ? idesc_f16_f32(KT, C::N) : idesc_bf16_f32(KT, C::N, 0, 0);
             const uint32_t kbase = smem_u32(kbuf), qbase = smem_u32(qbuf);
             int i = 0, qe = -1;
             bool ok = true;
             while (ok && sch.next(p, un)) {
                 if (un.first) {
                     ++qe;
-                    ok = mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                    ok = FP8 ? mbar_wait(&qconv[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)
+                             : mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                     if (!ok) break;
                 }
                 const int st = i % C::STAGES, acc = i % C::NACC, ab = i % C::NA;
@@ -316,12 +333,30 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             }
         }
     } else if (FP8 && warp >= 4 && warp < 8) {
-        // ------------------------- fp8 -> bf16 key widening into TMEM ----
+        // ------------------------- fp8 -> f16 key widening into TMEM ----
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                  // key row of the tile = TMEM lane
         sch.init(p);
-        int i = 0;
+        int i = 0, qe = -1;
         while (sch.next(p, un)) {
+            if (un.first) {
+                // the new query tile: bf16 -> f16 in place (8 x 16 bytes per thread)
+                ++qe;
+                if (!mbar_wait(&qfull[qe & 1], (qe >> 1) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
+                uint4* qv = (uint4*)(qbuf + (size_t)(qe & 1) * C::QBYTES);
+#pragma unroll 4
+                for (int c = threadIdx.x - 128; c < C::QBYTES / 16; c += 128) {
+                    uint4 x = qv[c];
+                    x.x = bf16x2_to_f16x2(x.x);
+                    x.y = bf16x2_to_f16x2(x.y);
+                    x.z = bf16x2_to_f16x2(x.z);
+                    x.w = bf16x2_to_f16x2(x.w);
+                    qv[c] = x;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qconv[qe & 1]);
+            }
             const int st = i % C::STAGES, ab = i % C::NA;
             if (!mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
             if (!mbar_wait(&aempty[ab], ((i / C::NA) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
@@ -338,8 +373,8 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                     const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        words[c4 * 8 + 2 * e] = e4m3x2_to_bf16x2((uint16_t)(xs[e] & 0xFFFFu));
-                        words[c4 * 8 + 2 * e + 1] = e4m3x2_to_bf16x2((uint16_t)(xs[e] >> 16));
+                        words[c4 * 8 + 2 * e] = e4m3x2_to_f16x2((uint16_t)(xs[e] & 0xFFFFu));
+                        words[c4 * 8 + 2 * e + 1] = e4m3x2_to_f16x2((uint16_t)(xs[e] >> 16));
                     }
                 }
                 uint32_t lo[16], hi[16];
