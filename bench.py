@@ -575,7 +575,7 @@ def run_other_decodes(dsa, workloads, device, peaks, args):
     for wl in (workloads.CSA_DECODE_1M, workloads.DECODE_128K_FP8_PAGED):
         inp = workloads.generate(wl, device=device, seed=300 + rank)
         step = DecodeStep(dsa, wl, inp, device)
-        ms, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device)
+        ms, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device, soak_s=0.5)
         ms = max_over_ranks(ms, device)
         b = indexer_bytes(wl) + mla_bytes(wl)
         if wl.page_size:

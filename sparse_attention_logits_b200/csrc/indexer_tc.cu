@@ -403,9 +403,15 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         while (sch.next(p, un)) {
             if (NQ == 1 && (i & 1) != eg) { ++i; continue; }
             const int acc = i % C::NACC;
+            const int key = un.tile * KT + quarter * 32 + lane;
+            // the key's row and (fp8) dequantisation scale are loaded before
+            // the wait for the accumulator, so their latency is hidden
+            const int b = __ldg(p.row_batch + un.t0);
+            const bool b_ok = b >= 0 && b < p.batch;
+            float ks = 1.f;
+            if (FP8 && b_ok && key < p.ctx) ks = __ldg(p.k_scale + (int64_t)b * p.ctx + key);
             if (!mbar_wait(&accfull[acc], (i / C::NACC) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
-            const int key = un.tile * KT + quarter * 32 + lane;
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * C::ACC_COLS;
             constexpr int QPW = NQ == 1 ? 1 : 2;           // query rows per epilogue warp
             float score[QPW];
@@ -437,11 +443,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
-            const int b = __ldg(p.row_batch + un.t0);
-            const bool b_ok = b >= 0 && b < p.batch;
             if (!b_ok && lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
-            float ks = 1.f;
-            if (FP8 && b_ok && key < p.ctx) ks = __ldg(p.k_scale + (int64_t)b * p.ctx + key);
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
                 const int t = un.t0 + (NQ == 1 ? 0 : eg * 2 + qq);
