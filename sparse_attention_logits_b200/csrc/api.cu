@@ -55,11 +55,11 @@ dsa_status_t make_launch(void* stream, dsa::Launch* L) {
     return DSA_OK;
 }
 
-// Fixed scratch of dsa_sparse_mla_noalloc: the fp32 partial outputs and
+// Fixed scratch of dsa_sparse_mla_noalloc: the bf16 partial outputs and fp32
 // log-sum-exps of a key list split over several clusters.  A (row, split)
-// pair takes 128 heads x 513 floats = 262,656 bytes, and the split count is
+// pair takes 128 heads x (512 x 2 + 4) = 131,584 bytes, and the split count is
 // chosen so that rows x splits <= SMs / 2, so 20 MiB covers every size on a
-// GPU of up to 159 SMs.  No byte of it has to start at zero: each cluster
+// GPU of up to 318 SMs.  No byte of it has to start at zero: each cluster
 // writes its whole partial block before the merge kernel, launched after it
 // on the same stream, reads it.  One copy per device: calls that overlap on
 // one device (two streams, two threads) race on it.

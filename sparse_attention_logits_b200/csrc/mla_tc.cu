@@ -25,16 +25,18 @@
 //                       O += P V (M=128, N=2x256, K=64) in its 512 TMEM
 //                       columns, and at the end writes O / l and
 //                       lse = ln(sum exp) -- or, when the key list is split
-//                       over several clusters, normalised fp32 partials that
-//                       dsa_mla_combine merges.
+//                       over several clusters, normalised bf16 partials and
+//                       their lse, which mla_combine_kernel merges in fp32
+//                       (rounding a partial to bf16 costs at most one more
+//                       bf16 ulp of the output).
 //
 // Two splits per row (decode with few rows): both pairs of a row form one
 // 4-CTA cluster (ranks 0-1 split 0, ranks 2-3 split 1) and their value CTAs
 // merge the splits themselves: each sends the 256 columns that the other
 // finalises (raw fp32, DSMEM stores) as soon as both gather regions are
 // drained, then they swap (max, sum) per head and each writes its half of
-// out = (a O_0 + a' O_1) / (a l_0 + a' l_1).  This replaces the fp32 partials
-// in global memory and the merge launch whenever all rows' 4-CTA clusters fit
+// out = (a O_0 + a' O_1) / (a l_0 + a' l_1).  This replaces the partials in
+// global memory and the merge launch whenever all rows' 4-CTA clusters fit
 // on the GPU at once.
 //
 // Warps (both CTAs): 0-15 gather producers (cp.async, 4 rows each); 16-23
@@ -111,7 +113,7 @@ struct MlaParams {
     int len2, window;
     __nv_bfloat16* out;
     float* lse;
-    float* part_o;                  // [rows, splits, H, DV] when splits > 1
+    __nv_bfloat16* part_o;          // [rows, splits, H, DV] normalised partials when splits > 1
     float* part_lse;                // [rows, splits, H]
     unsigned* err;
     int page_size, pages_per_seq, num_pages;
@@ -655,9 +657,10 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                             p.lse[(int64_t)w.t * H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
                     }
                 }
-            } else if (p.splits == 1) {
-                // bf16 tiles of 32 heads x 64 columns
-                const int row0 = w.t * H + quarter * 32;
+            } else {
+                // bf16 tiles of 32 heads x 64 columns: the output, or (key list
+                // split over several clusters) this split's normalised partial
+                const int row0 = (p.splits == 1 ? w.t * H : (w.t * p.splits + w.split) * H) + quarter * 32;
 #pragma unroll 1
                 for (int j = 0; j < 4; ++j) {
                     const int col = colhalf * 256 + j * 64;
@@ -688,34 +691,10 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                         bulk_commit_group();
                     }
                 }
-                if (colhalf == 0) p.lse[(int64_t)w.t * H + h] = lse;
-            } else {
-                // fp32 partial tiles of 32 heads x 32 columns
-                const int row0 = (w.t * p.splits + w.split) * H + quarter * 32;
-#pragma unroll 1
-                for (int j = 0; j < 8; ++j) {
-                    const int col = colhalf * 256 + j * 32;
-                    float v[32];
-                    tmem_ld32(tmem + lane_base + col, v);
-                    tmem_ld_wait();
-                    if (j >= 2) {
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
-                    }
-                    uint8_t* buf = srow + (j & 1) * EPI_BUF;
-#pragma unroll
-                    for (int ci = 0; ci < 8; ++ci)
-                        st_shared_v4(buf + ((ci ^ (lane & 7)) << 4), __float_as_uint(v[4 * ci] * inv),
-                                     __float_as_uint(v[4 * ci + 1] * inv), __float_as_uint(v[4 * ci + 2] * inv),
-                                     __float_as_uint(v[4 * ci + 3] * inv));
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&o_map, stage + (j & 1) * EPI_BUF, col, row0);
-                        bulk_commit_group();
-                    }
+                if (colhalf == 0) {
+                    if (p.splits == 1) p.lse[(int64_t)w.t * H + h] = lse;
+                    else p.part_lse[((int64_t)w.t * p.splits + w.split) * H + h] = lse;
                 }
-                if (colhalf == 0) p.part_lse[((int64_t)w.t * p.splits + w.split) * H + h] = lse;
             }
             if (lane == 0) bulk_wait_group<0>();
             __syncwarp();
@@ -785,8 +764,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     }
 }
 
-// Merge of split partials: out = sum_s exp(lse_s - lse) * O_s, lse = log sum_s exp(lse_s).
-__global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restrict__ part_o,
+// Merge of split partials: out = sum_s exp(lse_s - lse) * O_s, lse = log sum_s exp(lse_s),
+// in fp32 from the bf16 partials.
+__global__ void __launch_bounds__(128) mla_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
                                                           const float* __restrict__ part_lse, int splits,
                                                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
     pdl_wait();
@@ -803,9 +783,11 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const float* __restric
             if (ls == -INFINITY) continue;
             const float wgt = __expf(ls - mx);
             den += wgt;
-            const float4 o = __ldg((const float4*)(part_o + pr * DV + d));
-            acc.x = fmaf(wgt, o.x, acc.x); acc.y = fmaf(wgt, o.y, acc.y);
-            acc.z = fmaf(wgt, o.z, acc.z); acc.w = fmaf(wgt, o.w, acc.w);
+            const uint2 raw = __ldg((const uint2*)(part_o + pr * DV + d));
+            const float2 a = __bfloat1622float2(*(const __nv_bfloat162*)&raw.x);
+            const float2 b = __bfloat1622float2(*(const __nv_bfloat162*)&raw.y);
+            acc.x = fmaf(wgt, a.x, acc.x); acc.y = fmaf(wgt, a.y, acc.y);
+            acc.z = fmaf(wgt, b.x, acc.z); acc.w = fmaf(wgt, b.y, acc.w);
         }
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
@@ -871,7 +853,7 @@ bool mla_tc_supported(dsa_dtype_t dtype, int n_heads, int d_qk, int d_v) {
 size_t mla_tc_workspace_bytes(int rows, int k, int num_sms) {
     const int s = choose_splits(rows, k, num_sms);
     if (s == 1) return 0;
-    return (size_t)rows * s * H * (DV + 1) * sizeof(float);
+    return (size_t)rows * s * H * (DV * sizeof(__nv_bfloat16) + sizeof(float));
 }
 
 cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const int32_t* page_table, int page_size,
@@ -917,10 +899,10 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     // merge launch); otherwise split partials go to the workspace.
     p.fuse2 = (p.splits == 2 && rows <= max_active_quads()) ? 1 : 0;
     if (p.splits > 1 && !p.fuse2) {
-        const size_t need = (size_t)rows * p.splits * H * (DV + 1) * sizeof(float);
+        const size_t need = (size_t)rows * p.splits * H * (DV * sizeof(__nv_bfloat16) + sizeof(float));
         if (!workspace || ws_bytes < need || (uintptr_t)workspace % 16) return cudaErrorInvalidValue;
-        p.part_o = (float*)workspace;
-        p.part_lse = p.part_o + (size_t)rows * p.splits * H * DV;
+        p.part_o = (__nv_bfloat16*)workspace;
+        p.part_lse = (float*)(p.part_o + (size_t)rows * p.splits * H * DV);
     }
     // Q as [rows*128, 576] bf16 in boxes of 128 heads x 64 dims; the output as
     // [rows*128, 512] bf16 in boxes of 32 heads x 64 columns, or the partials
@@ -930,8 +912,8 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     if (p.splits == 1 || p.fuse2)
         ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, DV, (uint64_t)rows * H, 64, 32);
     else
-        ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.part_o, DV,
-                                  (uint64_t)rows * p.splits * H, 32, 32);
+        ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.part_o, DV,
+                                  (uint64_t)rows * p.splits * H, 64, 32);
     if (!ok) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2u * (unsigned)rows * (unsigned)p.splits);
@@ -957,7 +939,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
         cudaLaunchAttribute a2[1] = {pdl_attr()};
         c2.attrs = a2;
         c2.numAttrs = 1;
-        e = cudaLaunchKernelEx(&c2, mla_combine_kernel, (const float*)p.part_o, (const float*)p.part_lse, p.splits,
+        e = cudaLaunchKernelEx(&c2, mla_combine_kernel, (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, p.splits,
                                (__nv_bfloat16*)out, lse);
         count_launch();
     }
