@@ -34,7 +34,8 @@ constexpr int MAX_PASSES = 3;                  // 11 + 10 + 10 bits: the range i
 constexpr int CAND_CAP = 1024;                 // candidates ranked directly after the first pass
 // hist, merged (scan scratch), one cluster-wide histogram per pass, scratch,
 // candidate buffer, candidates' source CTAs, per-CTA counts (rank 0)
-constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 32 + 32) * 4;
+constexpr int MAX_CL = 16;                     // CTAs per row (16 needs the non-portable cluster size)
+constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 32 + 3 * MAX_CL + 16) * 4;
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* cand_n = cta_counts + 8;           // candidate count (rank 0's is used)
     uint32_t* cand = cta_counts + 16;            // [CAND_CAP] candidate keys (rank 0's is used)
     uint32_t* cand_src = cand + CAND_CAP;        // [CAND_CAP] the CTA each candidate comes from (rank 0's)
-    uint32_t* cta_cnt = cand_src + CAND_CAP;     // [3][8] per-CTA keys above the bin, candidates > T, == T (rank 0's)
+    uint32_t* cta_cnt = cand_src + CAND_CAP;     // [3][MAX_CL] per-CTA keys above the bin, candidates > T, == T (rank 0's)
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
 
     pdl_wait();                     // the scores of the previous kernel are visible from here on
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     if (CL > 1)
         for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
     if (tid == 0) *cand_n = 0u;
-    if (tid < 24) cta_cnt[tid] = 0u;
+    if (tid < 3 * MAX_CL) cta_cnt[tid] = 0u;
     __syncthreads();
     // the slice is padded with copies of its first key up to a multiple of 4
     // (cnt4), so that every walk below reads 16 bytes per lane
@@ -363,8 +364,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                 const uint32_t t_key = shared_res[4];
                 if ((uint32_t)tid < nc) {
                     const uint32_t key = cand[tid], src = cand_src[tid];
-                    if (key > t_key) atomicAdd(&cta_cnt[8 + src], 1u);
-                    else if (key == t_key) atomicAdd(&cta_cnt[16 + src], 1u);
+                    if (key > t_key) atomicAdd(&cta_cnt[MAX_CL + src], 1u);
+                    else if (key == t_key) atomicAdd(&cta_cnt[2 * MAX_CL + src], 1u);
                 }
                 __syncthreads();
                 if (tid == 0) {
@@ -378,9 +379,9 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                         st_cluster_u32(dst + 4, rem_eq);
                         st_cluster_u32(dst + 8, eqb);
                         st_cluster_u32(dst + 12, outb);
-                        const uint32_t e = cta_cnt[16 + r];
+                        const uint32_t e = cta_cnt[2 * MAX_CL + r];
                         const uint32_t take = eqb >= rem_eq ? 0u : min(e, rem_eq - eqb);
-                        outb += cta_cnt[r] + cta_cnt[8 + r] + take;
+                        outb += cta_cnt[r] + cta_cnt[MAX_CL + r] + take;
                         eqb += e;
                     }
                 }
@@ -540,11 +541,48 @@ namespace {
 // when there are few rows, as many more (up to 8) as keep every SM busy --
 // a decode batch of 32 rows would otherwise leave most SMs idle.  Many rows
 // that fit one SM each are selected one CTA per row (no cross-CTA traffic).
+// 16-CTA clusters of topk_cluster_kernel<16> (slices of 16,384 keys) that the
+// current device can hold at once (0 if none or the query fails); looked up
+// once per device.
+int max_active_16() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cache[dev] == 0) {
+        const size_t smem = 128 + SMEM_FIXED + (size_t)16384 * 4;
+        int n = 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(16);
+        cfg.blockDim = dim3(TOPK_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 16;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(topk_cluster_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<16>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev] = n > 0 ? n : -1;
+    }
+    return cache[dev] > 0 ? cache[dev] : 0;
+}
+
 int choose_cluster(int rows, int ctx_len, int num_sms) {
     const int need = (ctx_len + SLICE_CAP - 1) / SLICE_CAP;
     int cl = 1;
     while (cl < need && cl < 8) cl <<= 1;
     while (cl < 8 && (int64_t)rows * cl * 2 <= num_sms && ctx_len / (cl * 2) >= 4096) cl <<= 1;
+    // very long rows and very few of them: 16 CTAs per row, when the GPU can
+    // hold all rows' 16-CTA clusters at once
+    if (cl == 8 && (int64_t)rows * 16 <= num_sms && ctx_len / 16 >= 8192 && rows <= max_active_16()) cl = 16;
     return cl;
 }
 
@@ -555,6 +593,10 @@ cudaError_t launch_cl(const Launch& L, const float* logits, int64_t ld, const in
     const size_t smem = 128 + SMEM_FIXED + (size_t)per * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    if (CL > 8) {
+        e = cudaFuncSetAttribute(topk_cluster_kernel<CL>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)rows * CL);
     cfg.blockDim = dim3(TOPK_THREADS);
@@ -584,9 +626,11 @@ cudaError_t launch_topk(const Launch& L, const float* logits, int64_t ld, const 
     case 1: return launch_cl<1>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
     case 2: return launch_cl<2>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
     case 4: return launch_cl<4>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
-    default: return launch_cl<8>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    case 8: return launch_cl<8>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
+    default: return launch_cl<16>(L, logits, ld, row_pos, rows, ctx_len, k, idx);
     }
 }
+
 
 size_t topk_workspace_bytes(int /*rows*/, int /*ctx_len*/, int /*k*/) { return 0; }
 

@@ -71,7 +71,8 @@ def test_indexer_matches_oracle(cuda_device, wl):
 # ---------------------------------------------------------------- top-k ----
 
 @pytest.mark.parametrize("rows,L,k,seed", [(7, 1000, 64, 0), (4, 32768, 2048, 1), (3, 5000, 2048, 2),
-                                           (2, 262144, 1024, 3), (5, 300, 300, 4), (3, 129, 1, 5)])
+                                           (2, 262144, 1024, 3), (5, 300, 300, 4), (3, 129, 1, 5),
+                                           (9, 200000, 2048, 6)])
 def test_topk_bit_exact_on_given_scores(cuda_device, rows, L, k, seed):
     x = workloads.synthetic_scores(rows, L, seed=seed)
     pos = torch.tensor([L - 1 - (r * 37) % max(1, L // 3) for r in range(rows)], dtype=torch.int32)
