@@ -93,8 +93,8 @@ def measured_peaks():
 def indexer_bytes(wl) -> int:
     """Algorithmic bytes of one indexer launch: every visible key row read
     once, the queries and weights read once, the visible scores written."""
-    key_b = {"bf16": 2, "fp32": 4, "fp8": 1}[wl.idx_key_dtype]
-    scale_b = 4 if wl.idx_key_dtype == "fp8" else 0
+    key_b = {"bf16": 2, "fp32": 4, "fp8": 1, "fp4": 0.5}[wl.idx_key_dtype]
+    scale_b = 4 if wl.idx_key_dtype in ("fp8", "fp4") else 0
     q_b = 2 if wl.dtype == "bf16" else 4
     if wl.mode == "decode":
         vis = wl.ctx * wl.rows          # one query per cache in these workloads
@@ -102,7 +102,7 @@ def indexer_bytes(wl) -> int:
     else:
         vis = wl.rows * (wl.rows + 1) // 2
         keys = wl.ctx
-    return keys * wl.idx_dim * key_b + keys * scale_b + wl.rows * wl.idx_heads * (wl.idx_dim * q_b + 4) + vis * 4
+    return int(keys * wl.idx_dim * key_b + keys * scale_b + wl.rows * wl.idx_heads * (wl.idx_dim * q_b + 4) + vis * 4)
 
 
 def indexer_flops(wl) -> int:
@@ -568,11 +568,13 @@ def run_other_decodes(dsa, workloads, device, peaks, args):
     roofline of its algorithmic bytes: CSA decode over 4 x 262,144 pooled
     entries of 1,048,576-token caches (pooling is per 4 new tokens, outside
     the step), and decode over 64 x 131,072 keys with fp8 indexer keys and a
-    paged latent cache."""
+    paged latent cache, and the same with fp4 (e2m1) indexer keys."""
     import torch
     rank, world, _ = dist_env()
     res = {}
-    for wl in (workloads.CSA_DECODE_1M, workloads.DECODE_128K_FP8_PAGED):
+    fp4 = workloads.DECODE_128K_FP8_PAGED.with_(name="dsa_decode_fp4idx_paged64_B64_L131072_k2048",
+                                                idx_key_dtype="fp4")
+    for wl in (workloads.CSA_DECODE_1M, workloads.DECODE_128K_FP8_PAGED, fp4):
         inp = workloads.generate(wl, device=device, seed=300 + rank)
         step = DecodeStep(dsa, wl, inp, device)
         ms, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device, soak_s=0.5)

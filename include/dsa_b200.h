@@ -66,7 +66,9 @@ typedef enum {
 typedef enum {
     DSA_FP32 = 0,
     DSA_BF16 = 1,
-    DSA_FP8_E4M3 = 2            /* OCP e4m3 "fn": bias 7, max 448, no infinities */
+    DSA_FP8_E4M3 = 2,           /* OCP e4m3 "fn": bias 7, max 448, no infinities */
+    DSA_FP4_E2M1 = 3            /* OCP e2m1: bias 1, values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and their
+                                   negatives; two per byte, the lower dim in the low nibble */
 } dsa_dtype_t;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -108,9 +110,10 @@ DSA_API dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch,
  *
  *   q          [rows, n_heads, head_dim]  of q_dtype (DSA_FP32 or DSA_BF16)
  *   w          [rows, n_heads] fp32
- *   k          [batch, ctx_len, head_dim] of k_dtype (DSA_FP32, DSA_BF16 or DSA_FP8_E4M3)
- *   k_scale    [batch, ctx_len] fp32, one dequantisation scale per fp8 key row
- *              (stored key = code * scale); must be NULL unless k is fp8
+ *   k          [batch, ctx_len, head_dim] of k_dtype (DSA_FP32, DSA_BF16 or DSA_FP8_E4M3), or
+ *              [batch, ctx_len, head_dim / 2] bytes of DSA_FP4_E2M1 code pairs
+ *   k_scale    [batch, ctx_len] fp32, one dequantisation scale per fp8 / fp4 key
+ *              row (stored key = code * scale); must be NULL unless k is fp8 or fp4
  *   row_batch  [rows] int32, cache of each query row, in [0, batch)
  *   row_pos    [rows] int32, last visible key of each row, in [0, ctx_len):
  *              prefill rows use their own position (causal), decode rows use
@@ -119,8 +122,13 @@ DSA_API dsa_status_t csa_compress(const void* src, dsa_dtype_t dtype, int batch,
  *              s <= row_pos[t] are written; entries beyond row_pos[t] are
  *              left untouched (dsa_topk never reads them).
  * Accumulation is fp32.  Supported: head_dim in {32, 64, 128}; q and k of the
- * same floating type, or bf16 q with fp8 k; n_heads <= 128.  fp8 key codes
- * must be finite (0x7F and 0xFF, the e4m3 NaNs, are not valid codes).
+ * same floating type, or bf16 q with fp8 k; n_heads <= 128; fp4 keys (V4 CSA
+ * summary: the V4 indexer keys are FP4) with bf16 q, n_heads = 64 and
+ * head_dim = 128.  fp8 key codes must be finite (0x7F and 0xFF, the e4m3 NaNs,
+ * are not valid codes).  With fp8 or fp4 keys the products are formed in f16:
+ * every code is exact in f16, and so is every bf16 query value with
+ * 2^-14 <= |q| <= 65504 (smaller ones are rounded to f16's subnormal grid,
+ * an error below 2^-25 each; larger ones are not supported).
  */
 DSA_API dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float* w,
                                 const void* k, dsa_dtype_t k_dtype, const float* k_scale,

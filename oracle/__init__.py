@@ -29,7 +29,7 @@ _LIB_PATH = os.path.join(_OUT_DIR, "liboracle.so")
 _lock = threading.Lock()
 _lib = None
 
-FP32, BF16, FP8 = 0, 1, 2
+FP32, BF16, FP8, FP4 = 0, 1, 2, 3
 
 _I32P = ctypes.POINTER(ctypes.c_int32)
 _F32P = ctypes.POINTER(ctypes.c_float)
@@ -58,6 +58,8 @@ def lib():
             L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
             L.oracle_fp8_e4m3_to_double.restype = ctypes.c_double
             L.oracle_fp8_e4m3_to_double.argtypes = [ctypes.c_uint8]
+            L.oracle_fp4_e2m1_to_double.restype = ctypes.c_double
+            L.oracle_fp4_e2m1_to_double.argtypes = [ctypes.c_uint8]
             L.oracle_double_to_bf16_rne.restype = ctypes.c_uint16
             L.oracle_double_to_bf16_rne.argtypes = [ctypes.c_double]
             L.oracle_csa_compress.restype = None
@@ -128,6 +130,10 @@ def fp8_e4m3_to_double(code: int) -> float:
     return float(lib().oracle_fp8_e4m3_to_double(int(code) & 0xFF))
 
 
+def fp4_e2m1_to_double(code: int) -> float:
+    return lib().oracle_fp4_e2m1_to_double(code)
+
+
 def double_to_bf16_bits(x: float) -> int:
     return int(lib().oracle_double_to_bf16_rne(float(x)))
 
@@ -147,16 +153,21 @@ def csa_compress(src, m: int) -> np.ndarray:
 
 
 def index_scores(q_idx, w, k_idx, row_batch, row_pos, k_scale=None, row_ids=None) -> np.ndarray:
-    """Index scores of the requested query rows: float64 [n, L]."""
+    """Index scores of the requested query rows: float64 [n, L].  fp8 keys are
+    uint8 [B, L, D_I] codes, fp4 keys uint8 [B, L, D_I/2] code pairs (low
+    nibble first), each with k_scale [B, L]."""
     q = _host(q_idx)
     k = _host(k_idx)
     wf = np.ascontiguousarray(_host(w), dtype=np.float32)
     rows, H_I, D_I = q.shape
     B, L, D_I2 = k.shape
-    assert D_I2 == D_I
     kd = _dtype_code(k)
+    if kd == FP8 and 2 * D_I2 == D_I:
+        kd = FP4
+    else:
+        assert D_I2 == D_I
     ks = None
-    if kd == FP8:
+    if kd in (FP8, FP4):
         ks = np.ascontiguousarray(_host(k_scale), dtype=np.float32)
         assert ks.shape == (B, L)
     rb, rp = _i32(row_batch), _i32(row_pos)

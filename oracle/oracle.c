@@ -44,7 +44,7 @@
 #include <omp.h>
 #endif
 
-enum { ODT_FP32 = 0, ODT_BF16 = 1, ODT_FP8_E4M3 = 2 };
+enum { ODT_FP32 = 0, ODT_BF16 = 1, ODT_FP8_E4M3 = 2, ODT_FP4_E2M1 = 3 };
 enum { ORACLE_MAX_DIM = 1024 };
 
 /* ---- element formats --------------------------------------------------- */
@@ -70,6 +70,16 @@ double oracle_fp8_e4m3_to_double(uint8_t code)
         v = ldexp((double)m / 8.0, -6);
     else
         v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* OCP fp4 E2M1: 1 sign, 2 exponent (bias 1), 1 mantissa bit; exponent 0 is
+ * subnormal (m/2 * 2^0); no infinities or NaNs.  The 8 magnitudes are
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6.  `code` is one 4-bit code (low nibble). */
+double oracle_fp4_e2m1_to_double(uint8_t code)
+{
+    int s = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    double v = (e == 0) ? (double)m / 2.0 : ldexp(1.0 + (double)m / 2.0, e - 1);
     return s ? -v : v;
 }
 
@@ -107,6 +117,10 @@ static double load_elem(const void* p, int dtype, int64_t i)
     case ODT_FP32: return (double)((const float*)p)[i];
     case ODT_BF16: return oracle_bf16_to_double(((const uint16_t*)p)[i]);
     case ODT_FP8_E4M3: return oracle_fp8_e4m3_to_double(((const uint8_t*)p)[i]);
+    case ODT_FP4_E2M1: {   /* two codes per byte, element 2j in the low nibble */
+        uint8_t byte = ((const uint8_t*)p)[i >> 1];
+        return oracle_fp4_e2m1_to_double((i & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF));
+    }
     default: return NAN;
     }
 }
@@ -141,8 +155,9 @@ void oracle_csa_compress(const void* src, int dtype, int B, int L, int D, int m,
  *   out[n, s] = sum_j w[t,j] * max(0, sum_d q[t,j,d] * k[b,s,d])   for s <= row_pos[t]
  *   out[n, s] = -inf                                               for s >  row_pos[t]
  * with b = row_batch[t].  q [rows, H_I, D_I] (fp32 or bf16), w [rows, H_I]
- * fp32, k [B, L, D_I] (fp32, bf16 or fp8 codes).  For fp8 keys the stored
- * value is code * k_scale[b, s] (one scale per key row). */
+ * fp32, k [B, L, D_I] (fp32, bf16 or fp8 codes, or fp4 code pairs).  For fp8
+ * and fp4 keys the stored value is code * k_scale[b, s] (one scale per key
+ * row). */
 void oracle_index_scores(const void* q, int q_dtype, const float* w,
                          const void* k, int k_dtype, const float* k_scale,
                          const int32_t* row_batch, const int32_t* row_pos,
@@ -166,7 +181,7 @@ void oracle_index_scores(const void* q, int q_dtype, const float* w,
                 continue;
             }
             int64_t krow = (int64_t)b * L + s;
-            double ks = (k_dtype == ODT_FP8_E4M3) ? (double)k_scale[krow] : 1.0;
+            double ks = (k_dtype == ODT_FP8_E4M3 || k_dtype == ODT_FP4_E2M1) ? (double)k_scale[krow] : 1.0;
             for (int d = 0; d < D_I; ++d)
                 kv[d] = load_elem(k, k_dtype, krow * D_I + d) * ks;
             double score = 0.0;

@@ -30,7 +30,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_CUDA, DSA_ERR_DEVICE_TIMEOUT = range(5)
-DSA_FP32, DSA_BF16, DSA_FP8_E4M3 = 0, 1, 2
+DSA_FP32, DSA_BF16, DSA_FP8_E4M3, DSA_FP4_E2M1 = 0, 1, 2, 3
 
 _STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_CUDA",
                  4: "DSA_ERR_DEVICE_TIMEOUT"}
@@ -135,17 +135,22 @@ def csa_compress(src: torch.Tensor, m: int, out: Optional[torch.Tensor] = None) 
 def indexer_logits(q_idx: torch.Tensor, w: torch.Tensor, k_idx: torch.Tensor, row_batch: torch.Tensor,
                    row_pos: torch.Tensor, k_scale: Optional[torch.Tensor] = None,
                    out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Index scores [rows, L] fp32 (entries past row_pos untouched)."""
+    """Index scores [rows, L] fp32 (entries past row_pos untouched).  fp8 keys
+    are uint8 [B, L, D] e4m3 codes, fp4 keys uint8 [B, L, D/2] e2m1 code pairs
+    (low nibble first), each with k_scale [B, L]."""
     dev = _dev(q_idx, w, k_idx, row_batch, row_pos, k_scale, out)
     rows, H, D = q_idx.shape
     B, L, D2 = k_idx.shape
-    if D2 != D:
+    kdt = _dt(k_idx)
+    if kdt == DSA_FP8_E4M3 and 2 * D2 == D:
+        kdt = DSA_FP4_E2M1
+    elif D2 != D:
         raise ValueError("q_idx and k_idx head dims differ")
     if out is None:
         out = torch.empty((rows, L), dtype=torch.float32, device=dev)
     ld = out.stride(0) if out.dim() == 2 else L
     with torch.cuda.device(dev):
-        _check(_lib.dsa_indexer_logits(_ptr(q_idx), _dt(q_idx), _ptr(w), _ptr(k_idx), _dt(k_idx), _ptr(k_scale),
+        _check(_lib.dsa_indexer_logits(_ptr(q_idx), _dt(q_idx), _ptr(w), _ptr(k_idx), kdt, _ptr(k_scale),
                                        _ptr(row_batch), _ptr(row_pos), rows, B, L, H, D, _ptr(out), ld,
                                        _stream(dev)), "dsa_indexer_logits")
     return out

@@ -91,6 +91,7 @@ dsa_status_t mla_scratch(void** out) {
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 size_t dtype_size(dsa_dtype_t t) { return t == DSA_FP32 ? 4 : t == DSA_BF16 ? 2 : 1; }
 bool valid_dtype(dsa_dtype_t t) { return t == DSA_FP32 || t == DSA_BF16 || t == DSA_FP8_E4M3; }
+bool valid_key_dtype(dsa_dtype_t t) { return valid_dtype(t) || t == DSA_FP4_E2M1; }
 
 }  // namespace
 
@@ -134,16 +135,19 @@ dsa_status_t dsa_indexer_logits(const void* q, dsa_dtype_t q_dtype, const float*
     if (rows == 0 || ctx_len == 0) return DSA_OK;
     if (!q || !w || !k || !row_batch || !row_pos || !logits)
         return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: null pointer");
-    if (!valid_dtype(q_dtype) || !valid_dtype(k_dtype)) return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: bad dtype");
+    if (!valid_dtype(q_dtype) || !valid_key_dtype(k_dtype)) return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: bad dtype");
     if (ld_logits < ctx_len) return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: ld_logits < ctx_len");
-    if ((k_dtype == DSA_FP8_E4M3) != (k_scale != nullptr))
-        return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: k_scale must be given exactly when k is fp8");
+    if ((k_dtype == DSA_FP8_E4M3 || k_dtype == DSA_FP4_E2M1) != (k_scale != nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "dsa_indexer_logits: k_scale must be given exactly when k is fp8 or fp4");
     const bool combo_ok = (q_dtype == DSA_FP32 && k_dtype == DSA_FP32) || (q_dtype == DSA_BF16 && k_dtype == DSA_BF16) ||
-                          (q_dtype == DSA_BF16 && k_dtype == DSA_FP8_E4M3);
+                          (q_dtype == DSA_BF16 && k_dtype == DSA_FP8_E4M3) ||
+                          (q_dtype == DSA_BF16 && k_dtype == DSA_FP4_E2M1);
     if (!combo_ok) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: unsupported q/k dtype pair");
     if (head_dim != 32 && head_dim != 64 && head_dim != 128)
         return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: head_dim must be 32, 64 or 128");
     if (n_heads > 128) return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: n_heads > 128");
+    if (k_dtype == DSA_FP4_E2M1 && !dsa::indexer_tc_supported(q_dtype, k_dtype, n_heads, head_dim))
+        return fail(DSA_ERR_UNSUPPORTED, "dsa_indexer_logits: fp4 keys need n_heads = 64 and head_dim = 128");
     dsa::Launch L;
     dsa_status_t st = make_launch(stream, &L);
     if (st != DSA_OK) return st;

@@ -15,7 +15,7 @@
 // Warp roles (512 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: key tiles (ring of STAGES), query tiles (x2)
 //   warp 1      MMA issuer (one thread); allocates / frees TMEM
-//   warps 4-7   fp8 only: widen e4m3 key codes to f16 straight into TMEM
+//   warps 4-7   fp8 / fp4 only: widen e4m3 / e2m1 key codes to f16 straight into TMEM
 //               (the MMA then reads its A operand from TMEM, which keeps
 //               shared-memory traffic below the HBM rate), and convert each
 //               query tile from bf16 to f16 in shared memory once it lands:
@@ -49,11 +49,17 @@ constexpr int DI = 128;      // indexer head dim = MMA K
 constexpr int HI = 64;       // indexer heads
 constexpr int THREADS = 512;
 
-template <int NQ, bool FP8>
+// Key formats: KF_BF16, KF_FP8 (e4m3 codes, one byte per dim) and KF_FP4
+// (e2m1 codes, two dims per byte, low nibble first).  fp8 and fp4 keys carry
+// one fp32 dequantisation scale per key row and are widened to f16 in TMEM.
+enum { KF_BF16 = 0, KF_FP8 = 1, KF_FP4 = 2 };
+
+template <int NQ, int KF>
 struct Cfg {
+    static constexpr bool FP8 = KF != KF_BF16;      // narrow keys: widened into TMEM, scaled in the epilogue
     static constexpr int N = NQ * HI;
-    static constexpr int STAGES = FP8 ? 8 : (NQ == 1 ? 6 : 3);
-    static constexpr int KBYTES = FP8 ? KT * DI : KT * DI * 2;      // one key tile in shared memory
+    static constexpr int STAGES = KF == KF_FP4 ? 16 : KF == KF_FP8 ? 8 : (NQ == 1 ? 6 : 3);
+    static constexpr int KBYTES = KF == KF_FP4 ? KT * DI / 2 : KF == KF_FP8 ? KT * DI : KT * DI * 2;  // one key tile
     static constexpr int QBYTES = N * DI * 2;                        // one query tile (bf16)
     static constexpr int ACC_COLS = N;
     // accumulator ring: decode has 4 (two epilogue groups take alternate
@@ -175,6 +181,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
     return h2;
 }
 
+// e2m1 pair (low nibble = first element) -> f16 pair, exact (an e2m1 value
+// has at most 2 significant bits and lies within f16's range).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"(byte));
+    return h2;
+}
+
 // bf16 pair -> f16 pair (round to nearest even; exact for 2^-14 <= |x| <= 65504).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
     uint32_t r;
@@ -189,11 +203,12 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 
 }  // namespace
 
-template <int NQ, bool FP8>
+template <int NQ, int KF>
 __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                                 const __grid_constant__ CUtensorMap tmap_q,
                                                                 const Params p) {
-    using C = Cfg<NQ, FP8>;
+    using C = Cfg<NQ, KF>;
+    constexpr bool FP8 = C::FP8;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* kbuf = smem;                                            // [STAGES][KBYTES]
@@ -361,8 +376,24 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             if (!mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
             if (!mbar_wait(&aempty[ab], ((i / C::NA) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
-            const uint8_t* src = kbuf + (size_t)st * C::KBYTES + r * 128;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + ab * C::A_COLS;
+            if (KF == KF_FP4) {
+                // a 64-byte row of e2m1 pairs (64-byte swizzle: chunk c of row r
+                // sits at chunk c ^ ((r >> 1) & 3)); 16 bytes -> 32 dims -> 16 columns
+                const uint8_t* src = kbuf + (size_t)st * C::KBYTES + r * 64;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 x = *(const uint4*)(src + ((c ^ ((r >> 1) & 3)) << 4));
+                    const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t words[16];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+#pragma unroll
+                        for (int bb = 0; bb < 4; ++bb) words[4 * e + bb] = e2m1x2_to_f16x2((xs[e] >> (8 * bb)) & 0xFFu);
+                    tmem_st16(taddr + c * 16, words);
+                }
+            } else {
+            const uint8_t* src = kbuf + (size_t)st * C::KBYTES + r * 128;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t words[32];
@@ -382,6 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                 for (int m = 0; m < 16; ++m) { lo[m] = words[m]; hi[m] = words[16 + m]; }
                 tmem_st16(taddr + half * 32, lo);
                 tmem_st16(taddr + half * 32 + 16, hi);
+            }
             }
             tmem_st_wait();
             __syncwarp();
@@ -466,16 +498,18 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
 
 namespace {
 
-template <int NQ, bool FP8>
+template <int NQ, int KF>
 cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Params& p) {
-    using C = Cfg<NQ, FP8>;
+    using C = Cfg<NQ, KF>;
     CUtensorMap mk, mq;
     const uint64_t krows = (uint64_t)p.batch * p.ctx;
-    bool ok = FP8 ? make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
+    bool ok = KF == KF_FP4 ? make_map_swizzled(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI / 2, krows, 64, KT,
+                                               CU_TENSOR_MAP_SWIZZLE_64B)
+            : KF == KF_FP8 ? make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
                   : make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, DI, krows, 64, KT);
     ok = ok && make_map_sw128(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DI, (uint64_t)p.rows * HI, 64, NQ * HI);
     if (!ok) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<NQ, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<NQ, KF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM);
     if (e != cudaSuccess) return e;
     int64_t units;
@@ -490,7 +524,7 @@ cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Para
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, indexer_tc_kernel<NQ, FP8>, mk, mq, p);
+    e = cudaLaunchKernelEx(&cfg, indexer_tc_kernel<NQ, KF>, mk, mq, p);
     count_launch();
     return e;
 }
@@ -498,7 +532,8 @@ cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Para
 }  // namespace
 
 bool indexer_tc_supported(dsa_dtype_t q_dtype, dsa_dtype_t k_dtype, int n_heads, int head_dim) {
-    return q_dtype == DSA_BF16 && (k_dtype == DSA_BF16 || k_dtype == DSA_FP8_E4M3) && n_heads == HI &&
+    return q_dtype == DSA_BF16 && (k_dtype == DSA_BF16 || k_dtype == DSA_FP8_E4M3 || k_dtype == DSA_FP4_E2M1) &&
+           n_heads == HI &&
            head_dim == DI;
 }
 
@@ -507,12 +542,13 @@ cudaError_t launch_indexer_tc(const Launch& L, const void* q, dsa_dtype_t k_dtyp
                               int batch, int ctx_len, float* logits, int64_t ld) {
     if (rows == 0 || ctx_len == 0) return cudaSuccess;
     Params p{w, k_scale, row_batch, row_pos, logits, ld, rows, batch, ctx_len, L.err};
-    if (k_dtype == DSA_FP8_E4M3) return launch_cfg<1, true>(L, q, k, p);
+    if (k_dtype == DSA_FP8_E4M3) return launch_cfg<1, KF_FP8>(L, q, k, p);
+    if (k_dtype == DSA_FP4_E2M1) return launch_cfg<1, KF_FP4>(L, q, k, p);
     // Groups of 4 query rows share a key tile only when every row reads the
     // same cache (one sequence): then the MMA N grows to 256 and each key
     // tile is reused for 4 queries.
-    if (batch == 1 && rows >= 4 * L.num_sms) return launch_cfg<4, false>(L, q, k, p);
-    return launch_cfg<1, false>(L, q, k, p);
+    if (batch == 1 && rows >= 4 * L.num_sms) return launch_cfg<4, KF_BF16>(L, q, k, p);
+    return launch_cfg<1, KF_BF16>(L, q, k, p);
 }
 
 }  // namespace dsa

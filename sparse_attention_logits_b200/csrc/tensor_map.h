@@ -25,8 +25,21 @@ inline EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor [rows, cols] with boxes of box_rows x box_cols
-// elements laid out in shared memory with the 128-byte swizzle (box_cols *
-// element size must be at most 128 bytes).
+// elements laid out in shared memory with the given swizzle (box_cols *
+// element size must be at most the swizzle span: 32, 64 or 128 bytes).
+inline bool make_map_swizzled(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same with the 128-byte swizzle.
 inline bool make_map_sw128(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
                            uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();

@@ -57,7 +57,9 @@ def test_compress_bit_exact(cuda_device, dtype, B, L, D, m):
     workloads.PREFILL_16K.with_(ctx=1001, rows=1001),                   # causal, 4 queries per tile, ragged
     workloads.DECODE_128K_FP8_PAGED.with_(batch=2, rows=2, ctx=4096 + 64),
     workloads.DECODE_128K_FP8_PAGED.with_(batch=5, rows=5, ctx=777),    # fp8, ragged tail
-], ids=lambda w: f"{w.name}-ctx{w.ctx}")
+    workloads.DECODE_128K_FP8_PAGED.with_(batch=3, rows=4, ctx=4096 + 64, idx_key_dtype="fp4"),
+    workloads.DECODE_128K_FP8_PAGED.with_(batch=5, rows=5, ctx=777, idx_key_dtype="fp4"),    # fp4, ragged tail
+], ids=lambda w: f"{w.name}-{w.idx_key_dtype}-ctx{w.ctx}")
 def test_indexer_matches_oracle(cuda_device, wl):
     inp = workloads.generate(wl, parts=("indexer",))
     dv = _cuda(inp, cuda_device)
@@ -183,7 +185,8 @@ def test_sparse_mla_all_slots_unused(cuda_device):
     workloads.TINY_PREFILL_FP32,
     workloads.DECODE_32K.with_(batch=4, rows=4, ctx=5000),
     workloads.PREFILL_16K.with_(ctx=1200, rows=1200, topk=256),
-], ids=lambda w: f"{w.name}-ctx{w.ctx}")
+    workloads.DECODE_32K.with_(batch=4, rows=4, ctx=5000, idx_key_dtype="fp4"),
+], ids=lambda w: f"{w.name}-{w.idx_key_dtype}-ctx{w.ctx}")
 def test_chain_matches_oracle(cuda_device, wl):
     inp = workloads.generate(wl)
     dv = _cuda(inp, cuda_device)
@@ -191,7 +194,8 @@ def test_chain_matches_oracle(cuda_device, wl):
                                  wl.topk, wl.softmax_scale, wl.d_v, k_scale=dv.get("k_scale"),
                                  page_table=dv.get("page_table"))
     dsa.get_device_error()
-    scores = oracle.index_scores(inp["q_idx"], inp["w"], inp["k_idx"], inp["row_batch"], inp["row_pos"])
+    scores = oracle.index_scores(inp["q_idx"], inp["w"], inp["k_idx"], inp["row_batch"], inp["row_pos"],
+                                 k_scale=inp.get("k_scale"))
     ref_idx = oracle.topk(scores, inp["row_pos"], wl.topk)
     gidx = idx.cpu().numpy()
     check_sorted_unique(gidx, inp["row_pos"].numpy() + 1)

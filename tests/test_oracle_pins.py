@@ -213,6 +213,39 @@ def test_index_fp8_keys_equal_dequantized_fp32_keys():
     np.testing.assert_allclose(a[fin], b[fin], rtol=1e-6, atol=1e-9)
 
 
+def test_fp4_e2m1_decode_matches_the_format_table():
+    # OCP e2m1: codes 0-7 are the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (exponent
+    # bias 1, one mantissa bit, exponent 0 subnormal); bit 3 is the sign
+    table = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for c in range(16):
+        v = oracle.fp4_e2m1_to_double(c)
+        assert v == (-1.0 if c & 8 else 1.0) * table[c & 7], c
+        assert math.copysign(1.0, v) == (-1.0 if c & 8 else 1.0)
+
+
+def test_index_fp4_keys_equal_dequantized_fp32_keys():
+    g = torch.Generator().manual_seed(13)
+    q = torch.randn(3, 4, 16, generator=g).to(torch.bfloat16)
+    w = torch.rand(3, 4, generator=g)
+    kf = torch.randn(1, 50, 16, generator=g)
+    codes, scale = workloads.quantize_fp4_rows(kf)
+    assert codes.shape == (1, 50, 8)
+    # unpack independently: dim 2j is the low nibble of byte j
+    table = torch.tensor([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    nib = torch.stack([codes & 0xF, codes >> 4], dim=-1).reshape(1, 50, 16).long()
+    val = table[nib & 7] * torch.where(nib >= 8, -1.0, 1.0)
+    deq = val * scale[..., None]
+    # the quantiser picks the nearest magnitude of the scaled value
+    assert (deq - kf).abs().max() <= (scale.max() * 1.0 + 1e-6)
+    rb = torch.zeros(3, dtype=torch.int32)
+    rp = torch.tensor([49, 20, 0], dtype=torch.int32)
+    a = oracle.index_scores(q, w, codes, rb, rp, k_scale=scale)
+    b = oracle.index_scores(q.float(), w, deq, rb, rp)
+    fin = np.isfinite(a)
+    assert np.array_equal(np.isfinite(a), np.isfinite(b))
+    np.testing.assert_allclose(a[fin], b[fin], rtol=1e-6, atol=1e-9)
+
+
 # ------------------------------------------------------------------ top-k ----
 
 def test_topk_hand_fixture():

@@ -48,7 +48,7 @@ class Workload:
     d_qk: int              # D_K (latent + rope)
     d_v: int               # D_V (value = first D_V dims of the latent)
     dtype: str             # "fp32" or "bf16": q, kv, q_I storage and MLA output
-    idx_key_dtype: str     # "fp32", "bf16" or "fp8"
+    idx_key_dtype: str     # "fp32", "bf16", "fp8" or "fp4"
     page_size: int = 0     # 0: contiguous KV cache; else paged MLA KV cache
     compress_m: int = 1    # CSA pooling factor m (raw context = ctx * m)
 
@@ -109,6 +109,25 @@ def quantize_fp8_rows(x: torch.Tensor):
     return codes, scale.to(torch.float32)
 
 
+FP4_E2M1_MAX = 6.0
+_E2M1_MAG = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def quantize_fp4_rows(x: torch.Tensor):
+    """x [..., D] -> (codes uint8 [..., D/2], scale fp32 [...]): e2m1 codes,
+    two per byte (dim 2j in the low nibble), with one scale per row,
+    scale = amax(row) / 6; each value goes to the nearest e2m1 magnitude
+    (ties to the smaller one), saturating at 6."""
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / FP4_E2M1_MAX, torch.ones_like(amax))
+    y = (x / scale.unsqueeze(-1)).clamp(-FP4_E2M1_MAX, FP4_E2M1_MAX)
+    mags = torch.tensor(_E2M1_MAG, dtype=y.dtype, device=y.device)
+    code = (y.abs().unsqueeze(-1) - mags).abs().argmin(dim=-1).to(torch.uint8)
+    code = code | torch.where(y < 0, torch.full_like(code, 8), torch.zeros_like(code))
+    packed = code[..., 0::2] | (code[..., 1::2] << 4)
+    return packed.contiguous(), scale.to(torch.float32)
+
+
 def row_metadata(w: Workload, rows: Optional[int] = None, device="cpu"):
     """row_batch[r]: which cache query row r reads; row_pos[r]: the last key
     position it may see (keys s <= row_pos[r] are visible)."""
@@ -147,6 +166,8 @@ def generate(w: Workload, device="cpu", seed: int = 0, parts=("indexer", "mla"))
         out["w"] = wts
         if w.idx_key_dtype == "fp8":
             out["k_idx"], out["k_scale"] = quantize_fp8_rows(k_idx.to(torch.bfloat16).float())
+        elif w.idx_key_dtype == "fp4":
+            out["k_idx"], out["k_scale"] = quantize_fp4_rows(k_idx.to(torch.bfloat16).float())
         else:
             out["k_idx"] = k_idx.to(_TORCH_DT[w.idx_key_dtype])
     del q_idx, wts, k_idx
