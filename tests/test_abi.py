@@ -88,3 +88,32 @@ def test_invalid_arguments_rejected_before_launch(lib):
                               fake, None, 0, None) == 1
     # zero rows is a no-op success without touching the device
     assert lib.dsa_topk(fake, 100, fake, 0, 100, 5, fake, None, 0, None) == 0
+    # indexer: fp4 keys without scales; fp4 keys with a head geometry no kernel is built for
+    assert lib.dsa_indexer_logits(fake, 1, fake, fake, 3, None, fake, fake, 4, 4, 128, 64, 128, fake, 128, None) == 1
+    assert lib.dsa_indexer_logits(fake, 1, fake, fake, 3, fake, fake, fake, 4, 4, 128, 64, 64, fake, 128, None) == 2
+    assert "fp4" in _err(lib)
+
+
+def test_v4_attention_arguments_rejected_before_launch(lib):
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    fake = vp(0x1000)      # never dereferenced: validation fails first
+    lib.csa_core_attention.argtypes = [vp, vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, ci, vp, vp, ci, ci, ci, ci, ci,
+                                       ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
+
+    def csa(idx, k, kv_win, win_pos, win_len, window, n_heads=128):
+        return lib.csa_core_attention(fake, fake, 1, None, 0, 0, fake, idx, k, 4, 4, 1024, kv_win, win_pos, win_len,
+                                      window, n_heads, 576, 512, 0.04, fake, fake, None, 0, None)
+    assert csa(fake, 64, fake, fake, 4096, -1) == 1                  # negative window
+    assert csa(fake, 64, None, fake, 4096, 128) == 1                 # window without its cache
+    assert csa(fake, 64, fake, None, 4096, 128) == 1                 # window without positions
+    assert csa(None, 0, fake, fake, 4096, 0) == 1                    # no slot at all
+    assert csa(None, 64, fake, fake, 4096, 128) == 1                 # selected slots without an index list
+    assert csa(fake, 64, fake, fake, 4096, 128, n_heads=100) == 2    # no kernel for this geometry
+    lib.hca_attention.argtypes = [vp, vp, ci, vp, vp, ci, ci, ci, ci, ci, ci, ctypes.c_float, vp, vp, vp,
+                                  ctypes.c_size_t, vp]
+    assert lib.hca_attention(fake, fake, 1, fake, None, 4, 4, 8192, 128, 576, 512, 0.04, fake, fake, None, 0,
+                             None) == 1                              # no row_last
+    assert lib.hca_attention(fake, fake, 1, fake, fake, 4, 4, 8192, 96, 576, 512, 0.04, fake, fake, None, 0,
+                             None) == 2                              # no kernel for this geometry
+    assert lib.hca_attention(fake, fake, 1, fake, fake, 0, 4, 8192, 128, 576, 512, 0.04, fake, fake, None, 0,
+                             None) == 0                              # zero rows: nothing to do
