@@ -113,7 +113,7 @@ def test_v4_attention_arguments_rejected_before_launch(lib):
                                   ctypes.c_size_t, vp]
     assert lib.hca_attention(fake, fake, 1, fake, None, 4, 4, 8192, 128, 576, 512, 0.04, fake, fake, None, 0,
                              None) == 1                              # no row_last
-    assert lib.hca_attention(fake, fake, 1, fake, fake, 4, 4, 8192, 96, 576, 512, 0.04, fake, fake, None, 0,
+    assert lib.hca_attention(fake, fake, 1, fake, fake, 4, 4, 8192, 100, 576, 512, 0.04, fake, fake, None, 0,
                              None) == 2                              # no kernel for this geometry
     assert lib.hca_attention(fake, fake, 1, fake, fake, 0, 4, 8192, 128, 576, 512, 0.04, fake, fake, None, 0,
                              None) == 0                              # zero rows: nothing to do
