@@ -44,7 +44,7 @@ def build(force: bool = False) -> str:
         return _LIB_PATH
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
-                           "-Wall", "-Wno-unknown-pragmas", _SRC, "-o", tmp, "-lm"])
+                           "-Wall", "-Wno-unknown-pragmas", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -78,6 +78,23 @@ def lib():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, ctypes.c_double, _I32P, ctypes.c_int,
                                             _F64P, _F64P, _F64P]
+            L.oracle_rms_norm.restype = None
+            L.oracle_rms_norm.argtypes = [_F64P, _F64P, ctypes.c_int, ctypes.c_int, ctypes.c_double, _F64P]
+            L.oracle_rope.restype = None
+            L.oracle_rope.argtypes = [_F64P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32P,
+                                      _F32P, _F32P]
+            L.oracle_indexer_prepare.restype = None
+            L.oracle_indexer_prepare.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, _F32P,
+                                                 ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_int, _F32P, _F32P, _I32P]
+            L.oracle_indexer_prepare.argtypes += [ctypes.c_int] * 6 + [_F64P, _F64P, _F64P]
+            L.oracle_fp8_e4m3_encode.restype = ctypes.c_uint8
+            L.oracle_fp8_e4m3_encode.argtypes = [ctypes.c_float]
+            L.oracle_fp4_e2m1_encode.restype = ctypes.c_uint8
+            L.oracle_fp4_e2m1_encode.argtypes = [ctypes.c_float]
+            L.oracle_key_rows_f32.restype = None
+            L.oracle_key_rows_f32.argtypes = [_F32P, ctypes.c_int, ctypes.c_int, ctypes.c_int, _I32P, _F32P,
+                                              _F32P, ctypes.c_int, ctypes.c_void_p, _F32P]
             L.oracle_max_threads.restype = ctypes.c_int
             L.oracle_max_threads.argtypes = []
             _lib = L
@@ -136,6 +153,16 @@ def fp4_e2m1_to_double(code: int) -> float:
 
 def double_to_bf16_bits(x: float) -> int:
     return int(lib().oracle_double_to_bf16_rne(float(x)))
+
+
+def fp8_e4m3_encode(y: float) -> int:
+    """Nearest e4m3 code of a binary32 value (ties to even, saturating at 448)."""
+    return int(lib().oracle_fp8_e4m3_encode(float(y)))
+
+
+def fp4_e2m1_encode(y: float) -> int:
+    """Nearest e2m1 code (one nibble) of a binary32 value (ties to even, saturating at 6)."""
+    return int(lib().oracle_fp4_e2m1_encode(float(y)))
 
 
 # ---- the path -------------------------------------------------------------------
@@ -269,3 +296,85 @@ def hca_attention(q, kv, row_batch, row_last, scale: float, d_v: int):
     idx = torch.where(ar <= last, ar, torch.full_like(ar, -1)).to(torch.int32)
     out, lse, _ = sparse_mla(q, kv, idx, row_batch, scale, d_v, L)
     return out, lse
+
+
+# ---- preparation of the indexer's inputs (the step before the path) -----------
+
+def rms_norm(x, gamma, eps: float) -> np.ndarray:
+    """RMSNorm of each row of x [n, d] (float64 result)."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64))
+    n, d = a.shape
+    out = np.empty_like(a)
+    lib().oracle_rms_norm(_p(a, _F64P), _p(g, _F64P), n, d, float(eps), _p(out, _F64P))
+    return out
+
+
+def rope(x, pos, rope_cos, rope_sin, d_rope: int) -> np.ndarray:
+    """Rotary encoding of x [n, heads, d] (float64 copy): pairs (2i, 2i+1),
+    i < d_rope/2, of every head turned by the angle of row pos[r] of the
+    [max_pos, d_rope/2] cosine / sine tables."""
+    a = np.array(np.asarray(x, dtype=np.float64), copy=True, order="C")
+    n, heads, d = a.shape
+    c = np.ascontiguousarray(_host(rope_cos), dtype=np.float32)
+    s = np.ascontiguousarray(_host(rope_sin), dtype=np.float32)
+    lib().oracle_rope(_p(a, _F64P), n, heads, d, int(d_rope), _p(_i32(pos), _I32P), _p(c, _F32P), _p(s, _F32P))
+    return a
+
+
+def indexer_prepare(c_q, gamma, eps: float, wq_b, h, wk, w_proj, rope_cos, rope_sin, pos, n_heads: int,
+                    d_rope: int):
+    """Inputs of the lightning indexer for T tokens (float64):
+    q [T, n_heads, head_dim] = RoPE(W_qb . RMSNorm(c_q)), w [T, n_heads] = W_w . h,
+    k [T, head_dim] = RoPE(W_k . h).  Activations c_q [T, d_c], h [T, d_model]
+    and the weights W_qb [n_heads*head_dim, d_c], W_k [head_dim, d_model],
+    W_w [n_heads, d_model] are bf16 or fp32 tensors (all activations one
+    type, all weights one type)."""
+    cq, hh = _host(c_q), _host(h)
+    wqb, wkk, wpj = _host(wq_b), _host(wk), _host(w_proj)
+    assert cq.dtype == hh.dtype and wqb.dtype == wkk.dtype == wpj.dtype
+    T, d_c = cq.shape
+    d_model = hh.shape[1]
+    head_dim = wkk.shape[0]
+    assert wqb.shape == (n_heads * head_dim, d_c) and wpj.shape == (n_heads, d_model) and hh.shape[0] == T
+    g = np.ascontiguousarray(_host(gamma), dtype=np.float32)
+    c = np.ascontiguousarray(_host(rope_cos), dtype=np.float32)
+    s = np.ascontiguousarray(_host(rope_sin), dtype=np.float32)
+    q = np.empty((T, n_heads, head_dim), dtype=np.float64)
+    w = np.empty((T, n_heads), dtype=np.float64)
+    k = np.empty((T, head_dim), dtype=np.float64)
+    lib().oracle_indexer_prepare(cq.ctypes.data, hh.ctypes.data, _dtype_code(cq), _p(g, _F32P), float(eps),
+                                 wqb.ctypes.data, wkk.ctypes.data, wpj.ctypes.data, _dtype_code(wqb),
+                                 _p(c, _F32P), _p(s, _F32P), _p(_i32(pos), _I32P), T, d_c, d_model, n_heads,
+                                 head_dim, int(d_rope), _p(q, _F64P), _p(w, _F64P), _p(k, _F64P))
+    return q, w, k
+
+
+def key_rows_f32(x, pos, rope_cos, rope_sin, d_rope: int, fmt: int):
+    """The key-cache write decided in binary32: RoPE of dims [0, d_rope) of
+    each row of x [n, d] (separately rounded products and sums), then the
+    stored form: fmt BF16 -> (uint16 bits [n, d], None); FP8 -> (codes uint8
+    [n, d], scale float32 [n]); FP4 -> (code pairs uint8 [n, d/2], scale).
+    x is first rounded to binary32 (exact for bf16 and fp32 inputs)."""
+    a = np.array(np.asarray(_to_f32(x)), dtype=np.float32, copy=True, order="C")
+    n, d = a.shape
+    c = np.ascontiguousarray(_host(rope_cos), dtype=np.float32)
+    s = np.ascontiguousarray(_host(rope_sin), dtype=np.float32)
+    if fmt == BF16:
+        out = np.zeros((n, d), dtype=np.uint16)
+    elif fmt == FP8:
+        out = np.zeros((n, d), dtype=np.uint8)
+    elif fmt == FP4:
+        out = np.zeros((n, d // 2), dtype=np.uint8)
+    else:
+        raise ValueError("fmt must be BF16, FP8 or FP4")
+    scale = np.ones(n, dtype=np.float32)
+    lib().oracle_key_rows_f32(_p(a, _F32P), n, d, int(d_rope), _p(_i32(pos), _I32P), _p(c, _F32P), _p(s, _F32P),
+                              int(fmt), out.ctypes.data, _p(scale, _F32P))
+    return out, (None if fmt == BF16 else scale)
+
+
+def _to_f32(x) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        return x.detach().cpu().float().numpy()
+    return np.asarray(x, dtype=np.float32)

@@ -31,6 +31,28 @@
  *                        heads, value = first D_V dims of the latent (same
  *                        article, sections 1.3 细粒度稀疏注意力, 1.4 and 3 Step 4).
  *
+ *
+ * and the step before the path, the preparation of the indexer's inputs
+ * ("DeepSeek-V3.2稀疏注意力机制原理与TPU适配", section 3, Step 1: low-rank
+ * projections, RMSNorm of the query latent, the split into parts with and
+ * without rotary position encoding, apply_rotary_emb, weights_proj; section
+ * 1.3: a separate learned linear map takes query and key to 128 dims):
+ *
+ *  oracle_rms_norm       x / sqrt(mean(x^2) + eps) * gamma, per row.
+ *  oracle_rope           rotary position encoding of the first d_rope dims
+ *                        of each head: pair (2i, 2i+1) turned by the angle
+ *                        whose cosine and sine the table gives at (pos, i).
+ *  oracle_indexer_prepare  q_I = RoPE(W_qb . RMSNorm(c_q)) per head,
+ *                        w = W_w . h, k_I = RoPE(W_k . h), in double.
+ *  oracle_fp8_e4m3_encode / oracle_fp4_e2m1_encode  round a binary32 value
+ *                        to the nearest code, ties to the even code,
+ *                        saturating at the largest finite magnitude.
+ *  oracle_key_rows_f32   the key-cache write in binary32 arithmetic (the
+ *                        precision in which the stored codes are decided):
+ *                        RoPE with separately rounded products and sums,
+ *                        then per row scale = amax / qmax and code =
+ *                        encode(x / scale).
+ *
  * Parity pins (tests/test_oracle_pins.py) check each function against closed
  * forms, brute force, hand-computed fixtures and library routines.  The one
  * point left unpinned is whether the lost index-score formula carried an
@@ -308,4 +330,161 @@ int oracle_max_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ---- indexer input preparation (DSA article, section 3, Step 1) -------- */
+
+/* RMSNorm of each of the n rows of x [n, d]: x / sqrt(mean(x^2) + eps) * gamma. */
+void oracle_rms_norm(const double* x, const double* gamma, int n, int d, double eps, double* out)
+{
+    for (int r = 0; r < n; ++r) {
+        double ss = 0.0;
+        for (int j = 0; j < d; ++j) ss += x[(int64_t)r * d + j] * x[(int64_t)r * d + j];
+        double inv = 1.0 / sqrt(ss / d + eps);
+        for (int j = 0; j < d; ++j) out[(int64_t)r * d + j] = x[(int64_t)r * d + j] * inv * gamma[j];
+    }
+}
+
+/* Rotary position encoding, in place, of x [n, heads, d]: in every head, dims
+ * 2i and 2i+1 (i < d_rope/2) are turned by the angle of row pos[r] of the
+ * tables: (a, b) -> (a cos - b sin, a sin + b cos).  The tables are
+ * [max_pos, d_rope/2]; dims d_rope .. d-1 carry no position. */
+void oracle_rope(double* x, int n, int heads, int d, int d_rope, const int32_t* pos,
+                 const float* cos_t, const float* sin_t)
+{
+    int half = d_rope / 2;
+    for (int r = 0; r < n; ++r)
+        for (int h = 0; h < heads; ++h) {
+            double* v = x + ((int64_t)r * heads + h) * d;
+            for (int i = 0; i < half; ++i) {
+                double c = cos_t[(int64_t)pos[r] * half + i], s = sin_t[(int64_t)pos[r] * half + i];
+                double a = v[2 * i], b = v[2 * i + 1];
+                v[2 * i] = a * c - b * s;
+                v[2 * i + 1] = a * s + b * c;
+            }
+        }
+}
+
+static double* load_all(const void* p, int dtype, int64_t n)
+{
+    double* out = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    for (int64_t i = 0; i < n; ++i) out[i] = load_elem(p, dtype, i);
+    return out;
+}
+
+/* out[r, o] = sum_j W[o, j] * x[r, j]  (W [n_out, d] row-major: the linear
+ * map of a PyTorch-style weight). */
+static void linear(const double* x, const double* W, int n, int d, int n_out, double* out)
+{
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int r = 0; r < n; ++r)
+        for (int o = 0; o < n_out; ++o) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += W[(int64_t)o * d + j] * x[(int64_t)r * d + j];
+            out[(int64_t)r * n_out + o] = acc;
+        }
+}
+
+/* Inputs of the lightning indexer for T tokens, in the order of Step 1:
+ *   q_out [T, n_heads, head_dim] = RoPE( W_qb . RMSNorm(c_q; gamma, eps) )
+ *   w_out [T, n_heads]           = W_w . h
+ *   k_out [T, head_dim]          = RoPE( W_k . h )
+ * c_q [T, d_c] is the query latent (the low-rank projection the MLA query
+ * shares), h [T, d_model] the hidden states; W_qb [n_heads*head_dim, d_c],
+ * W_k [head_dim, d_model], W_w [n_heads, d_model]; act_dtype / w_dtype are
+ * the element formats of the activations and of the weights. */
+void oracle_indexer_prepare(const void* c_q, const void* h, int act_dtype, const float* gamma, double eps,
+                            const void* wq_b, const void* wk, const void* w_proj, int w_dtype,
+                            const float* cos_t, const float* sin_t, const int32_t* pos,
+                            int T, int d_c, int d_model, int n_heads, int head_dim, int d_rope,
+                            double* q_out, double* w_out, double* k_out)
+{
+    double* c = load_all(c_q, act_dtype, (int64_t)T * d_c);
+    double* x = load_all(h, act_dtype, (int64_t)T * d_model);
+    double* g = (double*)malloc(sizeof(double) * (size_t)d_c);
+    for (int j = 0; j < d_c; ++j) g[j] = gamma[j];
+    double* cn = (double*)malloc(sizeof(double) * (size_t)T * d_c + 8);
+    oracle_rms_norm(c, g, T, d_c, eps, cn);
+
+    double* W = load_all(wq_b, w_dtype, (int64_t)n_heads * head_dim * d_c);
+    linear(cn, W, T, d_c, n_heads * head_dim, q_out);
+    free(W);
+    oracle_rope(q_out, T, n_heads, head_dim, d_rope, pos, cos_t, sin_t);
+
+    W = load_all(w_proj, w_dtype, (int64_t)n_heads * d_model);
+    linear(x, W, T, d_model, n_heads, w_out);
+    free(W);
+
+    W = load_all(wk, w_dtype, (int64_t)head_dim * d_model);
+    linear(x, W, T, d_model, head_dim, k_out);
+    free(W);
+    oracle_rope(k_out, T, 1, head_dim, d_rope, pos, cos_t, sin_t);
+
+    free(c); free(x); free(g); free(cn);
+}
+
+/* Nearest code of a finite binary32 value among the non-negative codes
+ * 0 .. last of a format (ascending in value), ties to the even code (the
+ * code's last bit is the mantissa's last bit), the sign bit added after. */
+static unsigned encode_nearest_even(float y, int last, int sign_bit, double (*decode)(uint8_t))
+{
+    double a = fabs((double)y);
+    int best = 0;
+    double bd = INFINITY;
+    for (int c = 0; c <= last; ++c) {
+        double d = fabs(decode((uint8_t)c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            bd = d;
+            best = c;
+        }
+    }
+    return (unsigned)best | (signbit(y) ? (1u << sign_bit) : 0u);
+}
+
+/* E4M3: magnitudes are codes 0 .. 0x7E (0x7F is NaN); above 448 saturates. */
+uint8_t oracle_fp8_e4m3_encode(float y) { return (uint8_t)encode_nearest_even(y, 0x7E, 7, oracle_fp8_e4m3_to_double); }
+
+/* E2M1: magnitudes are codes 0 .. 7; above 6 saturates.  Returns one nibble. */
+uint8_t oracle_fp4_e2m1_encode(float y) { return (uint8_t)encode_nearest_even(y, 7, 3, oracle_fp4_e2m1_to_double); }
+
+/* The key-cache write, in binary32 (every product and sum rounded on its
+ * own, no fused multiply-add): x [n, d] binary32 rows (already projected),
+ * RoPE of dims [0, d_rope) at pos[r], then
+ *   fmt ODT_BF16:     out [n, d] bf16 bits (nearest-even), no scale
+ *   fmt ODT_FP8_E4M3: scale = amax / 448 (1 for a zero row), out [n, d] codes of x / scale
+ *   fmt ODT_FP4_E2M1: scale = amax / 6, out [n, d/2] code pairs, element 2j in the low nibble
+ * x is overwritten by the rotated values. */
+void oracle_key_rows_f32(float* x, int n, int d, int d_rope, const int32_t* pos, const float* cos_t,
+                         const float* sin_t, int fmt, void* out, float* scale)
+{
+    int half = d_rope / 2;
+    for (int r = 0; r < n; ++r) {
+        float* v = x + (int64_t)r * d;
+        for (int i = 0; i < half; ++i) {
+            float c = cos_t[(int64_t)pos[r] * half + i], s = sin_t[(int64_t)pos[r] * half + i];
+            float a = v[2 * i], b = v[2 * i + 1];
+            float ac = a * c, bs = b * s, as = a * s, bc = b * c;
+            v[2 * i] = ac - bs;
+            v[2 * i + 1] = as + bc;
+        }
+        if (fmt == ODT_BF16) {
+            for (int j = 0; j < d; ++j) ((uint16_t*)out)[(int64_t)r * d + j] = oracle_double_to_bf16_rne((double)v[j]);
+            continue;
+        }
+        float amax = 0.0f;
+        for (int j = 0; j < d; ++j) amax = fabsf(v[j]) > amax ? fabsf(v[j]) : amax;
+        float qmax = fmt == ODT_FP8_E4M3 ? 448.0f : 6.0f;
+        float sc = amax > 0.0f ? amax / qmax : 1.0f;
+        scale[r] = sc;
+        for (int j = 0; j < d; ++j) {
+            float y = v[j] / sc;
+            if (fmt == ODT_FP8_E4M3) {
+                ((uint8_t*)out)[(int64_t)r * d + j] = oracle_fp8_e4m3_encode(y);
+            } else {
+                uint8_t* o = (uint8_t*)out + (int64_t)r * (d / 2) + j / 2;
+                uint8_t code = oracle_fp4_e2m1_encode(y);
+                *o = (j & 1) ? (uint8_t)((*o & 0x0F) | (code << 4)) : (uint8_t)((*o & 0xF0) | code);
+            }
+        }
+    }
 }
