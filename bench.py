@@ -527,6 +527,8 @@ def run_ours(args):
         result["other_decodes"] = run_other_decodes(dsa, workloads, device, peaks, args)
     if args.v4:
         result["v4_variants"] = run_v4_variants(dsa, workloads, device, peaks, args)
+    if args.prepare:
+        result["indexer_prepare"] = run_prepare(dsa, workloads, device, peaks, args)
     if world == 1 and rank == 0 and args.cpu_baseline:
         qps, n, cores, secs = cpu_baseline_decode(wl, inp)
         result["cpu_baseline"] = {"value": round(qps, 4), "unit": "queries/s", "cores": cores, "kind": "oracle",
@@ -697,6 +699,87 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
     return {"csa_core_attention_decode": csa, "hca_decode": hca}
 
 
+PREP_D_C, PREP_D_MODEL = 1536, 7168      # query latent and hidden size of a V3-class model
+
+
+def run_prepare(dsa, workloads, device, peaks, args):
+    """The step before the path: the indexer's queries, head weights and keys
+    from the query latent and the hidden states (one dsa_indexer_prepare
+    call: three projections, RMSNorm, rotary encoding, the key-cache write).
+
+    decode: 64 new tokens (one per sequence of the 128K fp8-key decode), keys
+      appended to the 64 x 131072-row fp8 cache.  Memory-bound: the roofline
+      is the bytes that must cross HBM once (weights, activations, outputs)
+      over the event time, with a 256 MB buffer read between replays (the
+      30 MB of weights would otherwise stay in L2).
+    prefill: 16384 tokens of one sequence (bf16 key cache), against the bf16
+      tensor peak."""
+    import torch
+    rank, world, _ = dist_env()
+    H, D, d_rope = 64, 128, 64
+    evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    out = {}
+    for name, T, fmt, rows_cache, max_pos in (
+            (f"indexer_prepare_decode_T64_dc{PREP_D_C}_d{PREP_D_MODEL}_fp8cache", 64, "fp8", 64 * 131072, 131072),
+            (f"indexer_prepare_prefill_T16384_dc{PREP_D_C}_d{PREP_D_MODEL}_bf16cache", 16384, "bf16", 16384, 16384)):
+        shape = workloads.PrepareShape(T, PREP_D_C, PREP_D_MODEL, n_heads=H, head_dim=D, d_rope=d_rope,
+                                       max_pos=max_pos, cache_rows=rows_cache)
+        inp = {k: v.to(device) for k, v in workloads.make_prepare_inputs(shape, seed=300 + rank, skip=0.0).items()}
+        if fmt == "fp8":
+            cache = torch.zeros((rows_cache, D), dtype=torch.uint8, device=device)
+            scale = torch.ones(rows_cache, dtype=torch.float32, device=device)
+            seq = torch.arange(T, device=device, dtype=torch.int64)
+            inp["pos"] = torch.full((T,), max_pos - 1, dtype=torch.int32, device=device)
+            inp["slot"] = seq * 131072 + (max_pos - 1)         # each sequence's newest position
+        else:
+            cache = torch.zeros((rows_cache, D), dtype=torch.bfloat16, device=device)
+            scale = None
+            inp["pos"] = torch.arange(T, dtype=torch.int32, device=device)
+            inp["slot"] = torch.arange(T, dtype=torch.int64, device=device)
+        q_out = torch.empty((T, H, D), dtype=torch.bfloat16, device=device)
+        w_out = torch.empty((T, H), dtype=torch.float32, device=device)
+        ws = torch.empty(max(dsa.indexer_prepare_workspace_size(T, H, PREP_D_C, PREP_D_MODEL), 1), dtype=torch.uint8,
+                         device=device)
+
+        def call():
+            dsa.indexer_prepare(inp["c_q"], inp["gamma"], inp["wq_b"], inp["h"], inp["wk"], inp["w_proj"],
+                                inp["pos"], inp["slot"], cache, scale, inp["rope_cos"], inp["rope_sin"],
+                                q_out=q_out, w_out=w_out, workspace=ws)
+
+        n0 = dsa.launch_count()
+        g = _graph(call)
+        launches = (dsa.launch_count() - n0) // 2
+        for _ in range(3):
+            g.replay()
+        steps = max(5, args.steps)
+        ms = max_over_ranks(time_graph(g, steps, device, flush_read=evict), device)
+        del g
+        dsa.get_device_error(device)
+        w_bytes = (H * D * PREP_D_C + D * PREP_D_MODEL + H * PREP_D_MODEL) * 2 + PREP_D_C * 4
+        a_bytes = T * (PREP_D_C + PREP_D_MODEL) * 2 + T * (4 + 8)
+        o_bytes = T * H * D * 2 + T * H * 4 + T * (D + 4 if fmt == "fp8" else 2 * D)
+        hbm = w_bytes + a_bytes + o_bytes
+        flops = 2 * T * (H * D * PREP_D_C + (D + H) * PREP_D_MODEL)
+        rec = {"workload": name, "value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
+               "ms_per_call": round(ms, 4), "gpu_launches": launches,
+               "l2": "256 MB buffer read between replays"}
+        if T <= 128:
+            ach = hbm / (ms / 1e3) / 1e9
+            rec["roofline"] = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": round(ach / peaks["hbm_gbs"], 4), "algorithmic_bytes": hbm}
+        else:
+            ach = flops / (ms / 1e3) / 1e12
+            rec["roofline"] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
+                               "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
+                               "algorithmic_flops": flops}
+        out["decode" if T <= 128 else "prefill"] = rec
+        del inp, cache, scale, q_out, w_out, ws
+        torch.cuda.empty_cache()
+    del evict
+    torch.cuda.empty_cache()
+    return out
+
+
 def _finish():
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -748,6 +831,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="dsa_decode_bf16_B32_L32768_k2048")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false")
     ap.add_argument("--no-v4", dest="v4", action="store_false")
+    ap.add_argument("--no-prepare", dest="prepare", action="store_false")
     ap.add_argument("--no-other-decodes", dest="others", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla"], default=None,

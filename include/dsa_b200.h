@@ -13,6 +13,12 @@
  *   csa_core_attention  CSA: the selected compressed entries plus a window of raw rows
  *   hca_attention       HCA: dense attention over every visible heavily compressed entry
  *
+ * and the step before the path, which makes the indexer's inputs:
+ *
+ *   dsa_indexer_prepare     indexer queries, head weights and keys from the hidden
+ *                           states and the query latent; keys written into the cache
+ *   dsa_indexer_key_append  the key-cache write alone, for keys already projected
+ *
  * Conventions shared by every entry point
  *   - Every data pointer is a DEVICE pointer owned by the caller.  The library
  *     never allocates or frees device memory; scratch space, where a step
@@ -281,11 +287,87 @@ DSA_API dsa_status_t dsa_sparse_mla_noalloc(const void* q, const void* kv, dsa_d
                             int rows, int batch, int ctx_len, int n_heads, int d_qk, int d_v,
                             float scale, void* out, float* lse, void* stream);
 
+/* Workspace bytes dsa_indexer_prepare needs for these sizes on the current
+ * device (0 when tokens == 0). */
+DSA_API size_t dsa_indexer_prepare_workspace_size(int tokens, int n_heads, int d_c, int d_model);
+
+/*
+ * dsa_indexer_prepare -- the indexer's inputs for `tokens` new tokens (DSA
+ * article, section 3, Step 1: the query latent is RMS-normalised and
+ * projected up, the result split into a part with and a part without rotary
+ * position encoding, the former turned by apply_rotary_emb, and weights_proj
+ * gives the per-head weights; section 1.3: a learned linear map takes query
+ * and key to 128 dims), all in one launch on the tensor cores:
+ *
+ *   q_out[t, j, :] = RoPE( W_qb[j*128 .. j*128+127] . RMSNorm(c_q[t]) )
+ *   w_out[t, :]    = W_w . h[t]
+ *   key row        = RoPE( W_k . h[t] ), written to row slot[t] of the cache
+ *
+ *   RMSNorm(x)  = x / sqrt(mean(x^2) + eps) * q_norm_weight
+ *   RoPE        turns dims (2i, 2i+1), i < d_rope/2, of every 128-dim head by
+ *               the angle whose cosine / sine are rope_cos / rope_sin[pos[t], i]:
+ *               (a, b) -> (a cos - b sin, a sin + b cos); dims >= d_rope carry
+ *               no position.
+ *
+ *   c_q           [tokens, d_c] bf16: the low-rank query latent (before its norm)
+ *   q_norm_weight [d_c] fp32, the norm's gain; eps >= 0
+ *   wq_b          [n_heads * 128, d_c] bf16 (row-major, out x in)
+ *   h             [tokens, d_model] bf16 hidden states
+ *   wk            [128, d_model] bf16;  w_proj [n_heads, d_model] bf16
+ *   rope_cos, rope_sin  [max_pos, d_rope / 2] fp32 (may be NULL when d_rope = 0)
+ *   pos           [tokens] int32 position of each token, in [0, max_pos) when d_rope > 0
+ *   slot          [tokens] int64 cache row of each token's key, in [0, cache_rows),
+ *                 or -1: the key is not stored
+ *   q_out         [tokens, n_heads, 128] bf16;  w_out [tokens, n_heads] fp32
+ *   k_cache       [cache_rows, 128] of k_dtype: DSA_BF16 (rounded to nearest even),
+ *                 DSA_FP8_E4M3 (codes) or DSA_FP4_E2M1 ([cache_rows, 64] code pairs,
+ *                 element 2j in the low nibble); k_scale [cache_rows] fp32 for fp8 /
+ *                 fp4 (NULL for bf16): scale = amax / 448 (fp8) or amax / 6 (fp4) of
+ *                 the rotated row (1 for an all-zero row), code = the nearest code of
+ *                 value / scale, ties to even, saturating at the largest finite code;
+ *                 all of it in binary32 with every operation rounded on its own
+ *   workspace     dsa_indexer_prepare_workspace_size() bytes, 256-byte aligned; no
+ *                 part of it needs to hold anything on entry (it carries the fp32
+ *                 partial sums of the key and weight projections, which a second
+ *                 kernel adds up in a fixed order)
+ * The projections multiply bf16 operands with fp32 accumulation; the norm's
+ * gain is applied to c_q in bf16 (c_q * gain rounded once) and 1/RMS (fp32)
+ * to the product.  head_dim must be 128; d_c and d_model multiples of 64,
+ * d_c <= 16384;
+ * n_heads <= 256; d_rope even and <= 128.  c_q, h, the weights,
+ * q_norm_weight and q_out 16-byte aligned.  Rows of other tokens in the cache
+ * are not touched.  A token whose position or slot is out of range is
+ * skipped and recorded in the device error word (dsa_get_device_error()
+ * then returns DSA_ERR_INVALID_ARG).
+ */
+DSA_API dsa_status_t dsa_indexer_prepare(const void* c_q, const float* q_norm_weight, float eps, const void* wq_b,
+                                         const void* h, const void* wk, const void* w_proj, const float* rope_cos,
+                                         const float* rope_sin, int max_pos, int d_rope, const int32_t* pos,
+                                         const int64_t* slot, int tokens, int d_c, int d_model, int n_heads,
+                                         int head_dim, void* q_out, float* w_out, void* k_cache, dsa_dtype_t k_dtype,
+                                         float* k_scale, int64_t cache_rows, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
+ * dsa_indexer_key_append -- the key-cache write of dsa_indexer_prepare alone,
+ * for n key rows that are already projected (for instance the pooled keys
+ * of csa_compress): row r of k (fp32 or bf16, [n, 128]) is turned by RoPE at
+ * pos[r] (dims below d_rope) and written to cache row slot[r] (-1: skipped)
+ * in the cache's format, with the same rounding rules.  head_dim must be
+ * 128; k and k_cache 16-byte aligned.
+ */
+DSA_API dsa_status_t dsa_indexer_key_append(const void* k, dsa_dtype_t k_in_dtype, const float* rope_cos,
+                                            const float* rope_sin, int max_pos, int d_rope, const int32_t* pos,
+                                            const int64_t* slot, int n, int head_dim, void* k_cache,
+                                            dsa_dtype_t k_dtype, float* k_scale, int64_t cache_rows, void* stream);
+
 /*
  * dsa_get_device_error -- synchronizes `stream`, then reads and clears the
  * library's device error word on the current device.  Returns DSA_OK when
  * no kernel recorded an error, DSA_ERR_DEVICE_TIMEOUT when a kernel gave up
- * a bounded wait, DSA_ERR_CUDA when the synchronization itself failed.
+ * a bounded wait, DSA_ERR_INVALID_ARG when a kernel met an index, position
+ * or slot out of range and skipped it, DSA_ERR_CUDA when the synchronization
+ * itself failed.
  */
 DSA_API dsa_status_t dsa_get_device_error(void* stream);
 

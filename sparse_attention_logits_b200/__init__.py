@@ -56,6 +56,11 @@ _SIGS = {
                                   _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
     "hca_attention": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
                              _vp]),
+    "dsa_indexer_prepare_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
+    "dsa_indexer_prepare": (_i32, [_vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32,
+                                   _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _sz, _vp]),
+    "dsa_indexer_key_append": (_i32, [_vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _vp, _i32, _vp, _i64,
+                                      _vp]),
     "dsa_get_device_error": (_i32, [_vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -296,6 +301,76 @@ def sparse_mla_noalloc(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row
                                            _ptr(row_batch), _ptr(idx), k, rows, B, ctx_len, H, DK, d_v, float(scale),
                                            _ptr(out), _ptr(lse), _stream(dev)), "dsa_sparse_mla_noalloc")
     return out, lse
+
+
+def _key_cache_fmt(k_cache: torch.Tensor) -> Tuple[int, int]:
+    """(format, rows) of an indexer key cache: bf16 [..., 128], fp8 codes
+    (uint8 / float8_e4m3fn) [..., 128] or fp4 code pairs (uint8) [..., 64]."""
+    last = k_cache.shape[-1]
+    rows = k_cache.numel() // last if last else 0
+    if k_cache.dtype == torch.bfloat16 and last == 128:
+        return DSA_BF16, rows
+    if k_cache.dtype in (torch.uint8, torch.float8_e4m3fn) and last == 128:
+        return DSA_FP8_E4M3, rows
+    if k_cache.dtype == torch.uint8 and last == 64:
+        return DSA_FP4_E2M1, rows
+    raise TypeError("key cache must be bf16 [..., 128], fp8 [..., 128] or fp4 pairs uint8 [..., 64]")
+
+
+def indexer_prepare_workspace_size(tokens: int, n_heads: int, d_c: int, d_model: int) -> int:
+    return int(_lib.dsa_indexer_prepare_workspace_size(tokens, n_heads, d_c, d_model))
+
+
+def indexer_prepare(c_q: torch.Tensor, q_norm_weight: torch.Tensor, wq_b: torch.Tensor, h: torch.Tensor,
+                    wk: torch.Tensor, w_proj: torch.Tensor, pos: torch.Tensor, slot: torch.Tensor,
+                    k_cache: torch.Tensor, k_scale: Optional[torch.Tensor] = None,
+                    rope_cos: Optional[torch.Tensor] = None, rope_sin: Optional[torch.Tensor] = None,
+                    eps: float = 1e-6, q_out: Optional[torch.Tensor] = None, w_out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Indexer inputs of T new tokens: (q_out [T, H, 128] bf16, w_out [T, H]
+    fp32); each token's key is written to row slot[t] of k_cache (-1: not
+    stored).  d_rope = 2 * rope_cos.shape[1] (0 without tables)."""
+    dev = _dev(c_q, q_norm_weight, wq_b, h, wk, w_proj, pos, slot, k_cache, k_scale, rope_cos, rope_sin, q_out,
+               w_out, workspace)
+    T, d_c = c_q.shape
+    d_model = h.shape[1]
+    head_dim = wk.shape[0]
+    H = w_proj.shape[0]
+    fmt, rows = _key_cache_fmt(k_cache)
+    d_rope = 0 if rope_cos is None else 2 * rope_cos.shape[1]
+    max_pos = 0 if rope_cos is None else rope_cos.shape[0]
+    if q_out is None:
+        q_out = torch.empty((T, H, head_dim), dtype=torch.bfloat16, device=dev)
+    if w_out is None:
+        w_out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(indexer_prepare_workspace_size(T, H, d_c, d_model), 1), dtype=torch.uint8,
+                                device=dev)
+    wsb = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(dev):
+        _check(_lib.dsa_indexer_prepare(_ptr(c_q), _ptr(q_norm_weight), float(eps), _ptr(wq_b), _ptr(h), _ptr(wk),
+                                        _ptr(w_proj), _ptr(rope_cos), _ptr(rope_sin), max_pos, d_rope, _ptr(pos),
+                                        _ptr(slot), T, d_c, d_model, H, head_dim, _ptr(q_out), _ptr(w_out),
+                                        _ptr(k_cache), fmt, _ptr(k_scale), rows, _ptr(workspace), wsb,
+                                        _stream(dev)), "dsa_indexer_prepare")
+    return q_out, w_out
+
+
+def indexer_key_append(k: torch.Tensor, slot: torch.Tensor, k_cache: torch.Tensor,
+                       k_scale: Optional[torch.Tensor] = None, pos: Optional[torch.Tensor] = None,
+                       rope_cos: Optional[torch.Tensor] = None, rope_sin: Optional[torch.Tensor] = None) -> None:
+    """Write already-projected key rows k [n, 128] (fp32 or bf16) into rows
+    slot[r] of the key cache (RoPE of the first 2 * rope_cos.shape[1] dims
+    at pos[r] first, when tables are given)."""
+    dev = _dev(k, slot, k_cache, k_scale, pos, rope_cos, rope_sin)
+    n, head_dim = k.shape
+    fmt, rows = _key_cache_fmt(k_cache)
+    d_rope = 0 if rope_cos is None else 2 * rope_cos.shape[1]
+    max_pos = 0 if rope_cos is None else rope_cos.shape[0]
+    with torch.cuda.device(dev):
+        _check(_lib.dsa_indexer_key_append(_ptr(k), _dt(k), _ptr(rope_cos), _ptr(rope_sin), max_pos, d_rope,
+                                           _ptr(pos), _ptr(slot), n, head_dim, _ptr(k_cache), fmt, _ptr(k_scale),
+                                           rows, _stream(dev)), "dsa_indexer_key_append")
 
 
 def get_device_error(device: Optional[torch.device] = None) -> int:

@@ -190,6 +190,114 @@ size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int
     return dsa::mla_tc_workspace_bytes(rows, k, sms);
 }
 
+size_t dsa_indexer_prepare_workspace_size(int tokens, int n_heads, int d_c, int d_model) {
+    if (tokens <= 0 || n_heads <= 0 || d_c <= 0 || d_model <= 0) return 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 1024;  // no device: size for a large GPU (the most splits)
+    return dsa::indexer_prepare_workspace_bytes(tokens, n_heads, d_c, d_model, sms);
+}
+
+namespace {
+
+// Checks shared by the two key-cache writers.
+dsa_status_t check_key_cache(const char* name, const float* rope_cos, const float* rope_sin, int max_pos, int d_rope,
+                             const int32_t* pos, const int64_t* slot, int head_dim, const void* k_cache,
+                             dsa_dtype_t k_dtype, const float* k_scale, int64_t cache_rows) {
+    if (head_dim != 128) return fail(DSA_ERR_UNSUPPORTED, "%s: head_dim must be 128", name);
+    if (d_rope < 0 || d_rope > head_dim || (d_rope & 1))
+        return fail(DSA_ERR_INVALID_ARG, "%s: d_rope must be even and in [0, head_dim]", name);
+    if (d_rope > 0 && (!rope_cos || !rope_sin || !pos || max_pos < 1))
+        return fail(DSA_ERR_INVALID_ARG, "%s: rotary tables, positions and max_pos >= 1 needed when d_rope > 0", name);
+    if (!slot || !k_cache || cache_rows < 0) return fail(DSA_ERR_INVALID_ARG, "%s: null slot or cache pointer", name);
+    if (k_dtype != DSA_BF16 && k_dtype != DSA_FP8_E4M3 && k_dtype != DSA_FP4_E2M1)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: the key cache must be bf16, fp8 or fp4", name);
+    if ((k_dtype != DSA_BF16) != (k_scale != nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "%s: k_scale must be given exactly when the cache is fp8 or fp4", name);
+    if (!aligned(k_cache, 16)) return fail(DSA_ERR_INVALID_ARG, "%s: k_cache must be 16-byte aligned", name);
+    return DSA_OK;
+}
+
+}  // namespace
+
+dsa_status_t dsa_indexer_prepare(const void* c_q, const float* q_norm_weight, float eps, const void* wq_b,
+                                 const void* h, const void* wk, const void* w_proj, const float* rope_cos,
+                                 const float* rope_sin, int max_pos, int d_rope, const int32_t* pos,
+                                 const int64_t* slot, int tokens, int d_c, int d_model, int n_heads, int head_dim,
+                                 void* q_out, float* w_out, void* k_cache, dsa_dtype_t k_dtype, float* k_scale,
+                                 int64_t cache_rows, void* workspace, size_t workspace_bytes, void* stream) {
+    const char* name = "dsa_indexer_prepare";
+    if (tokens < 0 || d_c <= 0 || d_model <= 0 || n_heads <= 0 || head_dim <= 0)
+        return fail(DSA_ERR_INVALID_ARG, "%s: bad sizes", name);
+    if (tokens == 0) return DSA_OK;
+    if (!c_q || !q_norm_weight || !wq_b || !h || !wk || !w_proj || !pos || !q_out || !w_out)
+        return fail(DSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (!(eps >= 0.f)) return fail(DSA_ERR_INVALID_ARG, "%s: eps must be >= 0", name);
+    dsa_status_t st = check_key_cache(name, rope_cos, rope_sin, max_pos, d_rope, pos, slot, head_dim, k_cache,
+                                      k_dtype, k_scale, cache_rows);
+    if (st != DSA_OK) return st;
+    if (d_c % 64 || d_model % 64) return fail(DSA_ERR_UNSUPPORTED, "%s: d_c and d_model must be multiples of 64", name);
+    if (d_c > dsa::indexer_prepare_max_dc())
+        return fail(DSA_ERR_UNSUPPORTED, "%s: d_c above %d", name, dsa::indexer_prepare_max_dc());
+    if (n_heads > 256) return fail(DSA_ERR_UNSUPPORTED, "%s: n_heads > 256", name);
+    if (!aligned(c_q, 16) || !aligned(h, 16) || !aligned(wq_b, 16) || !aligned(wk, 16) || !aligned(w_proj, 16) ||
+        !aligned(q_norm_weight, 16) || !aligned(q_out, 16))
+        return fail(DSA_ERR_INVALID_ARG, "%s: c_q, h, the weights, q_norm_weight and q_out must be 16-byte aligned", name);
+    dsa::Launch L;
+    st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    const size_t need = dsa::indexer_prepare_workspace_bytes(tokens, n_heads, d_c, d_model, L.num_sms);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(DSA_ERR_INVALID_ARG, "%s: a 256-byte aligned workspace of %zu bytes is needed", name, need);
+    dsa::PrepareArgs a;
+    a.c_q = c_q;
+    a.gamma = q_norm_weight;
+    a.eps = eps;
+    a.wq_b = wq_b;
+    a.h = h;
+    a.wk = wk;
+    a.w_proj = w_proj;
+    a.rope_cos = rope_cos;
+    a.rope_sin = rope_sin;
+    a.max_pos = max_pos;
+    a.d_rope = d_rope;
+    a.pos = pos;
+    a.slot = slot;
+    a.T = tokens;
+    a.d_c = d_c;
+    a.d_model = d_model;
+    a.n_heads = n_heads;
+    a.q_out = q_out;
+    a.w_out = w_out;
+    a.k_cache = k_cache;
+    a.k_fmt = k_dtype;
+    a.k_scale = k_scale;
+    a.cache_rows = cache_rows;
+    return cuda_status(dsa::launch_indexer_prepare(L, a, workspace, workspace_bytes), "dsa_indexer_prepare launch");
+}
+
+dsa_status_t dsa_indexer_key_append(const void* k, dsa_dtype_t k_in_dtype, const float* rope_cos,
+                                    const float* rope_sin, int max_pos, int d_rope, const int32_t* pos,
+                                    const int64_t* slot, int n, int head_dim, void* k_cache, dsa_dtype_t k_dtype,
+                                    float* k_scale, int64_t cache_rows, void* stream) {
+    const char* name = "dsa_indexer_key_append";
+    if (n < 0 || head_dim <= 0) return fail(DSA_ERR_INVALID_ARG, "%s: bad sizes", name);
+    if (n == 0) return DSA_OK;
+    if (!k) return fail(DSA_ERR_INVALID_ARG, "%s: null pointer", name);
+    if (k_in_dtype != DSA_FP32 && k_in_dtype != DSA_BF16)
+        return fail(DSA_ERR_UNSUPPORTED, "%s: keys must be fp32 or bf16", name);
+    dsa_status_t st = check_key_cache(name, rope_cos, rope_sin, max_pos, d_rope, pos, slot, head_dim, k_cache,
+                                      k_dtype, k_scale, cache_rows);
+    if (st != DSA_OK) return st;
+    if (!aligned(k, 16)) return fail(DSA_ERR_INVALID_ARG, "%s: k must be 16-byte aligned", name);
+    dsa::Launch L;
+    st = make_launch(stream, &L);
+    if (st != DSA_OK) return st;
+    return cuda_status(dsa::launch_key_append(L, k, k_in_dtype, n, pos, slot, rope_cos, rope_sin, max_pos, d_rope,
+                                              k_cache, k_dtype, k_scale, cache_rows),
+                       "dsa_indexer_key_append launch");
+}
+
 }  // extern "C"
 
 namespace {

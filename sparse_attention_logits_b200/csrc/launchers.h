@@ -50,4 +50,33 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
                           int ctx_len, float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
                           const KvExtra& x = KvExtra());
 
+// Preparation of the indexer's inputs (validated arguments of
+// dsa_indexer_prepare).
+struct PrepareArgs {
+    const void* c_q;          // [T, d_c] bf16
+    const float* gamma;       // [d_c]
+    float eps;
+    const void* wq_b;         // [n_heads * 128, d_c] bf16
+    const void* h;            // [T, d_model] bf16
+    const void* wk;           // [128, d_model] bf16
+    const void* w_proj;       // [n_heads, d_model] bf16
+    const float* rope_cos;    // [max_pos, d_rope / 2]
+    const float* rope_sin;
+    int max_pos, d_rope;
+    const int32_t* pos;       // [T]
+    const int64_t* slot;      // [T]
+    int T, d_c, d_model, n_heads;
+    void* q_out;              // [T, n_heads, 128] bf16
+    float* w_out;             // [T, n_heads]
+    void* k_cache;
+    dsa_dtype_t k_fmt;
+    float* k_scale;
+    int64_t cache_rows;
+};
+size_t indexer_prepare_workspace_bytes(int T, int n_heads, int d_c, int d_model, int num_sms);
+int indexer_prepare_max_dc();
+cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* workspace, size_t ws_bytes);
+cudaError_t launch_key_append(const Launch& L, const void* k, dsa_dtype_t k_in, int n, const int32_t* pos,
+                              const int64_t* slot, const float* rope_cos, const float* rope_sin, int max_pos,
+                              int d_rope, void* cache, dsa_dtype_t fmt, float* k_scale, int64_t cache_rows);
 }  // namespace dsa

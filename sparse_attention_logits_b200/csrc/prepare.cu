@@ -1,0 +1,568 @@
+// Preparation of the lightning indexer's inputs and the write of new keys
+// into its key cache ("DeepSeek-V3.2稀疏注意力机制原理与TPU适配", section 3,
+// Step 1: the query latent is RMS-normalised and projected up, split into a
+// part with and a part without rotary position encoding, the former turned by
+// apply_rotary_emb, and weights_proj gives the per-head weights; section 1.3:
+// a separate learned linear map takes queries and keys to 128 dims):
+//
+//   q_I[t, j, :] = RoPE( W_qb[j] . RMSNorm(c_q[t]) )        [T, H, 128] bf16
+//   w[t, :]      = W_w . h[t]                               [T, H]      fp32
+//   k_I[t, :]    = RoPE( W_k . h[t] )  -> key cache row slot[t] (bf16, or
+//                  fp8 e4m3 / fp4 e2m1 codes with one fp32 scale per row)
+//
+// indexer_prepare_kernel -- all three projections in one launch on the
+// tcgen05 tensor cores.  Every CTA computes one 128-token x 64-feature tile
+// D = A . B^T (M = 128 tokens, N = 64 features, K streamed 64 at a time
+// through a 4-stage TMA ring, fp32 accumulator in TMEM):
+//   query tiles  A = c_q, B = 64 rows of W_qb.  While a stage is in shared
+//                memory the four epilogue warps add up each token's squares
+//                (the RMS) and multiply the stage by the norm gain in place;
+//                1/RMS is a per-token factor applied in the epilogue, which
+//                also turns the rotary pairs and stores bf16 q_I.
+//   key/weight tiles  A = h, B = 64 rows of [W_k ; W_w], with K split over S
+//                CTAs when the token count is small (so that the long
+//                d_model reduction is spread over as many SMs as the query
+//                tiles use).  Each writes its fp32 partial tile to the
+//                workspace.
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and
+// TMEM owner), warps 4-7 norm pass and epilogue (warp 4+q owns TMEM lanes
+// 32q .. 32q+31 = tokens of the tile).  The norm gain is copied to shared
+// memory once per CTA.
+//
+// prepare_finish_kernel -- launched right after (programmatic dependent
+// launch), one warp per token: adds the S partials in split order (the
+// result does not depend on scheduling), writes the head weights, turns the
+// key's rotary pairs and writes the key row into the cache.
+//
+// key_append_kernel -- the key-cache write alone for keys that are already
+// projected (for instance compressed CSA keys): one warp per key row, lane l
+// holding dims 4l .. 4l+3.
+//
+// The cache write is decided in binary32 with every operation rounded on
+// its own (no fused multiply-add): rotary pairs (a c - b s, a s + b c), scale
+// = amax / 448 (fp8) or amax / 6 (fp4), 1 for an all-zero row, code = the
+// nearest code of x / scale (ties to even, saturating), by the hardware
+// conversion instructions.
+#include "common.cuh"
+#include "launchers.h"
+#include "sm100.cuh"
+#include "tensor_map.h"
+
+namespace dsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int PT = 128;                         // tokens per tile (MMA M)
+constexpr int PN = 64;                          // features per tile (MMA N)
+constexpr int PK = 64;                          // reduction elements per stage (one 128-byte row)
+constexpr int PSTAGES = 4;
+constexpr int A_BYTES = PT * PK * 2;            // 16 KB
+constexpr int B_BYTES = PN * PK * 2;            // 8 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int PTHREADS = 256;
+constexpr int KDIM = 128;                       // indexer head dim (key row length)
+constexpr size_t BAR_OFF = (size_t)PSTAGES * STAGE_BYTES;                   // barriers, TMEM address, abort flag
+constexpr size_t GAIN_OFF = (BAR_OFF + (3 * PSTAGES + 1) * 8 + 16 + 15) & ~(size_t)15;
+constexpr size_t PREP_SMEM_BASE = 1024 + GAIN_OFF;                            // + d_c floats of gain
+constexpr int MAX_DC = 16384;                   // the gain (d_c floats) is held in shared memory
+
+struct KeyOut {
+    void* cache;          // [cache_rows, 128] bf16 / [cache_rows, 128] e4m3 / [cache_rows, 64] e2m1 pairs
+    float* scale;         // [cache_rows] (fp8 / fp4)
+    const float* cos;     // [max_pos, d_rope / 2]
+    const float* sin;
+    int64_t cache_rows;
+    int d_rope, max_pos, fmt;   // fmt: DSA_BF16, DSA_FP8_E4M3 or DSA_FP4_E2M1
+};
+
+struct PrepParams {
+    const float* gamma;   // [d_c] norm gain
+    const int32_t* pos;   // [T]
+    const int64_t* slot;  // [T]
+    __nv_bfloat16* q_out; // [T, H, 128]
+    float* w_out;         // [T, H]
+    float* ws;            // [S][n_tt * 128][kwc] partial sums of the key / weight tiles
+    KeyOut ko;
+    float eps;
+    int T, d_c, n_heads;
+    int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    unsigned* err;
+};
+
+struct Job {
+    bool q;          // query tile (else key / weight tile)
+    int tt, f, s;    // token tile, feature tile, split
+    int c0, c1;      // reduction chunks [c0, c1)
+};
+
+// Key / weight tiles come first in the grid: they are the longer ones.
+__device__ __forceinline__ Job job_of(const PrepParams& p, int b) {
+    Job j;
+    const int kw = p.n_tt * p.n_kwf * p.S;
+    if (b < kw) {
+        j.q = false;
+        j.tt = b / (p.n_kwf * p.S);
+        const int r = b - j.tt * p.n_kwf * p.S;
+        j.f = r / p.S;
+        j.s = r - j.f * p.S;
+        j.c0 = (int)((int64_t)p.kc_kw * j.s / p.S);
+        j.c1 = (int)((int64_t)p.kc_kw * (j.s + 1) / p.S);
+    } else {
+        b -= kw;
+        j.q = true;
+        j.tt = b / p.n_qf;
+        j.f = b - j.tt * p.n_qf;
+        j.s = 0;
+        j.c0 = 0;
+        j.c1 = p.kc_q;
+    }
+    return j;
+}
+
+__device__ __forceinline__ void rope_pair(float& a, float& b, float c, float s) {
+    const float ac = __fmul_rn(a, c), bs = __fmul_rn(b, s), as = __fmul_rn(a, s), bc = __fmul_rn(b, c);
+    a = __fsub_rn(ac, bs);
+    b = __fadd_rn(as, bc);
+}
+
+// Two binary32 values -> e4m3 pair, `lo` in the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two binary32 values -> e2m1 pair, `lo` in the low nibble.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// One warp writes one key row: lane l holds dims 4l .. 4l+3 (binary32);
+// rotary pairs of dims below d_rope turned at position `ps`, then stored at
+// row `row` of the cache in its format.
+__device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, int64_t row, const KeyOut& o) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d0 = 4 * lane + 2 * e;
+        if (d0 < o.d_rope) {
+            const int64_t ti = (int64_t)ps * (o.d_rope >> 1) + (d0 >> 1);
+            rope_pair(x[2 * e], x[2 * e + 1], __ldg(o.cos + ti), __ldg(o.sin + ti));
+        }
+    }
+    if (o.fmt == DSA_BF16) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
+        uint2 u;
+        u.x = *(uint32_t*)&a;
+        u.y = *(uint32_t*)&b;
+        ((uint2*)o.cache)[row * (KDIM / 4) + lane] = u;
+        return;
+    }
+    float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const bool fp8 = o.fmt == DSA_FP8_E4M3;
+    const float sc = amax > 0.f ? __fdiv_rn(amax, fp8 ? 448.f : 6.f) : 1.f;
+    float y[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) y[e] = __fdiv_rn(x[e], sc);
+    if (fp8) {
+        const uint32_t w = f32x2_to_e4m3x2(y[0], y[1]) | (f32x2_to_e4m3x2(y[2], y[3]) << 16);
+        ((uint32_t*)o.cache)[row * (KDIM / 4) + lane] = w;
+    } else {
+        const uint32_t w = f32x2_to_e2m1x2(y[0], y[1]) | (f32x2_to_e2m1x2(y[2], y[3]) << 8);
+        ((uint16_t*)o.cache)[row * (KDIM / 4) + lane] = (uint16_t)w;
+    }
+    if (lane == 0) o.scale[row] = sc;
+}
+
+__device__ __forceinline__ void bar_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __grid_constant__ CUtensorMap tm_cq,
+                                                                      const __grid_constant__ CUtensorMap tm_h,
+                                                                      const __grid_constant__ CUtensorMap tm_wqb,
+                                                                      const __grid_constant__ CUtensorMap tm_wk,
+                                                                      const __grid_constant__ CUtensorMap tm_ww,
+                                                                      const PrepParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = (uint64_t*)(smem + BAR_OFF);                         // [PSTAGES] stage landed
+    uint64_t* conv = full + PSTAGES;                                       // [PSTAGES] query stage scaled by the gain
+    uint64_t* empty = conv + PSTAGES;                                      // [PSTAGES] stage consumed by the MMA
+    uint64_t* accfull = empty + PSTAGES;                                   // accumulator complete
+    uint32_t* tmem_slot = (uint32_t*)(accfull + 1);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    float* gain = (float*)(smem + GAIN_OFF);                              // [d_c] (query tiles)
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Job jb = job_of(p, blockIdx.x);
+    const int nch = jb.c1 - jb.c0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < PSTAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&conv[i], 4);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(accfull, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, PN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer ----
+        if (elect_one()) {
+            const CUtensorMap* am = jb.q ? &tm_cq : &tm_h;
+            const CUtensorMap* bm = jb.q ? &tm_wqb : (jb.f < 2 ? &tm_wk : &tm_ww);
+            const int brow = (jb.q || jb.f < 2 ? jb.f : jb.f - 2) * PN;
+            tma_prefetch_desc(am);
+            tma_prefetch_desc(bm);
+            int i = 0;
+            for (; i < nch; ++i) {
+                const int st = i % PSTAGES;
+                if (!mbar_wait(&empty[st], ((i / PSTAGES) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+                mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+                uint8_t* dst = smem + (size_t)st * STAGE_BYTES;
+                const int kx = (jb.c0 + i) * PK;
+                tma_load_2d(dst, am, kx, jb.tt * PT, &full[st]);
+                tma_load_2d(dst + A_BYTES, bm, kx, brow, &full[st]);
+            }
+            if (*abort_flag) {
+                for (int j = (i > PSTAGES ? i - PSTAGES : 0); j < i; ++j)
+                    mbar_wait(&full[j % PSTAGES], (j / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------- MMA issuer ----
+        if (elect_one()) {
+            constexpr uint32_t idesc = idesc_bf16_f32(PT, PN, 0, 0);
+            const uint32_t base = smem_u32(smem);
+            bool ok = true;
+            for (int i = 0; i < nch; ++i) {
+                const int st = i % PSTAGES;
+                ok = jb.q ? mbar_wait(&conv[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)
+                          : mbar_wait(&full[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a = base + (uint32_t)(st * STAGE_BYTES), b = a + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < PK / 16; ++kk)
+                    mma_ss(tmem, desc_sw128(a + kk * 32, 1024), desc_sw128(b + kk * 32, 1024), idesc,
+                           (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&empty[st]);
+            }
+            if (ok) mma_commit(accfull);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------- norm pass and epilogue ----
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;                  // token of the tile = TMEM lane
+        const int t = jb.tt * PT + r;
+        float ss = 0.f;
+        bool ok = true;
+        if (jb.q) {
+            for (int c = threadIdx.x - 128; c < p.d_c / 4; c += 128)
+                ((float4*)gain)[c] = __ldg((const float4*)p.gamma + c);
+            bar_epilogue();
+            // every stage of c_q: this token's squares, then times the gain in place
+            for (int i = 0; i < nch && ok; ++i) {
+                const int st = i % PSTAGES;
+                ok = mbar_wait(&full[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                if (!ok) break;
+                uint8_t* row = smem + (size_t)st * STAGE_BYTES + r * 128;
+                const float4* g4 = (const float4*)(gain + (jb.c0 + i) * PK);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4* ptr = (uint4*)(row + ((c ^ (r & 7)) << 4));   // 128-byte swizzle
+                    uint4 x = *ptr;
+                    const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
+                    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                    uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                        __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
+                        xs[e] = *(uint32_t*)&v;
+                    }
+                    *ptr = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv[st]);
+            }
+        }
+        ok = ok && mbar_wait(accfull, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+        if (ok) tc_fence_after();
+        const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+        if (jb.q) {
+            const int col0 = jb.f * PN, o = col0 % KDIM;
+            const int ps = t < p.T ? __ldg(p.pos + t) : 0;
+            const bool rot = o < p.ko.d_rope;
+            const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
+            if (ok && t < p.T && !pos_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
+            const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)p.d_c), p.eps)));
+            const int half = p.ko.d_rope >> 1;
+#pragma unroll 1
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+                float v[32];
+                tmem_ld32(taddr + hh * 32, v);
+                tmem_ld_wait();
+                if (t >= p.T || !pos_ok) continue;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] *= inv;
+                if (rot) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const int d = o + hh * 32 + c;                  // dim within the head
+                        if (d < p.ko.d_rope) {
+                            const int64_t ti = (int64_t)ps * half + (d >> 1);
+                            rope_pair(v[c], v[c + 1], __ldg(p.ko.cos + ti), __ldg(p.ko.sin + ti));
+                        }
+                    }
+                }
+                uint4* dst = (uint4*)(p.q_out + (int64_t)t * p.n_heads * KDIM + col0 + hh * 32);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[8 * c + 2 * e], v[8 * c + 2 * e + 1]);
+                        w[e] = *(uint32_t*)&b2;
+                    }
+                    dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        } else if (ok) {
+            // partial tile of this split -> workspace (rows past T hold zeros)
+            float4* dst = (float4*)(p.ws + ((int64_t)jb.s * p.n_tt * PT + t) * p.kwc + jb.f * PN);
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                float v[32];
+                tmem_ld32(taddr + hh * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    dst[hh * 8 + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, PN);
+    }
+}
+
+__global__ void __launch_bounds__(256) prepare_finish_kernel(const PrepParams p) {
+    pdl_wait();                     // the partials of the projection kernel are visible from here on
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= p.T) return;
+    const int64_t split_stride = (int64_t)p.n_tt * PT * p.kwc;
+    const float* src = p.ws + (int64_t)t * p.kwc;
+    float4 a = __ldcg((const float4*)src + lane);
+#pragma unroll 4
+    for (int s = 1; s < p.S; ++s) {
+        const float4 b = __ldcg((const float4*)(src + s * split_stride) + lane);
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+    }
+    for (int j = lane; j < p.n_heads; j += 32) {
+        float acc = __ldcg(src + KDIM + j);
+#pragma unroll 4
+        for (int s = 1; s < p.S; ++s) acc += __ldcg(src + s * split_stride + KDIM + j);
+        p.w_out[(int64_t)t * p.n_heads + j] = acc;
+    }
+    const int64_t sl = __ldg(p.slot + t);
+    if (sl < 0) return;                                   // token not stored
+    const int ps = __ldg(p.pos + t);
+    if (sl >= p.ko.cache_rows || (p.ko.d_rope > 0 && (ps < 0 || ps >= p.ko.max_pos))) {
+        if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
+        return;
+    }
+    float x[4] = {a.x, a.y, a.z, a.w};
+    store_key_row(x, lane, ps, sl, p.ko);
+}
+
+__global__ void __launch_bounds__(256) key_append_kernel(const void* k, int k_fp32, int n, const int32_t* pos,
+                                                         const int64_t* slot, const KeyOut o, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += warps) {
+        const int64_t sl = __ldg(slot + r);
+        if (sl < 0) continue;
+        const int ps = o.d_rope > 0 ? __ldg(pos + r) : 0;
+        if (sl >= o.cache_rows || (o.d_rope > 0 && (ps < 0 || ps >= o.max_pos))) {
+            if (lane == 0) record_error(err, DEV_ERR_BAD_INDEX);
+            continue;
+        }
+        float x[4];
+        if (k_fp32) {
+            const float4 v = __ldg((const float4*)k + (int64_t)r * (KDIM / 4) + lane);
+            x[0] = v.x;
+            x[1] = v.y;
+            x[2] = v.z;
+            x[3] = v.w;
+        } else {
+            const uint2 u = __ldg((const uint2*)k + (int64_t)r * (KDIM / 4) + lane);
+            x[0] = __uint_as_float(u.x << 16);
+            x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+            x[2] = __uint_as_float(u.y << 16);
+            x[3] = __uint_as_float(u.y & 0xFFFF0000u);
+        }
+        store_key_row(x, lane, ps, sl, o);
+    }
+}
+
+// ------------------------------------------------------------------ host --
+
+namespace {
+
+struct PrepShape {
+    int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    size_t ws_bytes;
+};
+
+// Tiles and the split of the d_model reduction.  When the tiles alone fill
+// the GPU (two CTAs per SM) nothing is split; otherwise each key / weight
+// tile is split into about as many chunks as a query tile has, as far as
+// the free CTA slots allow.
+PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
+    PrepShape s;
+    s.n_tt = ceil_div(T, PT);
+    s.n_qf = n_heads * KDIM / PN;
+    s.n_kwf = KDIM / PN + ceil_div(n_heads, PN);
+    s.kc_q = d_c / PK;
+    s.kc_kw = d_model / PK;
+    s.kwc = s.n_kwf * PN;
+    const int slots = 2 * num_sms;
+    const int base = s.n_tt * (s.n_qf + s.n_kwf);
+    int S = 1;
+    if (base < slots) {
+        S = ceil_div(s.kc_kw, s.kc_q > 0 ? s.kc_q : 1);
+        const int room = (slots - s.n_tt * s.n_qf) / (s.n_tt * s.n_kwf);
+        if (S > room) S = room;
+        if (S > 16) S = 16;
+        if (S < 1) S = 1;
+    }
+    if (S > s.kc_kw) S = s.kc_kw;
+    s.S = S;
+    s.ws_bytes = (size_t)S * s.n_tt * PT * s.kwc * sizeof(float);
+    return s;
+}
+
+}  // namespace
+
+static_assert(GAIN_OFF % 16 == 0, "gain alignment");
+static_assert(PREP_SMEM_BASE + MAX_DC * sizeof(float) <= 227 * 1024, "shared memory");
+
+int indexer_prepare_max_dc() { return MAX_DC; }
+
+size_t indexer_prepare_workspace_bytes(int T, int n_heads, int d_c, int d_model, int num_sms) {
+    if (T <= 0) return 0;
+    return prep_shape(T, n_heads, d_c, d_model, num_sms).ws_bytes;
+}
+
+cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* workspace, size_t ws_bytes) {
+    if (a.T == 0) return cudaSuccess;
+    const PrepShape s = prep_shape(a.T, a.n_heads, a.d_c, a.d_model, L.num_sms);
+    if (ws_bytes < s.ws_bytes) return cudaErrorInvalidValue;
+    CUtensorMap m_cq, m_h, m_wqb, m_wk, m_ww;
+    const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    bool ok = make_map_sw128(&m_cq, BF, 2, a.c_q, a.d_c, a.T, PK, PT);
+    ok = ok && make_map_sw128(&m_h, BF, 2, a.h, a.d_model, a.T, PK, PT);
+    ok = ok && make_map_sw128(&m_wqb, BF, 2, a.wq_b, a.d_c, (uint64_t)a.n_heads * KDIM, PK, PN);
+    ok = ok && make_map_sw128(&m_wk, BF, 2, a.wk, a.d_model, KDIM, PK, PN);
+    ok = ok && make_map_sw128(&m_ww, BF, 2, a.w_proj, a.d_model, a.n_heads, PK, PN);
+    if (!ok) return cudaErrorInvalidValue;
+    PrepParams p;
+    p.gamma = a.gamma;
+    p.pos = a.pos;
+    p.slot = a.slot;
+    p.q_out = (__nv_bfloat16*)a.q_out;
+    p.w_out = a.w_out;
+    p.ws = (float*)workspace;
+    p.ko = KeyOut{a.k_cache, a.k_scale, a.rope_cos, a.rope_sin, a.cache_rows, a.d_rope, a.max_pos, (int)a.k_fmt};
+    p.eps = a.eps;
+    p.T = a.T;
+    p.d_c = a.d_c;
+    p.n_heads = a.n_heads;
+    p.n_tt = s.n_tt;
+    p.n_qf = s.n_qf;
+    p.n_kwf = s.n_kwf;
+    p.S = s.S;
+    p.kc_q = s.kc_q;
+    p.kc_kw = s.kc_kw;
+    p.kwc = s.kwc;
+    p.err = L.err;
+    const size_t smem = PREP_SMEM_BASE + (size_t)a.d_c * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(indexer_prepare_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s.n_tt * (s.n_qf + s.n_kwf * s.S));
+    cfg.blockDim = dim3(PTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, indexer_prepare_kernel, m_cq, m_h, m_wqb, m_wk, m_ww, p);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(ceil_div(a.T, 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, prepare_finish_kernel, p);
+    count_launch();
+    return e;
+}
+
+cudaError_t launch_key_append(const Launch& L, const void* k, dsa_dtype_t k_in, int n, const int32_t* pos,
+                              const int64_t* slot, const float* rope_cos, const float* rope_sin, int max_pos,
+                              int d_rope, void* cache, dsa_dtype_t fmt, float* k_scale, int64_t cache_rows) {
+    if (n == 0) return cudaSuccess;
+    const KeyOut o{cache, k_scale, rope_cos, rope_sin, cache_rows, d_rope, max_pos, (int)fmt};
+    const int warps_per_block = 8;
+    int grid = ceil_div(n, warps_per_block);
+    if (grid > 8 * L.num_sms) grid = 8 * L.num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * warps_per_block);
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1] = {pdl_attr()};
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, key_append_kernel, k, k_in == DSA_FP32 ? 1 : 0, n, pos, slot, o,
+                                             L.err);
+    count_launch();
+    return e;
+}
+
+}  // namespace dsa

@@ -117,3 +117,39 @@ def test_v4_attention_arguments_rejected_before_launch(lib):
                              None) == 2                              # no kernel for this geometry
     assert lib.hca_attention(fake, fake, 1, fake, fake, 0, 4, 8192, 128, 576, 512, 0.04, fake, fake, None, 0,
                              None) == 0                              # zero rows: nothing to do
+
+
+def test_indexer_prepare_arguments_rejected_before_launch(lib):
+    vp, ci, cf, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
+    fake = vp(0x1000)      # never dereferenced: validation fails first
+    lib.dsa_indexer_prepare.argtypes = [vp, vp, cf, vp, vp, vp, vp, vp, vp, ci, ci, vp, vp, ci, ci, ci, ci, ci, vp,
+                                        vp, vp, ci, vp, i64, vp, sz, vp]
+
+    def prep(tokens=64, d_c=1536, d_model=7168, head_dim=128, d_rope=64, tables=True, fmt=2, scale=True,
+             c_q=fake, eps=1e-6, slot=fake):
+        tab = fake if tables else None
+        return lib.dsa_indexer_prepare(c_q, fake, eps, fake, fake, fake, fake, tab, tab, 4096, d_rope, fake, slot,
+                                       tokens, d_c, d_model, 64, head_dim, fake, fake, fake, fmt,
+                                       fake if scale else None, 1 << 20, fake, 1 << 30, None)
+    assert prep(tokens=0) == 0                       # nothing to do
+    assert prep(head_dim=64) == 2                    # keys are 128-dim
+    assert prep(d_rope=63) == 1                      # odd rotary part
+    assert prep(d_rope=130) == 1                     # rotary part longer than the head
+    assert prep(tables=False) == 1                   # rotary part without tables
+    assert prep(fmt=1, scale=True) == 1              # bf16 cache with a scale array
+    assert prep(fmt=2, scale=False) == 1             # fp8 cache without one
+    assert prep(fmt=0, scale=False) == 2             # fp32 cache: no such format
+    assert prep(d_c=1000) == 2                       # reduction not a multiple of 64
+    assert prep(c_q=vp(0x1002)) == 1                 # misaligned activation
+    assert prep(eps=-1.0) == 1
+    assert prep(slot=None) == 1
+    lib.dsa_indexer_key_append.argtypes = [vp, ci, vp, vp, ci, ci, vp, vp, ci, ci, vp, ci, vp, i64, vp]
+
+    def app(k=fake, k_dt=1, n=8, head_dim=128, fmt=3, scale=True):
+        return lib.dsa_indexer_key_append(k, k_dt, None, None, 0, 0, None, fake, n, head_dim, fake, fmt,
+                                          fake if scale else None, 1 << 20, None)
+    assert app(n=0) == 0
+    assert app(k_dt=2) == 2                          # fp8 input keys
+    assert app(head_dim=64) == 2
+    assert app(k=vp(0x1004)) == 1
+    assert app(scale=False) == 1                     # fp4 cache without scales

@@ -206,3 +206,53 @@ def synthetic_scores(rows: int, ctx: int, device="cpu", seed: int = 0, ties: boo
         x = torch.where((z >= 0.05) & (z < 0.08), torch.full_like(x, -0.0), x)
         x = torch.where((z >= 0.08) & (z < 0.09), torch.full_like(x, float("-inf")), x)
     return x
+
+
+# ---- inputs of the step before the path (the indexer's own projections) -------
+#
+# Recipe (one generator, fixed draw order): the query latent c_q ~ N(0,1) and
+# the hidden states h ~ N(0,1) (bf16); stand-in weights, since no trained ones
+# exist here: the norm gain ~ U(0.5, 1.5) (fp32) and every projection
+# ~ N(0,1)/sqrt(fan_in) (bf16); positions uniform in [0, max_pos); cache slots
+# distinct random rows of the cache, each token's slot -1 (not stored) with
+# probability `skip`.  The rotary tables are the usual ones,
+# angle(p, i) = p * base^(-2i/d_rope), computed in float64 and rounded to fp32.
+
+@dataclasses.dataclass(frozen=True)
+class PrepareShape:
+    tokens: int
+    d_c: int           # query latent width
+    d_model: int       # hidden size
+    n_heads: int = 64  # indexer heads
+    head_dim: int = 128
+    d_rope: int = 64
+    max_pos: int = 4096
+    cache_rows: int = 8192
+
+
+def rope_tables(max_pos: int, d_rope: int, base: float = 10000.0):
+    """(cos, sin) fp32 [max_pos, d_rope/2]."""
+    i = torch.arange(d_rope // 2, dtype=torch.float64)
+    theta = base ** (-2.0 * i / d_rope)
+    ang = torch.arange(max_pos, dtype=torch.float64).unsqueeze(1) * theta.unsqueeze(0)
+    return torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+
+
+def make_prepare_inputs(s: PrepareShape, seed: int = 0, skip: float = 0.1) -> Dict[str, torch.Tensor]:
+    g = torch.Generator().manual_seed(seed)
+    T = s.tokens
+    out = {
+        "c_q": torch.randn(T, s.d_c, generator=g).to(torch.bfloat16),
+        "h": torch.randn(T, s.d_model, generator=g).to(torch.bfloat16),
+        "gamma": (0.5 + torch.rand(s.d_c, generator=g)).float(),
+        "wq_b": (torch.randn(s.n_heads * s.head_dim, s.d_c, generator=g) / math.sqrt(s.d_c)).to(torch.bfloat16),
+        "wk": (torch.randn(s.head_dim, s.d_model, generator=g) / math.sqrt(s.d_model)).to(torch.bfloat16),
+        "w_proj": (torch.randn(s.n_heads, s.d_model, generator=g) / math.sqrt(s.d_model)).to(torch.bfloat16),
+        "pos": torch.randint(0, s.max_pos, (T,), generator=g, dtype=torch.int32),
+    }
+    slot = torch.randperm(s.cache_rows, generator=g)[:T].to(torch.int64)
+    drop = torch.rand(T, generator=g) < skip
+    out["slot"] = torch.where(drop, torch.full_like(slot, -1), slot)
+    if s.d_rope:
+        out["rope_cos"], out["rope_sin"] = rope_tables(s.max_pos, s.d_rope)
+    return out
