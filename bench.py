@@ -445,6 +445,8 @@ def run_kernel_only(args):
     torch.cuda.set_device(device)
     import sparse_attention_logits_b200 as dsa
     import workloads
+    if args.kernel_only == "prepare":
+        return run_prepare_only(dsa, workloads, device, args)
     wl = workloads.BY_NAME[args.workload]
     inp = workloads.generate(wl, device=device, seed=0)
     step = DecodeStep(dsa, wl, inp, device)
@@ -473,6 +475,36 @@ def run_kernel_only(args):
     g = _graph(launch)
     dev_ms = time_graph(g, args.steps, device)
     print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": dev_ms, "ms_stream_launches": host_ms}))
+
+
+def run_prepare_only(dsa, workloads, device, args):
+    """dsa_indexer_prepare alone on `--prep-tokens` tokens (V3-class sizes,
+    fp8 key cache of 64K rows, about 0.1 GB on the device): for profiler
+    captures.  Prints the mean event time of one call."""
+    import torch
+    T = args.prep_tokens
+    shape = workloads.PrepareShape(T, PREP_D_C, PREP_D_MODEL, max_pos=4096, cache_rows=max(T, 65536))
+    inp = {k: v.to(device) for k, v in workloads.make_prepare_inputs(shape, seed=0, skip=0.0).items()}
+    cache = torch.zeros((shape.cache_rows, 128), dtype=torch.uint8, device=device)
+    scale = torch.ones(shape.cache_rows, dtype=torch.float32, device=device)
+    q_out = torch.empty((T, 64, 128), dtype=torch.bfloat16, device=device)
+    w_out = torch.empty((T, 64), dtype=torch.float32, device=device)
+    ws = torch.empty(max(dsa.indexer_prepare_workspace_size(T, 64, PREP_D_C, PREP_D_MODEL), 1), dtype=torch.uint8,
+                     device=device)
+
+    def launch():
+        dsa.indexer_prepare(inp["c_q"], inp["gamma"], inp["wq_b"], inp["h"], inp["wk"], inp["w_proj"], inp["pos"],
+                            inp["slot"], cache, scale, inp["rope_cos"], inp["rope_sin"], q_out=q_out, w_out=w_out,
+                            workspace=ws)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    dsa.get_device_error(device)
+    g = _graph(launch)
+    evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+    dev_ms = time_graph(g, args.steps, device, flush_read=evict)
+    print(json.dumps({"kernel": "prepare", "tokens": T, "ms": dev_ms}))
 
 
 def run_ours(args):
@@ -834,7 +866,8 @@ def main(argv=None):
     ap.add_argument("--no-prepare", dest="prepare", action="store_false")
     ap.add_argument("--no-other-decodes", dest="others", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla"], default=None,
+    ap.add_argument("--prep-tokens", type=int, default=64, help="tokens of --kernel-only prepare")
+    ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla", "prepare"], default=None,
                     help="time one kernel of the step alone (for profiler captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -13,7 +13,8 @@
 // indexer_prepare_kernel -- all three projections in one launch on the
 // tcgen05 tensor cores.  Every CTA computes one 128-token x 64-feature tile
 // D = A . B^T (M = 128 tokens, N = 64 features, K streamed 64 at a time
-// through a 4-stage TMA ring, fp32 accumulator in TMEM):
+// through a 4-stage TMA ring of one or two 64-wide chunks per stage, fp32
+// accumulator in TMEM):
 //   query tiles  A = c_q, B = 64 rows of W_qb.  While a stage is in shared
 //                memory the four epilogue warps add up each token's squares
 //                (the RMS) and multiply the stage by the norm gain in place;
@@ -57,15 +58,26 @@ namespace {
 constexpr int PT = 128;                         // tokens per tile (MMA M)
 constexpr int PN = 64;                          // features per tile (MMA N)
 constexpr int PK = 64;                          // reduction elements per stage (one 128-byte row)
-constexpr int PSTAGES = 4;
-constexpr int A_BYTES = PT * PK * 2;            // 16 KB
+constexpr int A_BYTES = PT * PK * 2;            // 16 KB (stage room; a 64-token box fills half)
 constexpr int B_BYTES = PN * PK * 2;            // 8 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int PTHREADS = 256;
 constexpr int KDIM = 128;                       // indexer head dim (key row length)
-constexpr size_t BAR_OFF = (size_t)PSTAGES * STAGE_BYTES;                   // barriers, TMEM address, abort flag
-constexpr size_t GAIN_OFF = (BAR_OFF + (3 * PSTAGES + 1) * 8 + 16 + 15) & ~(size_t)15;
-constexpr size_t PREP_SMEM_BASE = 1024 + GAIN_OFF;                            // + d_c floats of gain
+// Shared-memory layout for a ring of STG stages of NSUB reduction chunks
+// each (A boxes then B boxes): stages, barriers / TMEM address / abort flag,
+// then the norm gain (d_c floats).  When the grid fits on the SMs at one CTA
+// each (small token counts) a stage carries two chunks (256 contiguous bytes
+// of every weight row per stage, half the hand-offs) in a ring of 4; else
+// one chunk in a ring of 4 and two CTAs per SM.
+template <int STG, int NSUB>
+struct Ring {
+    static constexpr size_t SLOT = (size_t)NSUB * STAGE_BYTES;                 // one stage: NSUB A boxes, NSUB B boxes
+    static constexpr size_t BAR_OFF = (size_t)STG * SLOT;
+    static constexpr size_t GAIN_OFF = (BAR_OFF + (3 * STG + 1) * 8 + 16 + 15) & ~(size_t)15;
+    static constexpr size_t SMEM_BASE = 1024 + GAIN_OFF;
+    static_assert(GAIN_OFF % 16 == 0, "gain alignment");
+};
+constexpr size_t SMEM_LIMIT = 227 * 1024;
 constexpr int MAX_DC = 16384;                   // the gain (d_c floats) is held in shared memory
 
 struct KeyOut {
@@ -88,6 +100,7 @@ struct PrepParams {
     float eps;
     int T, d_c, n_heads;
     int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    int a_bytes;          // bytes of one A box (64 or 128 token rows)
     unsigned* err;
 };
 
@@ -185,28 +198,31 @@ __device__ __forceinline__ void bar_epilogue() { asm volatile("bar.sync 1, 128;"
 
 }  // namespace
 
+template <int STG, int NSUB>
 __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __grid_constant__ CUtensorMap tm_cq,
                                                                       const __grid_constant__ CUtensorMap tm_h,
                                                                       const __grid_constant__ CUtensorMap tm_wqb,
                                                                       const __grid_constant__ CUtensorMap tm_wk,
                                                                       const __grid_constant__ CUtensorMap tm_ww,
                                                                       const PrepParams p) {
+    using R = Ring<STG, NSUB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = (uint64_t*)(smem + BAR_OFF);                         // [PSTAGES] stage landed
-    uint64_t* conv = full + PSTAGES;                                       // [PSTAGES] query stage scaled by the gain
-    uint64_t* empty = conv + PSTAGES;                                      // [PSTAGES] stage consumed by the MMA
-    uint64_t* accfull = empty + PSTAGES;                                   // accumulator complete
+    uint64_t* full = (uint64_t*)(smem + R::BAR_OFF);                      // [STG] stage landed
+    uint64_t* conv = full + STG;                                           // [STG] query stage scaled by the gain
+    uint64_t* empty = conv + STG;                                          // [STG] stage consumed by the MMA
+    uint64_t* accfull = empty + STG;                                       // accumulator complete
     uint32_t* tmem_slot = (uint32_t*)(accfull + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-    float* gain = (float*)(smem + GAIN_OFF);                              // [d_c] (query tiles)
+    float* gain = (float*)(smem + R::GAIN_OFF);                            // [d_c] (query tiles)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Job jb = job_of(p, blockIdx.x);
-    const int nch = jb.c1 - jb.c0;
+    const int nch = jb.c1 - jb.c0;                  // reduction chunks of 64
+    const int nst = (nch + NSUB - 1) / NSUB;        // stages (the last may hold fewer chunks)
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < PSTAGES; ++i) {
+        for (int i = 0; i < STG; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&conv[i], 4);
             mbar_init(&empty[i], 1);
@@ -235,18 +251,21 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             tma_prefetch_desc(am);
             tma_prefetch_desc(bm);
             int i = 0;
-            for (; i < nch; ++i) {
-                const int st = i % PSTAGES;
-                if (!mbar_wait(&empty[st], ((i / PSTAGES) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
-                mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
-                uint8_t* dst = smem + (size_t)st * STAGE_BYTES;
-                const int kx = (jb.c0 + i) * PK;
-                tma_load_2d(dst, am, kx, jb.tt * PT, &full[st]);
-                tma_load_2d(dst + A_BYTES, bm, kx, brow, &full[st]);
+            for (; i < nst; ++i) {
+                const int st = i % STG;
+                if (!mbar_wait(&empty[st], ((i / STG) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+                const int ns = min(NSUB, nch - i * NSUB);
+                mbar_arrive_expect_tx(&full[st], (uint32_t)(ns * (p.a_bytes + B_BYTES)));
+                uint8_t* dst = smem + st * R::SLOT;
+                for (int j = 0; j < ns; ++j) {
+                    const int kx = (jb.c0 + i * NSUB + j) * PK;
+                    tma_load_2d(dst + j * A_BYTES, am, kx, jb.tt * PT, &full[st]);
+                    tma_load_2d(dst + NSUB * A_BYTES + j * B_BYTES, bm, kx, brow, &full[st]);
+                }
             }
             if (*abort_flag) {
-                for (int j = (i > PSTAGES ? i - PSTAGES : 0); j < i; ++j)
-                    mbar_wait(&full[j % PSTAGES], (j / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr);
+                for (int j = (i > STG ? i - STG : 0); j < i; ++j)
+                    mbar_wait(&full[j % STG], (j / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr);
             }
         }
     } else if (warp == 1) {
@@ -255,17 +274,21 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             constexpr uint32_t idesc = idesc_bf16_f32(PT, PN, 0, 0);
             const uint32_t base = smem_u32(smem);
             bool ok = true;
-            for (int i = 0; i < nch; ++i) {
-                const int st = i % PSTAGES;
-                ok = jb.q ? mbar_wait(&conv[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)
-                          : mbar_wait(&full[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+            for (int i = 0; i < nst; ++i) {
+                const int st = i % STG;
+                ok = jb.q ? mbar_wait(&conv[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)
+                          : mbar_wait(&full[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a = base + (uint32_t)(st * STAGE_BYTES), b = a + A_BYTES;
+                const int ns = min(NSUB, nch - i * NSUB);
+                for (int j = 0; j < ns; ++j) {
+                    const uint32_t a = base + (uint32_t)(st * R::SLOT + j * A_BYTES);
+                    const uint32_t b = base + (uint32_t)(st * R::SLOT + NSUB * A_BYTES + j * B_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < PK / 16; ++kk)
-                    mma_ss(tmem, desc_sw128(a + kk * 32, 1024), desc_sw128(b + kk * 32, 1024), idesc,
-                           (i > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < PK / 16; ++kk)
+                        mma_ss(tmem, desc_sw128(a + kk * 32, 1024), desc_sw128(b + kk * 32, 1024), idesc,
+                               (i > 0 || j > 0 || kk > 0) ? 1u : 0u);
+                }
                 mma_commit(&empty[st]);
             }
             if (ok) mma_commit(accfull);
@@ -282,28 +305,38 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                 ((float4*)gain)[c] = __ldg((const float4*)p.gamma + c);
             bar_epilogue();
             // every stage of c_q: this token's squares, then times the gain in place
-            for (int i = 0; i < nch && ok; ++i) {
-                const int st = i % PSTAGES;
-                ok = mbar_wait(&full[st], (i / PSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+            for (int i = 0; i < nst && ok; ++i) {
+                const int st = i % STG;
+                ok = mbar_wait(&full[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                 if (!ok) break;
-                uint8_t* row = smem + (size_t)st * STAGE_BYTES + r * 128;
-                const float4* g4 = (const float4*)(gain + (jb.c0 + i) * PK);
+                const int ns = min(NSUB, nch - i * NSUB);
+                for (int j = 0; j < ns; ++j) {
+                    uint8_t* row = smem + st * R::SLOT + j * A_BYTES + r * 128;
+                    const float4* g4 = (const float4*)(gain + (jb.c0 + i * NSUB + j) * PK);
+                    // the whole 128-byte row first, then the arithmetic, then the
+                    // stores: no load waits behind a store it might alias
+                    uint4 xv[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4* ptr = (uint4*)(row + ((c ^ (r & 7)) << 4));   // 128-byte swizzle
-                    uint4 x = *ptr;
-                    const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
-                    const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                    uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+                    for (int c = 0; c < 8; ++c) xv[c] = *(const uint4*)(row + ((c ^ (r & 7)) << 4));   // 128-byte swizzle
+                    float s2[2] = {0.f, 0.f};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
-                        ss = fmaf(lo, lo, ss);
-                        ss = fmaf(hi, hi, ss);
-                        __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
-                        xs[e] = *(uint32_t*)&v;
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
+                        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                        uint32_t xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
+                            s2[e & 1] = fmaf(lo, lo, s2[e & 1]);
+                            s2[e & 1] = fmaf(hi, hi, s2[e & 1]);
+                            __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
+                            xs[e] = *(uint32_t*)&v;
+                        }
+                        xv[c] = make_uint4(xs[0], xs[1], xs[2], xs[3]);
                     }
-                    *ptr = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+                    ss += s2[0] + s2[1];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) *(uint4*)(row + ((c ^ (r & 7)) << 4)) = xv[c];
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -380,6 +413,15 @@ __global__ void __launch_bounds__(256) prepare_finish_kernel(const PrepParams p)
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (t >= p.T) return;
+    // independent loads first: slot, position and this lane's rotary factors
+    const int64_t sl = __ldg(p.slot + t);
+    const int ps = __ldg(p.pos + t);
+    const bool pos_ok = p.ko.d_rope == 0 || (ps >= 0 && ps < p.ko.max_pos);
+    if (pos_ok && p.ko.d_rope > 0 && 4 * lane < p.ko.d_rope) {
+        const int64_t ti = (int64_t)ps * (p.ko.d_rope >> 1) + 2 * lane;
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.cos + ti));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.sin + ti));
+    }
     const int64_t split_stride = (int64_t)p.n_tt * PT * p.kwc;
     const float* src = p.ws + (int64_t)t * p.kwc;
     float4 a = __ldcg((const float4*)src + lane);
@@ -397,10 +439,8 @@ __global__ void __launch_bounds__(256) prepare_finish_kernel(const PrepParams p)
         for (int s = 1; s < p.S; ++s) acc += __ldcg(src + s * split_stride + KDIM + j);
         p.w_out[(int64_t)t * p.n_heads + j] = acc;
     }
-    const int64_t sl = __ldg(p.slot + t);
     if (sl < 0) return;                                   // token not stored
-    const int ps = __ldg(p.pos + t);
-    if (sl >= p.ko.cache_rows || (p.ko.d_rope > 0 && (ps < 0 || ps >= p.ko.max_pos))) {
+    if (sl >= p.ko.cache_rows || !pos_ok) {
         if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
         return;
     }
@@ -479,8 +519,7 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
 
 }  // namespace
 
-static_assert(GAIN_OFF % 16 == 0, "gain alignment");
-static_assert(PREP_SMEM_BASE + MAX_DC * sizeof(float) <= 227 * 1024, "shared memory");
+static_assert(Ring<4, 1>::SMEM_BASE + MAX_DC * sizeof(float) <= SMEM_LIMIT, "shared memory");
 
 int indexer_prepare_max_dc() { return MAX_DC; }
 
@@ -495,8 +534,9 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     if (ws_bytes < s.ws_bytes) return cudaErrorInvalidValue;
     CUtensorMap m_cq, m_h, m_wqb, m_wk, m_ww;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    bool ok = make_map_sw128(&m_cq, BF, 2, a.c_q, a.d_c, a.T, PK, PT);
-    ok = ok && make_map_sw128(&m_h, BF, 2, a.h, a.d_model, a.T, PK, PT);
+    const uint32_t a_rows = a.T <= 64 ? 64 : PT;     // rows past the box feed accumulator rows never stored
+    bool ok = make_map_sw128(&m_cq, BF, 2, a.c_q, a.d_c, a.T, PK, a_rows);
+    ok = ok && make_map_sw128(&m_h, BF, 2, a.h, a.d_model, a.T, PK, a_rows);
     ok = ok && make_map_sw128(&m_wqb, BF, 2, a.wq_b, a.d_c, (uint64_t)a.n_heads * KDIM, PK, PN);
     ok = ok && make_map_sw128(&m_wk, BF, 2, a.wk, a.d_model, KDIM, PK, PN);
     ok = ok && make_map_sw128(&m_ww, BF, 2, a.w_proj, a.d_model, a.n_heads, PK, PN);
@@ -520,20 +560,24 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     p.kc_q = s.kc_q;
     p.kc_kw = s.kc_kw;
     p.kwc = s.kwc;
+    p.a_bytes = (int)a_rows * PK * 2;
     p.err = L.err;
-    const size_t smem = PREP_SMEM_BASE + (size_t)a.d_c * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(indexer_prepare_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    const int grid = s.n_tt * (s.n_qf + s.n_kwf * s.S);
+    const size_t gain_bytes = (size_t)a.d_c * sizeof(float);
+    const bool deep = grid <= L.num_sms && Ring<4, 2>::SMEM_BASE + gain_bytes <= SMEM_LIMIT;
+    const size_t smem = (deep ? Ring<4, 2>::SMEM_BASE : Ring<4, 1>::SMEM_BASE) + gain_bytes;
+    auto kern = deep ? indexer_prepare_kernel<4, 2> : indexer_prepare_kernel<4, 1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(s.n_tt * (s.n_qf + s.n_kwf * s.S));
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(PTHREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, indexer_prepare_kernel, m_cq, m_h, m_wqb, m_wk, m_ww, p);
+    e = cudaLaunchKernelEx(&cfg, kern, m_cq, m_h, m_wqb, m_wk, m_ww, p);
     count_launch();
     if (e != cudaSuccess) return e;
     cfg.gridDim = dim3(ceil_div(a.T, 8));
