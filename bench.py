@@ -436,6 +436,18 @@ def cpu_baseline_decode(wl, inp, budget_s: float = 12.0):
     return done / t_used, done, oracle.max_threads(), t_used
 
 
+def _oracle_rows(fn, n_rows: int, budget_s: float):
+    """Call fn(r) for r = 0, 1, ... (cycling over n_rows) until budget_s of
+    CPU time is used; returns (calls/s, calls, seconds)."""
+    done, t_used = 0, 0.0
+    while t_used < budget_s:
+        t0 = time.perf_counter()
+        fn(done % n_rows)
+        t_used += time.perf_counter() - t0
+        done += 1
+    return done / t_used, done, t_used
+
+
 def run_kernel_only(args):
     """One kernel of the step, alone, on the workload's real inputs (the step
     runs once first so that top-k indices exist).  Used for profiler captures
@@ -703,6 +715,24 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
                         "algorithmic_bytes": step_bytes},
            "core_attention_bytes": attn_bytes,
            "l2": "step: pooled keys (268 MB) exceed L2, no flush; core attention alone: 256 MB read between replays"}
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        import oracle
+        win_rows = raw_kv[:, wl.raw_ctx - V4_WINDOW:].cpu()           # the window's raw rows, host copy
+        keys_h, kvc_h = k_c.cpu(), kv_c.cpu()
+        rb0 = torch.zeros(1, dtype=torch.int32)
+
+        def csa_row(r):
+            b = int(inp["row_batch"][r])
+            rp = inp["row_pos"][r:r + 1].cpu()
+            sc = oracle.index_scores(inp["q_idx"][r:r + 1].cpu(), inp["w"][r:r + 1].cpu(), keys_h[b:b + 1], rb0, rp)
+            sel = oracle.topk(sc, rp, wl.topk)
+            oracle.csa_core_attention(inp["q"][r:r + 1].cpu(), kvc_h[b:b + 1], sel, rb0, wl.softmax_scale, wl.d_v,
+                                      ctx, win_rows[b:b + 1], torch.tensor([V4_WINDOW - 1], dtype=torch.int32),
+                                      V4_WINDOW)
+        v, n, secs = _oracle_rows(csa_row, rows, 6.0)
+        csa["cpu_baseline"] = {"value": round(v, 4), "unit": "queries/s", "cores": oracle.max_threads(),
+                               "kind": "oracle", "sample": f"{n} whole query rows ({secs:.1f} s of CPU work)"}
+        del win_rows, keys_h, kvc_h
     del logits, idx, tws, k_c, kv_c
     # HCA over the 128:1 pooled cache
     kv_h = dsa.csa_compress(raw_kv, HCA_M)
@@ -726,6 +756,17 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
                         "frac": round(h_bytes / (ms_h / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                         "algorithmic_bytes": h_bytes},
            "l2": "256 MB buffer read between replays (the 38 MB pooled cache would stay in L2)"}
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        import oracle
+        kvh_h = kv_h.cpu()
+
+        def hca_row(r):
+            oracle.hca_attention(inp["q"][r:r + 1].cpu(), kvh_h[int(inp["row_batch"][r]):][:1],
+                                 torch.zeros(1, dtype=torch.int32), last[r:r + 1].cpu(), wl.softmax_scale, wl.d_v)
+        v, n, secs = _oracle_rows(hca_row, rows, 4.0)
+        hca["cpu_baseline"] = {"value": round(v, 4), "unit": "queries/s", "cores": oracle.max_threads(),
+                               "kind": "oracle", "sample": f"{n} whole query rows ({secs:.1f} s of CPU work)"}
+        del kvh_h
     del kv_h, inp, out, lse, hws, evict
     torch.cuda.empty_cache()
     return {"csa_core_attention_decode": csa, "hca_decode": hca}
@@ -756,7 +797,8 @@ def run_prepare(dsa, workloads, device, peaks, args):
             (f"indexer_prepare_prefill_T16384_dc{PREP_D_C}_d{PREP_D_MODEL}_bf16cache", 16384, "bf16", 16384, 16384)):
         shape = workloads.PrepareShape(T, PREP_D_C, PREP_D_MODEL, n_heads=H, head_dim=D, d_rope=d_rope,
                                        max_pos=max_pos, cache_rows=rows_cache)
-        inp = {k: v.to(device) for k, v in workloads.make_prepare_inputs(shape, seed=300 + rank, skip=0.0).items()}
+        host_inp = workloads.make_prepare_inputs(shape, seed=300 + rank, skip=0.0)
+        inp = {k: v.to(device) for k, v in host_inp.items()}
         if fmt == "fp8":
             cache = torch.zeros((rows_cache, D), dtype=torch.uint8, device=device)
             scale = torch.ones(rows_cache, dtype=torch.float32, device=device)
@@ -804,6 +846,21 @@ def run_prepare(dsa, workloads, device, peaks, args):
             rec["roofline"] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
                                "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
                                "algorithmic_flops": flops}
+        if T <= 128 and rank == 0 and world == 1 and args.cpu_baseline:
+            import oracle
+            pos_h = inp["pos"].cpu().numpy()
+            fmt = oracle.FP8 if scale is not None else oracle.BF16
+
+            def prep_call(_):
+                _, _, k64 = oracle.indexer_prepare(host_inp["c_q"], host_inp["gamma"], 1e-6, host_inp["wq_b"],
+                                                   host_inp["h"], host_inp["wk"], host_inp["w_proj"],
+                                                   host_inp["rope_cos"], host_inp["rope_sin"], pos_h, H, d_rope)
+                oracle.key_rows_f32(k64.astype("float32"), pos_h, host_inp["rope_cos"], host_inp["rope_sin"], 0,
+                                    fmt)
+            v, n, secs = _oracle_rows(prep_call, 1, 3.0)
+            rec["cpu_baseline"] = {"value": round(v * T, 2), "unit": "tokens/s", "cores": oracle.max_threads(),
+                                   "kind": "oracle",
+                                   "sample": f"{n} whole {T}-token calls ({secs:.1f} s of CPU work)"}
         out["decode" if T <= 128 else "prefill"] = rec
         del inp, cache, scale, q_out, w_out, ws
         torch.cuda.empty_cache()

@@ -300,6 +300,17 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         const int t = jb.tt * PT + r;
         float ss = 0.f;
         bool ok = true;
+        // query tiles: the token's position now, and its rotary factors into L1,
+        // so that the epilogue does not wait on them
+        const int col0 = jb.f * PN, o = col0 % KDIM;
+        const bool rot = jb.q && o < p.ko.d_rope;
+        const int ps = (jb.q && t < p.T) ? __ldg(p.pos + t) : 0;
+        const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
+        if (rot && pos_ok && t < p.T) {
+            const int64_t ti = (int64_t)ps * (p.ko.d_rope >> 1) + (o >> 1);
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.cos + ti));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.sin + ti));
+        }
         if (jb.q) {
             for (int c = threadIdx.x - 128; c < p.d_c / 4; c += 128)
                 ((float4*)gain)[c] = __ldg((const float4*)p.gamma + c);
@@ -347,10 +358,6 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         if (ok) tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
         if (jb.q) {
-            const int col0 = jb.f * PN, o = col0 % KDIM;
-            const int ps = t < p.T ? __ldg(p.pos + t) : 0;
-            const bool rot = o < p.ko.d_rope;
-            const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
             if (ok && t < p.T && !pos_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
             const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)p.d_c), p.eps)));
             const int half = p.ko.d_rope >> 1;

@@ -206,3 +206,21 @@ def test_chain_matches_oracle(cuda_device, wl):
     ro, rl, _ = oracle.sparse_mla(inp["q"], inp["kv"], ref_idx, inp["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
     assert np.abs(out2.float().cpu().numpy() - ro).max() <= ATOL_OUT[wl.dtype]
     assert np.abs(lse2.cpu().numpy() - rl).max() <= ATOL_LSE[wl.dtype]
+
+
+def test_index_reuse_across_layers(cuda_device):
+    # index reuse between adjacent layers (IndexShare): the second layer runs no
+    # indexer or top-k of its own and attends over its own queries and latent
+    # cache with the first layer's selection
+    wl = workloads.DECODE_32K.with_(batch=3, rows=6, ctx=3000, topk=512)
+    l1 = workloads.generate(wl, seed=21)
+    l2 = workloads.generate(wl, seed=22)
+    d1, d2 = _cuda(l1, cuda_device), _cuda(l2, cuda_device)
+    _, _, idx = dsa.dsa_step(d1["q_idx"], d1["w"], d1["k_idx"], d1["row_batch"], d1["row_pos"], d1["q"], d1["kv"],
+                             wl.topk, wl.softmax_scale, wl.d_v)
+    out2, lse2 = dsa.sparse_mla(d2["q"], d2["kv"], idx, d2["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
+    dsa.get_device_error()
+    gidx = idx.cpu().numpy()
+    ro, rl, _ = oracle.sparse_mla(l2["q"], l2["kv"], gidx, l2["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
+    assert np.abs(out2.float().cpu().numpy() - ro).max() <= ATOL_OUT[wl.dtype]
+    assert np.abs(lse2.cpu().numpy() - rl).max() <= ATOL_LSE[wl.dtype]
