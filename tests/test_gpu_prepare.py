@@ -157,33 +157,40 @@ def _run_prepare(shape: workloads.PrepareShape, fmt: str, seed: int):
     q_g, w_g = dsa.indexer_prepare(d["c_q"], d["gamma"], d["wq_b"], d["h"], d["wk"], d["w_proj"], d["pos"],
                                    d["slot"], cache, scale, d.get("rope_cos"), d.get("rope_sin"), eps=1e-6)
     assert dsa.get_device_error() == 0
+    _verify(inp, q_g.cpu(), w_g.cpu(), cache, scale, shape, fmt)
+    _check_untouched(cache, scale, inp["slot"].numpy(), fmt, shape.cache_rows)
+
+
+def _verify(inp, q_g, w_g, cache, scale, shape, fmt):
+    """GPU outputs of the tokens in `inp` (host inputs of those tokens only:
+    c_q, h, pos, slot; the weights whole) against the oracle."""
     q_o, w_o, k_o = _prepare_oracle(inp, shape)
-    T, H = shape.tokens, shape.n_heads
+    T, H = inp["c_q"].shape[0], shape.n_heads
 
     # queries
     cn = oracle.rms_norm(inp["c_q"].double().numpy(), inp["gamma"].numpy(), 1e-6)
     W = inp["wq_b"].double().numpy()
     sq = np.sqrt((cn ** 2) @ (W ** 2).T).reshape(T, H, 128)
     tol_q = 2.0 ** -7 * np.abs(q_o) + 2.0 ** -6 * _pair_sum(sq, shape.d_rope) + 1e-6
-    err_q = np.abs(q_g.double().cpu().numpy() - q_o)
+    err_q = np.abs(q_g.double().numpy() - q_o)
     assert (err_q <= tol_q).all(), f"q: worst excess {float((err_q - tol_q).max())}"
 
     # head weights
     hd = np.abs(inp["h"].double().numpy())
     aw = hd @ np.abs(inp["w_proj"].double().numpy()).T
-    np.testing.assert_array_less(np.abs(w_g.double().cpu().numpy() - w_o), 1e-5 * aw + 1e-6)
+    np.testing.assert_array_less(np.abs(w_g.double().numpy() - w_o), 1e-5 * aw + 1e-6)
 
     # keys in the cache
     s = inp["slot"].numpy()
     ok = s >= 0
     ak = _pair_sum(hd @ np.abs(inp["wk"].double().numpy()).T, shape.d_rope)
     if fmt == "bf16":
-        kg = cache.double().cpu().numpy()[s[ok]]
+        kg = cache[torch.from_numpy(s[ok]).to(cache.device)].double().cpu().numpy()
         tol_k = 1.01 * 2.0 ** -8 * np.abs(k_o[ok]) + 1e-5 * ak[ok] + 1e-6
         assert (np.abs(kg - k_o[ok]) <= tol_k).all()
     else:
-        _check_codes(cache.cpu().numpy()[s[ok]], scale.cpu().numpy()[s[ok]], k_o[ok], fmt, ak[ok])
-    _check_untouched(cache, scale, s, fmt, shape.cache_rows)
+        _check_codes(cache[torch.from_numpy(s[ok]).to(cache.device)].cpu().numpy(),
+                     scale[torch.from_numpy(s[ok]).to(scale.device)].cpu().numpy(), k_o[ok], fmt, ak[ok])
 
 
 @pytest.mark.parametrize("tokens", [1, 64, 200])
@@ -228,3 +235,41 @@ def test_prepare_then_indexer_scores_the_new_keys():
                               k_scale=scale.view(64, 256).cpu())
     want = ref[t.numpy(), inp["pos"].numpy()]
     np.testing.assert_allclose(got.double().numpy(), want, rtol=2e-3, atol=2e-3)
+
+
+@pytest.mark.parametrize("case", ["decode", "prefill"])
+def test_prepare_full_size_sampled(case):
+    # the launch configurations bench.py times: 64 decode tokens appending into the
+    # 64 x 131072-row fp8 key cache, and 16384 prefill tokens into a bf16 cache;
+    # every output of the sampled tokens is checked (the oracle treats tokens
+    # one by one, so it runs on the sample only)
+    dev = torch.device("cuda:0")
+    if case == "decode":
+        T, fmt, rows, max_pos = 64, "fp8", 64 * 131072, 131072
+        sample = np.array([0, 1, 31, 62, 63])
+    else:
+        T, fmt, rows, max_pos = 16384, "bf16", 16384, 16384
+        sample = np.array([0, 1, 127, 128, 4095, 8191, 12345, 16383])
+    shape = workloads.PrepareShape(T, 1536, 7168, max_pos=max_pos, cache_rows=rows)
+    inp = workloads.make_prepare_inputs(shape, seed=77, skip=0.0)
+    if case == "decode":
+        inp["pos"] = torch.full((T,), max_pos - 1, dtype=torch.int32)
+        inp["slot"] = torch.arange(T, dtype=torch.int64) * 131072 + (max_pos - 1)
+    else:
+        inp["pos"] = torch.arange(T, dtype=torch.int32)
+        inp["slot"] = torch.arange(T, dtype=torch.int64)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    if fmt == "fp8":
+        cache = torch.zeros((rows, 128), dtype=torch.uint8, device=dev)
+        scale = torch.ones(rows, dtype=torch.float32, device=dev)
+    else:
+        cache = torch.zeros((rows, 128), dtype=torch.bfloat16, device=dev)
+        scale = None
+    q_g, w_g = dsa.indexer_prepare(d["c_q"], d["gamma"], d["wq_b"], d["h"], d["wk"], d["w_proj"], d["pos"],
+                                   d["slot"], cache, scale, d["rope_cos"], d["rope_sin"], eps=1e-6)
+    assert dsa.get_device_error() == 0
+    sub = dict(inp)
+    for k in ("c_q", "h", "pos", "slot"):
+        sub[k] = inp[k][torch.from_numpy(sample)]
+    ts = torch.from_numpy(sample).to(dev)
+    _verify(sub, q_g[ts].cpu(), w_g[ts].cpu(), cache, scale, shape, fmt)
