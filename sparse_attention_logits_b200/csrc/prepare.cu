@@ -11,8 +11,9 @@
 //                  fp8 e4m3 / fp4 e2m1 codes with one fp32 scale per row)
 //
 // indexer_prepare_kernel -- all three projections in one launch on the
-// tcgen05 tensor cores.  Every CTA computes one 128-token x 64-feature tile
-// D = A . B^T (M = 128 tokens, N = 64 features, K streamed 64 at a time
+// tcgen05 tensor cores.  Every CTA computes one tile of 128 tokens x 64
+// features (256 for query tiles when there are many tokens)
+// D = A . B^T (M = 128 tokens, N = 64 or 256 features, K streamed 64 at a time
 // through a 4-stage TMA ring of one or two 64-wide chunks per stage, fp32
 // accumulator in TMEM):
 //   query tiles  A = c_q, B = 64 rows of W_qb.  While a stage is in shared
@@ -56,22 +57,23 @@ using namespace sm100;
 namespace {
 
 constexpr int PT = 128;                         // tokens per tile (MMA M)
-constexpr int PN = 64;                          // features per tile (MMA N)
+constexpr int PN = 64;                          // features per key / weight tile, and per query tile for few tokens
 constexpr int PK = 64;                          // reduction elements per stage (one 128-byte row)
 constexpr int A_BYTES = PT * PK * 2;            // 16 KB (stage room; a 64-token box fills half)
-constexpr int B_BYTES = PN * PK * 2;            // 8 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int PTHREADS = 256;
 constexpr int KDIM = 128;                       // indexer head dim (key row length)
 // Shared-memory layout for a ring of STG stages of NSUB reduction chunks
 // each (A boxes then B boxes): stages, barriers / TMEM address / abort flag,
-// then the norm gain (d_c floats).  When the grid fits on the SMs at one CTA
-// each (small token counts) a stage carries two chunks (256 contiguous bytes
-// of every weight row per stage, half the hand-offs) in a ring of 4; else
-// one chunk in a ring of 4 and two CTAs per SM.
-template <int STG, int NSUB>
+// then the norm gain (d_c floats).  Three variants: few tokens (the grid fits
+// on the SMs at one CTA each): query tiles 64 wide, two chunks per stage (256
+// contiguous bytes of every weight row per stage, half the hand-offs); many
+// tokens: query tiles 256 wide, one chunk per stage (each c_q tile feeds four
+// times the features: half the bytes an SM takes in per multiply-add); in
+// between: 64-wide tiles, one chunk per stage, two CTAs per SM.
+template <int STG, int NSUB, int QN>
 struct Ring {
-    static constexpr size_t SLOT = (size_t)NSUB * STAGE_BYTES;                 // one stage: NSUB A boxes, NSUB B boxes
+    static constexpr int B_ROOM = QN * PK * 2;                                 // one B box (query tiles are QN wide)
+    static constexpr size_t SLOT = (size_t)NSUB * (A_BYTES + B_ROOM);          // one stage: NSUB A boxes, NSUB B boxes
     static constexpr size_t BAR_OFF = (size_t)STG * SLOT;
     static constexpr size_t GAIN_OFF = (BAR_OFF + (3 * STG + 1) * 8 + 16 + 15) & ~(size_t)15;
     static constexpr size_t SMEM_BASE = 1024 + GAIN_OFF;
@@ -198,14 +200,14 @@ __device__ __forceinline__ void bar_epilogue() { asm volatile("bar.sync 1, 128;"
 
 }  // namespace
 
-template <int STG, int NSUB>
+template <int STG, int NSUB, int QN>
 __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __grid_constant__ CUtensorMap tm_cq,
                                                                       const __grid_constant__ CUtensorMap tm_h,
                                                                       const __grid_constant__ CUtensorMap tm_wqb,
                                                                       const __grid_constant__ CUtensorMap tm_wk,
                                                                       const __grid_constant__ CUtensorMap tm_ww,
                                                                       const PrepParams p) {
-    using R = Ring<STG, NSUB>;
+    using R = Ring<STG, NSUB, QN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* full = (uint64_t*)(smem + R::BAR_OFF);                      // [STG] stage landed
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, PN);
+        tmem_alloc(tmem_slot, QN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -247,7 +249,8 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         if (elect_one()) {
             const CUtensorMap* am = jb.q ? &tm_cq : &tm_h;
             const CUtensorMap* bm = jb.q ? &tm_wqb : (jb.f < 2 ? &tm_wk : &tm_ww);
-            const int brow = (jb.q || jb.f < 2 ? jb.f : jb.f - 2) * PN;
+            const int brow = jb.q ? jb.f * QN : (jb.f < 2 ? jb.f : jb.f - 2) * PN;
+            const uint32_t b_bytes = (uint32_t)(jb.q ? QN : PN) * PK * 2;
             tma_prefetch_desc(am);
             tma_prefetch_desc(bm);
             int i = 0;
@@ -255,12 +258,12 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                 const int st = i % STG;
                 if (!mbar_wait(&empty[st], ((i / STG) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
                 const int ns = min(NSUB, nch - i * NSUB);
-                mbar_arrive_expect_tx(&full[st], (uint32_t)(ns * (p.a_bytes + B_BYTES)));
+                mbar_arrive_expect_tx(&full[st], (uint32_t)ns * ((uint32_t)p.a_bytes + b_bytes));
                 uint8_t* dst = smem + st * R::SLOT;
                 for (int j = 0; j < ns; ++j) {
                     const int kx = (jb.c0 + i * NSUB + j) * PK;
                     tma_load_2d(dst + j * A_BYTES, am, kx, jb.tt * PT, &full[st]);
-                    tma_load_2d(dst + NSUB * A_BYTES + j * B_BYTES, bm, kx, brow, &full[st]);
+                    tma_load_2d(dst + NSUB * A_BYTES + j * R::B_ROOM, bm, kx, brow, &full[st]);
                 }
             }
             if (*abort_flag) {
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
         if (elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(PT, PN, 0, 0);
+            const uint32_t idesc = jb.q ? idesc_bf16_f32(PT, QN, 0, 0) : idesc_bf16_f32(PT, PN, 0, 0);
             const uint32_t base = smem_u32(smem);
             bool ok = true;
             for (int i = 0; i < nst; ++i) {
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                 const int ns = min(NSUB, nch - i * NSUB);
                 for (int j = 0; j < ns; ++j) {
                     const uint32_t a = base + (uint32_t)(st * R::SLOT + j * A_BYTES);
-                    const uint32_t b = base + (uint32_t)(st * R::SLOT + NSUB * A_BYTES + j * B_BYTES);
+                    const uint32_t b = base + (uint32_t)(st * R::SLOT + NSUB * A_BYTES + j * R::B_ROOM);
 #pragma unroll
                     for (int kk = 0; kk < PK / 16; ++kk)
                         mma_ss(tmem, desc_sw128(a + kk * 32, 1024), desc_sw128(b + kk * 32, 1024), idesc,
@@ -302,7 +305,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         bool ok = true;
         // query tiles: the token's position now, and its rotary factors into L1,
         // so that the epilogue does not wait on them
-        const int col0 = jb.f * PN, o = col0 % KDIM;
+        const int col0 = jb.f * QN, o = col0 % KDIM;    // query tiles: first feature, its dim in the head
         const bool rot = jb.q && o < p.ko.d_rope;
         const int ps = (jb.q && t < p.T) ? __ldg(p.pos + t) : 0;
         const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
@@ -362,17 +365,18 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)p.d_c), p.eps)));
             const int half = p.ko.d_rope >> 1;
 #pragma unroll 1
-            for (int hh = 0; hh < 2 && ok; ++hh) {
+            for (int hh = 0; hh < QN / 32 && ok; ++hh) {
                 float v[32];
                 tmem_ld32(taddr + hh * 32, v);
                 tmem_ld_wait();
                 if (t >= p.T || !pos_ok) continue;
 #pragma unroll
                 for (int c = 0; c < 32; ++c) v[c] *= inv;
-                if (rot) {
+                const int o32 = (col0 + hh * 32) % KDIM;                // dim in the head of this block's first column
+                if (o32 < p.ko.d_rope) {
 #pragma unroll
                     for (int c = 0; c < 32; c += 2) {
-                        const int d = o + hh * 32 + c;                  // dim within the head
+                        const int d = o32 + c;                          // dim within the head
                         if (d < p.ko.d_rope) {
                             const int64_t ti = (int64_t)ps * half + (d >> 1);
                             rope_pair(v[c], v[c + 1], __ldg(p.ko.cos + ti), __ldg(p.ko.sin + ti));
@@ -410,7 +414,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, PN);
+        tmem_dealloc(tmem, QN);
     }
 }
 
@@ -492,7 +496,7 @@ __global__ void __launch_bounds__(256) key_append_kernel(const void* k, int k_fp
 namespace {
 
 struct PrepShape {
-    int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    int n_tt, qn, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
     size_t ws_bytes;
 };
 
@@ -503,7 +507,11 @@ struct PrepShape {
 PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
     PrepShape s;
     s.n_tt = ceil_div(T, PT);
-    s.n_qf = n_heads * KDIM / PN;
+    // 256-wide query tiles when they alone give at least one CTA per SM
+    const bool wide = (n_heads * KDIM) % 256 == 0 && s.n_tt * (n_heads * KDIM / 256) >= num_sms &&
+                      Ring<4, 1, 256>::SMEM_BASE + (size_t)d_c * sizeof(float) <= SMEM_LIMIT;
+    s.qn = wide ? 256 : PN;
+    s.n_qf = n_heads * KDIM / s.qn;
     s.n_kwf = KDIM / PN + ceil_div(n_heads, PN);
     s.kc_q = d_c / PK;
     s.kc_kw = d_model / PK;
@@ -526,7 +534,7 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
 
 }  // namespace
 
-static_assert(Ring<4, 1>::SMEM_BASE + MAX_DC * sizeof(float) <= SMEM_LIMIT, "shared memory");
+static_assert(Ring<4, 1, PN>::SMEM_BASE + MAX_DC * sizeof(float) <= SMEM_LIMIT, "shared memory");
 
 int indexer_prepare_max_dc() { return MAX_DC; }
 
@@ -544,7 +552,7 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     const uint32_t a_rows = a.T <= 64 ? 64 : PT;     // rows past the box feed accumulator rows never stored
     bool ok = make_map_sw128(&m_cq, BF, 2, a.c_q, a.d_c, a.T, PK, a_rows);
     ok = ok && make_map_sw128(&m_h, BF, 2, a.h, a.d_model, a.T, PK, a_rows);
-    ok = ok && make_map_sw128(&m_wqb, BF, 2, a.wq_b, a.d_c, (uint64_t)a.n_heads * KDIM, PK, PN);
+    ok = ok && make_map_sw128(&m_wqb, BF, 2, a.wq_b, a.d_c, (uint64_t)a.n_heads * KDIM, PK, (uint32_t)s.qn);
     ok = ok && make_map_sw128(&m_wk, BF, 2, a.wk, a.d_model, KDIM, PK, PN);
     ok = ok && make_map_sw128(&m_ww, BF, 2, a.w_proj, a.d_model, a.n_heads, PK, PN);
     if (!ok) return cudaErrorInvalidValue;
@@ -571,9 +579,13 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     p.err = L.err;
     const int grid = s.n_tt * (s.n_qf + s.n_kwf * s.S);
     const size_t gain_bytes = (size_t)a.d_c * sizeof(float);
-    const bool deep = grid <= L.num_sms && Ring<4, 2>::SMEM_BASE + gain_bytes <= SMEM_LIMIT;
-    const size_t smem = (deep ? Ring<4, 2>::SMEM_BASE : Ring<4, 1>::SMEM_BASE) + gain_bytes;
-    auto kern = deep ? indexer_prepare_kernel<4, 2> : indexer_prepare_kernel<4, 1>;
+    const bool deep = s.qn == PN && grid <= L.num_sms && Ring<4, 2, PN>::SMEM_BASE + gain_bytes <= SMEM_LIMIT;
+    const size_t smem = (s.qn == 256 ? Ring<4, 1, 256>::SMEM_BASE
+                         : deep      ? Ring<4, 2, PN>::SMEM_BASE
+                                     : Ring<4, 1, PN>::SMEM_BASE) + gain_bytes;
+    auto kern = s.qn == 256 ? indexer_prepare_kernel<4, 1, 256>
+              : deep        ? indexer_prepare_kernel<4, 2, PN>
+                            : indexer_prepare_kernel<4, 1, PN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};

@@ -207,9 +207,11 @@ def test_prepare_other_geometries(n_heads, d_rope):
                  seed=n_heads)
 
 
-def test_prepare_prefill_many_token_tiles():
-    # enough tiles to fill the GPU: no split of the d_model reduction
-    _run_prepare(workloads.PrepareShape(2304, 512, 1024, cache_rows=4096), "fp8", seed=5)
+@pytest.mark.parametrize("fmt", ["fp8", "bf16"])
+def test_prepare_prefill_many_token_tiles(fmt):
+    # enough tiles to fill the GPU: 256-wide query tiles, no split of the d_model
+    # reduction, a ragged last token tile (2400 = 18 * 128 + 96)
+    _run_prepare(workloads.PrepareShape(2400, 512, 1024, cache_rows=4096), fmt, seed=5)
 
 
 def test_prepare_then_indexer_scores_the_new_keys():
