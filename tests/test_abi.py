@@ -153,3 +153,26 @@ def test_indexer_prepare_arguments_rejected_before_launch(lib):
     assert app(head_dim=64) == 2
     assert app(k=vp(0x1004)) == 1
     assert app(scale=False) == 1                     # fp4 cache without scales
+
+
+def test_indexer_prepare_workspace_sizes(lib):
+    # no device here: the size is taken for a 1024-SM GPU (the most splits).
+    # 64 tokens: one token tile, the 112-chunk d_model reduction split 5 ways
+    # (about the 24 chunks of a query tile), fp32 partials of 128 key + 64
+    # weight columns for 128 token rows per split
+    lib.dsa_indexer_prepare_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_indexer_prepare_workspace_size.argtypes = [ctypes.c_int] * 4
+    assert lib.dsa_indexer_prepare_workspace_size(64, 64, 1536, 7168) == 5 * 128 * 192 * 4
+    # 16384 tokens: 256-wide query tiles fill the GPU, no split
+    assert lib.dsa_indexer_prepare_workspace_size(16384, 64, 1536, 7168) == 1 * 16384 * 192 * 4
+    assert lib.dsa_indexer_prepare_workspace_size(0, 64, 1536, 7168) == 0
+
+
+def test_key_cache_format_inference():
+    torch = pytest.importorskip("torch")
+    dsa = pytest.importorskip("sparse_attention_logits_b200")
+    assert dsa._key_cache_fmt(torch.zeros(10, 128, dtype=torch.bfloat16)) == (dsa.DSA_BF16, 10)
+    assert dsa._key_cache_fmt(torch.zeros(2, 5, 128, dtype=torch.uint8)) == (dsa.DSA_FP8_E4M3, 10)
+    assert dsa._key_cache_fmt(torch.zeros(2, 5, 64, dtype=torch.uint8)) == (dsa.DSA_FP4_E2M1, 10)
+    with pytest.raises(TypeError):
+        dsa._key_cache_fmt(torch.zeros(10, 128, dtype=torch.float32))
