@@ -249,14 +249,29 @@ def _graph(fn):
     return g
 
 
+def replay_stats(ms_list):
+    """Summary of per-replay device times (ms): the median is the headline
+    figure; mean, min, p90 and max show whether a slow replay is an outlier
+    or a steady slowdown."""
+    s = sorted(ms_list)
+    n = len(s)
+    return {"median": statistics.median(s), "mean": statistics.mean(s), "min": s[0],
+            "p90": s[min(n - 1, int(math.ceil(0.9 * n)) - 1)], "max": s[-1], "n": n}
+
+
+def stats_json(st, nd=4):
+    return {k: (round(v, nd) if k != "n" else v) for k, v in st.items()}
+
+
 def time_graph(g, steps, device, flush=None, flush_read=None):
     """Replay `g` `steps` times, each bracketed by CUDA events on the current
     stream; with `flush` (a buffer larger than L2) it is written before each
-    replay, outside the events.  Returns the mean device time of one replay
-    in ms.  Without `flush` the inputs themselves must exceed L2: a written
-    flush leaves L2 full of dirty lines whose write-back would then be
-    charged to the next replay.  `flush_read` (a buffer larger than L2) is
-    instead read before each replay, which evicts L2 without dirtying it."""
+    replay, outside the events.  Returns replay_stats() of the per-replay
+    device times in ms.  Without `flush` the inputs themselves must exceed
+    L2: a written flush leaves L2 full of dirty lines whose write-back would
+    then be charged to the next replay.  `flush_read` (a buffer larger than
+    L2) is instead read before each replay, which evicts L2 without dirtying
+    it."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(device)
@@ -272,15 +287,15 @@ def time_graph(g, steps, device, flush=None, flush_read=None):
         b.record()
     torch.cuda.synchronize(device)
     barrier(device)
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return replay_stats([a.elapsed_time(b) for a, b in evs])
 
 
 def time_steps(step, steps, warmup, device, flush=None, soak_s=0.0):
     """The step (indexer -> top-k -> sparse MLA) is captured once into a CUDA
     graph and replayed: timings are device time, free of host launch gaps.
     Per-kernel times come from graphs holding one library call each.
-    Returns (mean step ms, {kernel: mean ms}, library kernel launches in the
-    timed steps)."""
+    Returns (replay_stats of the step in ms, {kernel: median ms}, library
+    kernel launches in the timed steps)."""
     import torch
     dsa = step.dsa
     n0 = dsa.launch_count()
@@ -295,14 +310,14 @@ def time_steps(step, steps, warmup, device, flush=None, soak_s=0.0):
             for _ in range(50):
                 g_step.replay()
             torch.cuda.synchronize(device)
-    ms = time_graph(g_step, steps, device, flush)
+    st = time_graph(g_step, steps, device, flush)
     kern = {}
     for name in ("dsa_indexer_logits", "dsa_topk", "dsa_sparse_mla"):
         g = _graph(lambda n=name: step.run_one(n))
         g.replay()
-        kern[name] = time_graph(g, max(3, steps // 2), device, flush)
+        kern[name] = time_graph(g, max(3, steps // 2), device, flush)["median"]
         del g
-    return ms, kern, per_step * steps
+    return st, kern, per_step * steps
 
 
 def e2e_decode(dsa, wl, inp, step, steps, device):
@@ -485,8 +500,9 @@ def run_kernel_only(args):
     dsa.get_device_error(device)
     host_ms = a.elapsed_time(b) / args.steps
     g = _graph(launch)
-    dev_ms = time_graph(g, args.steps, device)
-    print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": dev_ms, "ms_stream_launches": host_ms}))
+    dev = time_graph(g, args.steps, device)
+    print(json.dumps({"kernel": args.kernel_only, "workload": wl.name, "ms": dev["median"],
+                      "ms_stats": stats_json(dev), "ms_stream_launches": host_ms}))
 
 
 def run_prepare_only(dsa, workloads, device, args):
@@ -515,8 +531,8 @@ def run_prepare_only(dsa, workloads, device, args):
     dsa.get_device_error(device)
     g = _graph(launch)
     evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
-    dev_ms = time_graph(g, args.steps, device, flush_read=evict)
-    print(json.dumps({"kernel": "prepare", "tokens": T, "ms": dev_ms}))
+    dev = time_graph(g, args.steps, device, flush_read=evict)
+    print(json.dumps({"kernel": "prepare", "tokens": T, "ms": dev["median"], "ms_stats": stats_json(dev)}))
 
 
 def run_ours(args):
@@ -534,9 +550,9 @@ def run_ours(args):
     peaks = measured_peaks()
 
     with ClockSampler(device.index if "CUDA_VISIBLE_DEVICES" not in os.environ else local) as clk:
-        ms, kern, launches = time_steps(step, args.steps, args.warmup, device, soak_s=1.5)
+        st, kern, launches = time_steps(step, args.steps, args.warmup, device, soak_s=1.5)
     dsa.get_device_error(device)
-    ms_max = max_over_ranks(ms, device)
+    ms_max = max_over_ranks(st["median"], device)
     value = wl.rows * world / (ms_max / 1e3)
 
     ib = indexer_bytes(wl)
@@ -552,11 +568,13 @@ def run_ours(args):
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "ms_stats": stats_json(st),
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "topk": wl.topk,
                    "indexer": f"{wl.idx_heads}x{wl.idx_dim}", "mla": f"{wl.heads}h {wl.d_qk}/{wl.d_v}",
-                   "parallelism": f"replicas{world}", "launch": "CUDA graph of the step (device time)",
+                   "parallelism": f"replicas{world}",
+                   "launch": "CUDA graph of the step (device time, median of the timed replays)",
                    "l2": "inputs larger than L2 (keys 268 MB, latent cache 1.2 GB); no flush between steps"},
         "roofline": roof,
         "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
@@ -567,6 +585,10 @@ def run_ours(args):
     }
     if args.prefill:
         result["prefill"] = run_prefill(dsa, workloads, device, peaks, args)
+    if args.tiny:
+        result["tiny_prefill"] = run_tiny(dsa, workloads, device, peaks, args)
+    if args.compress:
+        result["csa_compress"] = run_compress(dsa, workloads, device, peaks, args)
     if args.others:
         result["other_decodes"] = run_other_decodes(dsa, workloads, device, peaks, args)
     if args.v4:
@@ -590,22 +612,64 @@ def run_prefill(dsa, workloads, device, peaks, args):
     step = DecodeStep(dsa, wl, inp, device)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
     steps = max(2, args.steps // 4)
-    ms, kern, launches = time_steps(step, steps, max(3, args.warmup // 2), device, flush)
-    ms_max = max_over_ranks(ms, device)
+    st, kern, launches = time_steps(step, steps, max(3, args.warmup // 2), device, flush)
+    ms_max = max_over_ranks(st["median"], device)
     fl_i, fl_m = indexer_flops(wl), mla_flops(wl)
     pk = peaks["bf16_tflops"]
     mla_t = fl_m / (kern["dsa_sparse_mla"] / 1e3) / 1e12
     idx_t = fl_i / (kern["dsa_indexer_logits"] / 1e3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        cpu = cpu_baseline_prefill(wl, inp)
     del inp, step, flush
     torch.cuda.empty_cache()
-    return {"workload": wl.name, "value": round(wl.rows * world / (ms_max / 1e3), 1), "unit": "tokens/s",
-            "ms_per_step": round(ms_max, 3), "steps": steps,
+    res = {"workload": wl.name, "value": round(wl.rows * world / (ms_max / 1e3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms_max, 3), "ms_stats": stats_json(st, 3), "steps": steps,
             "kernels_ms": {k: round(v, 3) for k, v in kern.items()},
             "roofline": {"kernel": "dsa_sparse_mla", "bound": "tensor", "achieved": round(mla_t, 1), "peak": pk,
                          "unit": "TFLOP/s", "frac": round(mla_t / pk, 4), "traffic": None,
                          "algorithmic_flops": fl_m},
             "indexer_roofline": {"bound": "tensor", "achieved": round(idx_t, 1), "peak": pk, "unit": "TFLOP/s",
                                  "frac": round(idx_t / pk, 4), "algorithmic_flops": fl_i}}
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    return res
+
+
+def prefill_sample_rows(n_tokens: int, n: int = 256, seed: int = 7):
+    """Seeded sample of prefill query rows for the oracle baseline: the
+    keep-all boundary (0, k-1, k) and the last token, plus rows drawn
+    uniformly without replacement from the rest."""
+    import torch
+    fixed = [0, 2047, 2048, n_tokens - 1]
+    g = torch.Generator().manual_seed(seed)
+    rest = [int(x) for x in torch.randperm(n_tokens, generator=g) if int(x) not in fixed]
+    return sorted(fixed + rest[:n - len(fixed)])
+
+
+def cpu_baseline_prefill(wl, inp):
+    """The oracle, as it stands, on a seeded sample of 256 query rows of the
+    16K-token prefill (index scores over each row's visible prefix, top-k,
+    attention over the selected rows), in one call per stage so that its
+    OpenMP loop over rows uses every core.  Throughput is the sample's rows
+    over its time: an extrapolation to the whole prefill, labelled as such."""
+    import oracle
+    import torch
+    rows = prefill_sample_rows(wl.rows)
+    ids = torch.tensor(rows, dtype=torch.long, device=inp["q"].device)
+    # host copies of the sampled rows' queries and of the shared caches (outside the timing)
+    q_idx, w, q = inp["q_idx"][ids].cpu(), inp["w"][ids].cpu(), inp["q"][ids].cpu()
+    rb, rp = inp["row_batch"][ids].cpu(), inp["row_pos"][ids].cpu()
+    k_idx, kv = inp["k_idx"].cpu(), inp["kv"].cpu()
+    t0 = time.perf_counter()
+    scores = oracle.index_scores(q_idx, w, k_idx, rb, rp)
+    sel = oracle.topk(scores, rp, wl.topk)
+    oracle.sparse_mla(q, kv, sel, rb, wl.softmax_scale, wl.d_v, wl.ctx)
+    secs = time.perf_counter() - t0
+    return {"value": round(len(rows) / secs, 3), "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": (f"{len(rows)} seeded query rows of {wl.name} (positions 0, 2047, 2048, {wl.rows - 1} and "
+                       f"{len(rows) - 4} uniform others), {secs:.1f} s of CPU work; tokens/s extrapolated from the "
+                       f"sample's mean time per row")}
 
 
 def run_other_decodes(dsa, workloads, device, peaks, args):
@@ -623,20 +687,112 @@ def run_other_decodes(dsa, workloads, device, peaks, args):
     for wl in (workloads.CSA_DECODE_1M, workloads.DECODE_128K_FP8_PAGED, fp4):
         inp = workloads.generate(wl, device=device, seed=300 + rank)
         step = DecodeStep(dsa, wl, inp, device)
-        ms, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device, soak_s=0.5)
-        ms = max_over_ranks(ms, device)
+        st, kern, _ = time_steps(step, max(5, args.steps // 2), 3, device, soak_s=0.5)
+        ms = max_over_ranks(st["median"], device)
         b = indexer_bytes(wl) + mla_bytes(wl)
         if wl.page_size:
             b += wl.batch * (wl.ctx // wl.page_size) * 4          # the page table
         ach = b / (ms / 1e3) / 1e9
         res[wl.name] = {"value": round(wl.rows * world / (ms / 1e3), 1), "unit": "queries/s",
-                        "ms_per_step": round(ms, 4), "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+                        "ms_per_step": round(ms, 4), "ms_stats": stats_json(st),
+                        "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
                         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
                                      "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
                                      "algorithmic_bytes": b},
                         "l2": "inputs larger than L2; no flush between steps"}
         del inp, step
         torch.cuda.empty_cache()
+    return res
+
+
+def run_compress(dsa, workloads, device, peaks, args):
+    """CSA token compression (csa_compress, m = 4) of the raw caches of the
+    1M-token CSA decode: the 4 x 1,048,576 x 576 latent cache and the
+    4 x 1,048,576 x 128 indexer key cache, both bf16, pooled into 262,144
+    entries per sequence.  One graph holds the two calls; the raw caches
+    (5.9 GB) exceed L2, so nothing is flushed between replays.  Roofline:
+    every raw row read once and every pooled row written once (7.38 GB) over
+    the event time, against the measured HBM copy bandwidth."""
+    import torch
+    rank, world, _ = dist_env()
+    wl = workloads.CSA_DECODE_1M
+    inp = workloads.generate(wl, device=device, seed=400 + rank)
+    raw_k, raw_kv = inp["k_idx"], inp["kv"]
+    del inp
+    m = wl.compress_m
+    out_k = torch.empty((wl.batch, wl.ctx, wl.idx_dim), dtype=raw_k.dtype, device=device)
+    out_kv = torch.empty((wl.batch, wl.ctx, wl.d_qk), dtype=raw_kv.dtype, device=device)
+
+    def call():
+        dsa.csa_compress(raw_kv, m, out=out_kv)
+        dsa.csa_compress(raw_k, m, out=out_k)
+
+    n0 = dsa.launch_count()
+    g = _graph(call)
+    launches = (dsa.launch_count() - n0) // 2
+    for _ in range(3):
+        g.replay()
+    st = time_graph(g, max(5, args.steps // 2), device)
+    ms = max_over_ranks(st["median"], device)
+    dsa.get_device_error(device)
+    del g
+    moved = (raw_k.numel() + raw_kv.numel()) * raw_k.element_size() + \
+        (out_k.numel() + out_kv.numel()) * out_k.element_size()
+    ach = moved / (ms / 1e3) / 1e9
+    raw_tokens = wl.batch * wl.raw_ctx
+    res = {"workload": f"csa_compress_bf16_B{wl.batch}_L{wl.raw_ctx}_m{m}_d{wl.d_qk}+d{wl.idx_dim}",
+           "value": round(raw_tokens * world / (ms / 1e3), 1), "unit": "raw tokens/s",
+           "ms_per_step": round(ms, 4), "ms_stats": stats_json(st), "gpu_launches": launches,
+           "roofline": {"kernel": "csa_compress", "bound": "hbm", "achieved": round(ach, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                        "algorithmic_bytes": moved},
+           "l2": "raw caches (5.9 GB) larger than L2; no flush between replays"}
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        import oracle
+        n_raw = 65536                                # raw rows of each cache in the sample (sequence 0)
+        kv_h, k_h = raw_kv[:1, :n_raw].cpu(), raw_k[:1, :n_raw].cpu()
+
+        def pool(_):
+            oracle.csa_compress(kv_h, m)
+            oracle.csa_compress(k_h, m)
+        v, n, secs = _oracle_rows(pool, 1, 3.0)
+        res["cpu_baseline"] = {"value": round(v * n_raw, 1), "unit": "raw tokens/s", "cores": oracle.max_threads(),
+                               "kind": "oracle",
+                               "sample": f"{n} poolings of {n_raw} raw rows of both caches ({secs:.1f} s of CPU work)"}
+    del raw_k, raw_kv, out_k, out_kv
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_tiny(dsa, workloads, device, peaks, args):
+    """The tiny fp32 causal prefill (256 tokens, top-64, 4 x 32 indexer, 8 MQA
+    heads over a 64-d latent): the whole path as one graph.  It moves about
+    0.3 MB and is bound by launch and synchronisation latency, so it is
+    reported as microseconds per step; its inputs stay in L2."""
+    import oracle
+    import torch
+    rank, world, _ = dist_env()
+    wl = workloads.TINY_PREFILL_FP32
+    inp = workloads.generate(wl, device=device, seed=500 + rank)
+    step = DecodeStep(dsa, wl, inp, device)
+    st, kern, launches = time_steps(step, max(20, args.steps), 3, device)
+    us = max_over_ranks(st["median"], device) * 1e3
+    res = {"workload": wl.name, "us_per_step": round(us, 2), "value": round(wl.rows * world / (us / 1e6), 1),
+           "unit": "tokens/s", "ms_stats": stats_json(st, 5),
+           "kernels_us": {k: round(v * 1e3, 2) for k, v in kern.items()}, "gpu_launches": launches,
+           "l2": "inputs (0.3 MB) stay in L2: latency-bound"}
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        h = {k: v.cpu() for k, v in inp.items()}
+
+        def whole(_):
+            sc = oracle.index_scores(h["q_idx"], h["w"], h["k_idx"], h["row_batch"], h["row_pos"])
+            sel = oracle.topk(sc, h["row_pos"], wl.topk)
+            oracle.sparse_mla(h["q"], h["kv"], sel, h["row_batch"], wl.softmax_scale, wl.d_v, wl.ctx)
+        v, n, secs = _oracle_rows(whole, 1, 2.0)
+        res["cpu_baseline"] = {"value": round(v * wl.rows, 1), "unit": "tokens/s", "cores": oracle.max_threads(),
+                               "kind": "oracle", "sample": f"{n} whole steps ({secs:.1f} s of CPU work)"}
+    del inp, step
+    torch.cuda.empty_cache()
     return res
 
 
@@ -695,20 +851,22 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
     for _ in range(3):
         g.replay()
     steps = max(5, args.steps)
-    ms = max_over_ranks(time_graph(g, steps, device), device)
+    st_step = time_graph(g, steps, device)
+    ms = max_over_ranks(st_step["median"], device)
     del g
     # alone, the gathered rows (5 MB) would stay in L2 between replays: read
     # a 256 MB buffer before each one
     evict = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
     ga = _graph(lambda: st.run_one("csa_core_attention"))
     ga.replay()
-    ms_attn = time_graph(ga, steps, device, flush_read=evict)
+    ms_attn = time_graph(ga, steps, device, flush_read=evict)["median"]
     del ga
     sel_rows = rows * (wl.topk + V4_WINDOW)
     step_bytes = (indexer_bytes(wl) + sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2)
     attn_bytes = sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2
     csa = {"workload": f"{wl.name}+window{V4_WINDOW}", "value": round(rows * world / (ms / 1e3), 1),
-           "unit": "queries/s", "ms_per_step": round(ms, 4), "core_attention_ms": round(ms_attn, 4),
+           "unit": "queries/s", "ms_per_step": round(ms, 4), "ms_stats": stats_json(st_step),
+           "core_attention_ms": round(ms_attn, 4),
            "roofline": {"bound": "hbm", "achieved": round(step_bytes / (ms / 1e3) / 1e9, 1),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -746,11 +904,12 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
                                           out=out, lse=lse, workspace=hws))
     for _ in range(3):
         gh.replay()
-    ms_h = max_over_ranks(time_graph(gh, steps, device, flush_read=evict), device)
+    st_h = time_graph(gh, steps, device, flush_read=evict)
+    ms_h = max_over_ranks(st_h["median"], device)
     del gh
     h_bytes = rows * L_h * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2
     hca = {"workload": f"hca_decode_bf16_B4_L1048576_m{HCA_M}", "value": round(rows * world / (ms_h / 1e3), 1),
-           "unit": "queries/s", "ms_per_step": round(ms_h, 4),
+           "unit": "queries/s", "ms_per_step": round(ms_h, 4), "ms_stats": stats_json(st_h),
            "roofline": {"bound": "hbm", "achieved": round(h_bytes / (ms_h / 1e3) / 1e9, 1),
                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
                         "frac": round(h_bytes / (ms_h / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
@@ -826,7 +985,8 @@ def run_prepare(dsa, workloads, device, peaks, args):
         for _ in range(3):
             g.replay()
         steps = max(5, args.steps)
-        ms = max_over_ranks(time_graph(g, steps, device, flush_read=evict), device)
+        st = time_graph(g, steps, device, flush_read=evict)
+        ms = max_over_ranks(st["median"], device)
         del g
         dsa.get_device_error(device)
         w_bytes = (H * D * PREP_D_C + D * PREP_D_MODEL + H * PREP_D_MODEL) * 2 + PREP_D_C * 4
@@ -835,7 +995,7 @@ def run_prepare(dsa, workloads, device, peaks, args):
         hbm = w_bytes + a_bytes + o_bytes
         flops = 2 * T * (H * D * PREP_D_C + (D + H) * PREP_D_MODEL)
         rec = {"workload": name, "value": round(T * world / (ms / 1e3), 1), "unit": "tokens/s",
-               "ms_per_call": round(ms, 4), "gpu_launches": launches,
+               "ms_per_call": round(ms, 4), "ms_stats": stats_json(st), "gpu_launches": launches,
                "l2": "256 MB buffer read between replays"}
         if T <= 128:
             ach = hbm / (ms / 1e3) / 1e9
@@ -922,6 +1082,8 @@ def main(argv=None):
     ap.add_argument("--no-v4", dest="v4", action="store_false")
     ap.add_argument("--no-prepare", dest="prepare", action="store_false")
     ap.add_argument("--no-other-decodes", dest="others", action="store_false")
+    ap.add_argument("--no-compress", dest="compress", action="store_false")
+    ap.add_argument("--no-tiny", dest="tiny", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--prep-tokens", type=int, default=64, help="tokens of --kernel-only prepare")
     ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla", "prepare"], default=None,

@@ -4,6 +4,7 @@
 #include <stdio.h>
 #include <stdarg.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -30,8 +31,11 @@ dsa_status_t cuda_status(cudaError_t e, const char* what) {
 // One error word per device; its device address is looked up once per device.
 __device__ unsigned g_device_error;
 
-constexpr int kMaxDevices = 64;
-unsigned* g_err_ptr[kMaxDevices] = {};
+constexpr int kMaxDevices = dsa::kMaxDevices;
+// Filled once per device under dsa::init_mutex(): the SM count is stored
+// first and the error-word address is then published with release order, so
+// a thread that sees the address (acquire) also sees the SM count.
+std::atomic<unsigned*> g_err_ptr[kMaxDevices] = {};
 int g_num_sms[kMaxDevices] = {};
 
 dsa_status_t make_launch(void* stream, dsa::Launch* L) {
@@ -39,18 +43,24 @@ dsa_status_t make_launch(void* stream, dsa::Launch* L) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
-    if (!g_err_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_device_error);
-        if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(device error word)");
-        int sms = 0;
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return cuda_status(e, "cudaDeviceGetAttribute");
-        g_num_sms[dev] = sms;
-        g_err_ptr[dev] = (unsigned*)p;
+    unsigned* err = g_err_ptr[dev].load(std::memory_order_acquire);
+    if (!err) {
+        std::lock_guard<std::mutex> lock(dsa::init_mutex());
+        err = g_err_ptr[dev].load(std::memory_order_relaxed);
+        if (!err) {
+            void* p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_device_error);
+            if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(device error word)");
+            int sms = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return cuda_status(e, "cudaDeviceGetAttribute");
+            g_num_sms[dev] = sms;
+            err = (unsigned*)p;
+            g_err_ptr[dev].store(err, std::memory_order_release);
+        }
     }
     L->stream = (cudaStream_t)stream;
-    L->err = g_err_ptr[dev];
+    L->err = err;
     L->num_sms = g_num_sms[dev];
     return DSA_OK;
 }
@@ -97,6 +107,10 @@ bool valid_key_dtype(dsa_dtype_t t) { return valid_dtype(t) || t == DSA_FP4_E2M1
 
 namespace dsa {
 void count_launch(int n) { g_launches += (uint64_t)n; }
+std::mutex& init_mutex() {
+    static std::mutex mu;
+    return mu;
+}
 }  // namespace dsa
 
 extern "C" {
@@ -185,8 +199,10 @@ dsa_status_t dsa_topk(const float* logits, int64_t ld, const int32_t* row_pos, i
 size_t dsa_sparse_mla_workspace_size(int rows, int k, int n_heads, int d_qk, int d_v, dsa_dtype_t dtype) {
     if (rows <= 0 || k <= 0 || !dsa::mla_tc_supported(dtype, n_heads, d_qk, d_v)) return 0;
     int dev = 0, sms = 0;
+    // No device: size for a very large GPU.  The split count grows with the
+    // SM count (up to one split per 64 keys), so this bounds every device.
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        sms = 1;     // no device: size for the smallest GPU (most splits)
+        sms = 1024;
     return dsa::mla_tc_workspace_bytes(rows, k, sms);
 }
 

@@ -6,6 +6,9 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/dsa_b200.h"
 
 namespace dsa {
@@ -19,6 +22,34 @@ enum : unsigned {
     DEV_ERR_TIMEOUT_PEER = 4u,     // a wait on a partner CTA of the cluster ran out
     DEV_ERR_BAD_INDEX = 8u,        // an index outside [0, ctx_len) was met and skipped
 };
+
+constexpr int kMaxDevices = 64;
+
+// Lock held while a per-device value is computed for the first time (the
+// device error word's address, occupancy queries); later calls read the
+// published value without it.
+std::mutex& init_mutex();
+
+// Per-device integer computed on first use: 0 = not yet known.  The first
+// callers on a device run `compute` under init_mutex(); its result (or -1
+// when it gives no positive value) is then published.  Returns the cached
+// value, or 0 when there is none.
+template <class F>
+int device_cached(std::atomic<int> (&cache)[kMaxDevices], F&& compute) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    int v = cache[dev].load(std::memory_order_acquire);
+    if (v == 0) {
+        std::lock_guard<std::mutex> lock(init_mutex());
+        v = cache[dev].load(std::memory_order_relaxed);
+        if (v == 0) {
+            const int n = compute();
+            v = n > 0 ? n : -1;
+            cache[dev].store(v, std::memory_order_release);
+        }
+    }
+    return v > 0 ? v : 0;
+}
 
 struct Launch {
     cudaStream_t stream;

@@ -816,10 +816,8 @@ int choose_splits(int rows, int k, int num_sms) {
 // How many 4-CTA clusters of mla_tc_kernel can be resident at once on the
 // current device (0 if the query fails); looked up once per device.
 int max_active_quads() {
-    static int cache[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cache[dev] == 0) {
+    static std::atomic<int> cache[kMaxDevices] = {};
+    return device_cached(cache, [] {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(4);
         cfg.blockDim = dim3(THREADS);
@@ -839,9 +837,8 @@ int max_active_quads() {
             cudaGetLastError();
             n = 0;
         }
-        cache[dev] = n > 0 ? n : -1;
-    }
-    return cache[dev] > 0 ? cache[dev] : 0;
+        return n;
+    });
 }
 
 }  // namespace

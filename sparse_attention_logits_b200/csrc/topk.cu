@@ -36,6 +36,15 @@ constexpr int CAND_CAP = 1024;                 // candidates ranked directly aft
 // candidate buffer, candidates' source CTAs, per-CTA counts (rank 0)
 constexpr int MAX_CL = 16;                     // CTAs per row (16 needs the non-portable cluster size)
 constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 32 + 3 * MAX_CL + 16) * 4;
+// Alignment of the vector accesses, by construction: the base is rounded up
+// to 128 B in the kernel (the launch reserves exactly that rounding room,
+// SMEM_ROUND), the key slice starts SMEM_FIXED bytes after it, and every
+// 16-byte access of the slice is at a multiple of 4 keys (the slice length
+// `per` and every walk's start are multiples of 4); the cluster histograms
+// read with 8-byte loads start at even words of an 8-byte aligned array.
+constexpr int SMEM_ROUND = 128;
+static_assert(SMEM_FIXED % 16 == 0, "the key slice must start 16-byte aligned");
+static_assert((2 * NBINS * 4) % 8 == 0 && NBINS % 2 == 0, "cluster histograms: 8-byte aligned pairs");
 
 // Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
@@ -114,7 +123,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     extern __shared__ uint8_t tk_smem_raw[];
     // the runtime's placement of dynamic shared memory is not relied upon:
     // the base is rounded up here (the launch reserves the slack)
-    uint32_t* tk_smem = (uint32_t*)(((uintptr_t)tk_smem_raw + 127) & ~(uintptr_t)127);
+    uint32_t* tk_smem = (uint32_t*)(((uintptr_t)tk_smem_raw + SMEM_ROUND - 1) & ~(uintptr_t)(SMEM_ROUND - 1));
     uint32_t* hist = tk_smem;                    // [NBINS]   this CTA's histogram
     uint32_t* merged = hist + NBINS;             // [NBINS]   scratch for the suffix scan
     uint32_t* cl_hist = merged + NBINS;          // [MAX_PASSES][NBINS] cluster-wide histograms (rank 0 holds them)
@@ -545,11 +554,9 @@ namespace {
 // current device can hold at once (0 if none or the query fails); looked up
 // once per device.
 int max_active_16() {
-    static int cache[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cache[dev] == 0) {
-        const size_t smem = 128 + SMEM_FIXED + (size_t)16384 * 4;
+    static std::atomic<int> cache[kMaxDevices] = {};
+    return device_cached(cache, [] {
+        const size_t smem = SMEM_ROUND + SMEM_FIXED + (size_t)16384 * 4;
         int n = 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(16);
@@ -570,9 +577,8 @@ int max_active_16() {
             cudaGetLastError();
             n = 0;
         }
-        cache[dev] = n > 0 ? n : -1;
-    }
-    return cache[dev] > 0 ? cache[dev] : 0;
+        return n;
+    });
 }
 
 int choose_cluster(int rows, int ctx_len, int num_sms) {
@@ -590,7 +596,7 @@ template <int CL>
 cudaError_t launch_cl(const Launch& L, const float* logits, int64_t ld, const int32_t* row_pos, int rows, int ctx_len,
                       int k, int32_t* idx) {
     const int per = ((ctx_len + CL - 1) / CL + 3) & ~3;
-    const size_t smem = 128 + SMEM_FIXED + (size_t)per * 4;
+    const size_t smem = SMEM_ROUND + SMEM_FIXED + (size_t)per * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel<CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (CL > 8) {

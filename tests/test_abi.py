@@ -176,3 +176,24 @@ def test_key_cache_format_inference():
     assert dsa._key_cache_fmt(torch.zeros(2, 5, 64, dtype=torch.uint8)) == (dsa.DSA_FP4_E2M1, 10)
     with pytest.raises(TypeError):
         dsa._key_cache_fmt(torch.zeros(10, 128, dtype=torch.float32))
+
+
+def test_sparse_mla_workspace_size_without_device_bounds_every_gpu(lib):
+    # No device here: the size is taken for a 1024-SM GPU.  The split count
+    # grows with the SM count (up to one split per 64 selected keys), so this
+    # must be at least what a 148-SM B200 asks for.  A (row, split) pair holds
+    # a bf16 partial of 128 heads x 512 dims and an fp32 lse per head.
+    lib.dsa_sparse_mla_workspace_size.restype = ctypes.c_size_t
+    lib.dsa_sparse_mla_workspace_size.argtypes = [ctypes.c_int] * 6
+    pair = 128 * (512 * 2 + 4)
+
+    def b200_size(rows, k):                       # the split rule on 148 SMs (74 CTA pairs)
+        s = 1 if rows >= 74 else 74 // rows
+        s = max(1, min(s, (k + 63) // 64))
+        return 0 if s == 1 else rows * s * pair
+
+    for rows, k in ((2, 2048), (4, 1152), (32, 2048), (64, 2048), (1, 64)):
+        got = lib.dsa_sparse_mla_workspace_size(rows, k, 128, 576, 512, 1)
+        assert got >= b200_size(rows, k), (rows, k, got)
+    assert lib.dsa_sparse_mla_workspace_size(2, 2048, 128, 576, 512, 1) == 2 * 32 * pair   # one split per 64 keys
+    assert lib.dsa_sparse_mla_workspace_size(0, 2048, 128, 576, 512, 1) == 0
