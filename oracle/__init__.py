@@ -256,17 +256,23 @@ def sparse_mla(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int,
 
 
 def csa_core_attention(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int, kv_win, win_pos, window: int,
-                       page_table=None):
-    """CSA core attention with the window segment ("DeepSeek V4 发布：1.6T 参数、
-    百万上下文…", CSA: the window KV and the compressed KV are concatenated and
-    take part in core attention together).  Slots are the selected compressed
-    entries idx[t] of kv followed by the raw rows win_pos[t]-window+1 ..
-    win_pos[t] of kv_win (negative positions unused).
+                       page_table=None, n_sink: int = 0):
+    """CSA core attention with the window and attention-sink segments
+    ("DeepSeek V4 发布：1.6T 参数、百万上下文…", CSA: the window KV and the
+    compressed KV are concatenated and take part in core attention together;
+    "解密DeepSeek-V4 预览版…" section 4.3 and "打破幻觉与成本魔咒：DeepSeek-V4 …"
+    section 3.3.2: CSA keeps local dependencies with sliding-window attention
+    and an attention sink).  Slots are the selected compressed entries idx[t]
+    of kv, then the raw rows win_pos[t]-window+1 .. win_pos[t] of kv_win
+    (negative positions unused), then the sink: raw rows 0 .. n_sink-1 of the
+    sequence, each used only if it lies before the window's first position
+    (a raw row inside the window is not attended twice).
 
     Written as that concatenation: one cache [B, ctx + win_len, D] holding the
     (de-paged) compressed cache then the raw cache, and one index list holding
-    the selected entries then ctx + the window positions; attention over it is
-    sparse_mla.  Returns (out [rows,H,D_V] f64, lse [rows,H] f64)."""
+    the selected entries, then ctx + the window positions, then ctx + the
+    sink positions; attention over it is sparse_mla.  Returns
+    (out [rows,H,D_V] f64, lse [rows,H] f64)."""
     kva = torch.as_tensor(kv)
     if page_table is not None:
         pt = torch.as_tensor(page_table).long()
@@ -279,8 +285,10 @@ def csa_core_attention(q, kv, idx, row_batch, scale: float, d_v: int, ctx: int, 
     pos = torch.as_tensor(win_pos).long().view(rows, 1)
     wi = pos - window + 1 + torch.arange(window).view(1, -1)
     wi = torch.where(wi >= 0, wi + ctx, torch.full_like(wi, -1))
+    si = torch.arange(n_sink).view(1, -1).expand(rows, n_sink)
+    si = torch.where(si < pos - window + 1, si + ctx, torch.full_like(si, -1))
     parts = [] if idx is None else [torch.as_tensor(idx).long()]
-    full = torch.cat(parts + [wi], dim=1).to(torch.int32)
+    full = torch.cat(parts + [wi, si], dim=1).to(torch.int32)
     out, lse, _ = sparse_mla(q, comb, full, row_batch, scale, d_v, ctx + win.shape[1])
     return out, lse
 

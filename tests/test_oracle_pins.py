@@ -433,6 +433,43 @@ def test_csa_core_attention_is_attention_over_the_concatenated_keys():
     np.testing.assert_allclose(ow[t], ro, rtol=0, atol=1e-12)
 
 
+def test_csa_core_attention_sink_is_attention_over_the_union_of_raw_positions():
+    # The sink and the window are both raw rows: the attended raw positions
+    # are the union {0 .. n_sink-1} u {pos-W+1 .. pos}, clipped to [0, pos],
+    # each once; with the selected compressed entries beside them.
+    g = torch.Generator().manual_seed(34)
+    B, Lc, Lr, H, D, dv, k = 2, 20, 80, 3, 12, 8, 5
+    rows = 7
+    q = torch.randn(rows, H, D, generator=g)
+    kv = torch.randn(B, Lc, D, generator=g)
+    raw = torch.randn(B, Lr, D, generator=g)
+    rb = torch.tensor([0, 1, 1, 0, 1, 0, 1], dtype=torch.int32)
+    # far from the start, window touching the sink, overlapping it, inside it, at position 0
+    pos = torch.tensor([79, 9, 7, 5, 2, 0, 40], dtype=torch.int32)
+    idx = torch.stack([torch.randperm(Lc, generator=g)[:k] for _ in range(rows)]).to(torch.int32)
+    idx[3, 1] = -1
+    for W, n_sink in ((6, 4), (0, 4), (6, 0), (3, 12), (1, 1)):
+        out, lse = oracle.csa_core_attention(q, kv, idx, rb, 0.4, dv, Lc, raw, pos, W, n_sink=n_sink)
+        for t in range(rows):
+            b, p_t = int(rb[t]), int(pos[t])
+            raw_pos = sorted(set(range(min(n_sink, p_t + 1))) | set(range(max(0, p_t - W + 1), p_t + 1)))
+            sel = [kv[b, int(s)] for s in idx[t] if s >= 0]
+            vecs = torch.stack(sel + [raw[b, p] for p in raw_pos]).double().numpy()
+            ro, rl = _brute_attention(q[t].double().numpy(), vecs, 0.4, dv)
+            np.testing.assert_allclose(out[t], ro, rtol=0, atol=1e-12, err_msg=f"W={W} sink={n_sink} t={t}")
+            np.testing.assert_allclose(lse[t], rl, rtol=0, atol=1e-12)
+    # no sink: the window-only composition, unchanged
+    a, la = oracle.csa_core_attention(q, kv, idx, rb, 0.4, dv, Lc, raw, pos, 6)
+    b_, lb = oracle.csa_core_attention(q, kv, idx, rb, 0.4, dv, Lc, raw, pos, 6, n_sink=0)
+    np.testing.assert_array_equal(a, b_)
+    # sink only (no window, no selection): attention over raw rows 0 .. min(n_sink, pos+1)-1
+    so, sl = oracle.csa_core_attention(q, kv, None, rb, 0.4, dv, Lc, raw, pos, 0, n_sink=4)
+    ro, rl = _brute_attention(q[0].double().numpy(), raw[0, :4].double().numpy(), 0.4, dv)
+    np.testing.assert_allclose(so[0], ro, rtol=0, atol=1e-12)
+    ro, rl = _brute_attention(q[5].double().numpy(), raw[0, :1].double().numpy(), 0.4, dv)
+    np.testing.assert_allclose(so[5], ro, rtol=0, atol=1e-12)
+
+
 def test_csa_core_attention_paged_equals_contiguous():
     g = torch.Generator().manual_seed(32)
     B, Lc, page, H, D = 2, 16, 4, 2, 8
