@@ -797,6 +797,7 @@ def run_tiny(dsa, workloads, device, peaks, args):
 
 
 V4_WINDOW = 128       # raw rows in the CSA window (the pages give no size)
+V4_SINK = 4           # raw rows in the CSA attention sink: the sequence's first rows (the pages give no size)
 HCA_M = 128           # HCA pooling factor m'
 
 
@@ -805,7 +806,8 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
     shapes (4 sequences of 1,048,576 raw tokens, one new query each):
 
     csa_step: pooled indexer keys -> top-1024 pooled entries -> CSA core
-      attention over those entries plus a window of the last 128 raw rows.
+      attention over those entries plus a window of the last 128 raw rows
+      and a sink of the first 4 raw rows.
       The pooling itself (csa_compress) runs once per 4 new tokens in a real
       cache and is not part of the step.
     hca: dense attention of each query over all 8,192 entries of the 128:1
@@ -825,7 +827,7 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
     idx = torch.empty((rows, wl.topk), dtype=torch.int32, device=device)
     n = dsa.topk_workspace_size(rows, ctx, wl.topk)
     tws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
-    n = dsa.sparse_mla_workspace_size(rows, wl.topk + V4_WINDOW, wl.heads, wl.d_qk, wl.d_v, torch.bfloat16)
+    n = dsa.sparse_mla_workspace_size(rows, wl.topk + V4_WINDOW + V4_SINK, wl.heads, wl.d_qk, wl.d_v, torch.bfloat16)
     mws = torch.empty(max(n, 1), dtype=torch.uint8, device=device)
     out = torch.empty((rows, wl.heads, wl.d_v), dtype=torch.bfloat16, device=device)
     lse = torch.empty((rows, wl.heads), dtype=torch.float32, device=device)
@@ -839,7 +841,7 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
                 dsa.topk(logits, inp["row_pos"], wl.topk, ctx_len=ctx, out=idx, workspace=tws)
             else:
                 dsa.csa_core_attention(inp["q"], kv_c, idx, inp["row_batch"], wl.softmax_scale, wl.d_v, ctx, raw_kv,
-                                       win_pos, V4_WINDOW, out=out, lse=lse, workspace=mws)
+                                       win_pos, V4_WINDOW, out=out, lse=lse, workspace=mws, n_sink=V4_SINK)
 
         def run(self):
             for nm in ("dsa_indexer_logits", "dsa_topk", "csa_core_attention"):
@@ -861,10 +863,10 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
     ga.replay()
     ms_attn = time_graph(ga, steps, device, flush_read=evict)["median"]
     del ga
-    sel_rows = rows * (wl.topk + V4_WINDOW)
+    sel_rows = rows * (wl.topk + V4_WINDOW + V4_SINK)
     step_bytes = (indexer_bytes(wl) + sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2)
     attn_bytes = sel_rows * wl.d_qk * 2 + rows * wl.heads * (wl.d_qk + wl.d_v) * 2
-    csa = {"workload": f"{wl.name}+window{V4_WINDOW}", "value": round(rows * world / (ms / 1e3), 1),
+    csa = {"workload": f"{wl.name}+window{V4_WINDOW}+sink{V4_SINK}", "value": round(rows * world / (ms / 1e3), 1),
            "unit": "queries/s", "ms_per_step": round(ms, 4), "ms_stats": stats_json(st_step),
            "core_attention_ms": round(ms_attn, 4),
            "roofline": {"bound": "hbm", "achieved": round(step_bytes / (ms / 1e3) / 1e9, 1),
@@ -875,7 +877,8 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
            "l2": "step: pooled keys (268 MB) exceed L2, no flush; core attention alone: 256 MB read between replays"}
     if rank == 0 and world == 1 and args.cpu_baseline:
         import oracle
-        win_rows = raw_kv[:, wl.raw_ctx - V4_WINDOW:].cpu()           # the window's raw rows, host copy
+        # host copy of the raw rows the step reads: the sink rows, then the window's rows
+        win_rows = torch.cat([raw_kv[:, :V4_SINK], raw_kv[:, wl.raw_ctx - V4_WINDOW:]], dim=1).cpu()
         keys_h, kvc_h = k_c.cpu(), kv_c.cpu()
         rb0 = torch.zeros(1, dtype=torch.int32)
 
@@ -885,8 +888,8 @@ def run_v4_variants(dsa, workloads, device, peaks, args):
             sc = oracle.index_scores(inp["q_idx"][r:r + 1].cpu(), inp["w"][r:r + 1].cpu(), keys_h[b:b + 1], rb0, rp)
             sel = oracle.topk(sc, rp, wl.topk)
             oracle.csa_core_attention(inp["q"][r:r + 1].cpu(), kvc_h[b:b + 1], sel, rb0, wl.softmax_scale, wl.d_v,
-                                      ctx, win_rows[b:b + 1], torch.tensor([V4_WINDOW - 1], dtype=torch.int32),
-                                      V4_WINDOW)
+                                      ctx, win_rows[b:b + 1], torch.tensor([V4_SINK + V4_WINDOW - 1], dtype=torch.int32),
+                                      V4_WINDOW, n_sink=V4_SINK)
         v, n, secs = _oracle_rows(csa_row, rows, 6.0)
         csa["cpu_baseline"] = {"value": round(v, 4), "unit": "queries/s", "cores": oracle.max_threads(),
                                "kind": "oracle", "sample": f"{n} whole query rows ({secs:.1f} s of CPU work)"}

@@ -10,7 +10,7 @@
  *
  * and two variants of the last step for DeepSeek-V4's compressed attention:
  *
- *   csa_core_attention  CSA: the selected compressed entries plus a window of raw rows
+ *   csa_core_attention  CSA: the selected compressed entries plus a window and a sink of raw rows
  *   hca_attention       HCA: dense attention over every visible heavily compressed entry
  *
  * and the step before the path, which makes the indexer's inputs:
@@ -201,39 +201,53 @@ DSA_API dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t d
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * csa_core_attention -- CSA core attention with the window segment
- * ("DeepSeek V4 发布：1.6T 参数、百万上下文…", section on CSA: the window KV
- * and the compressed KV are concatenated and attended together; CSA
- * pipeline "compress -> index selection -> core attention" in
- * "DeepSeek-V4 技术报告深度解析").  Slot s of query row t holds
+ * csa_core_attention -- CSA core attention with the window and attention-sink
+ * segments ("DeepSeek V4 发布：1.6T 参数、百万上下文…", section on CSA: the
+ * window KV and the compressed KV are concatenated and attended together;
+ * CSA pipeline "compress -> index selection -> core attention" in
+ * "DeepSeek-V4 技术报告深度解析"; "解密DeepSeek-V4 预览版…" section 4.3 and
+ * "打破幻觉与成本魔咒：DeepSeek-V4 …" section 3.3.2: local dependencies are
+ * kept by sliding-window attention together with an attention sink).  Slot
+ * s of query row t holds
  *   s <  k:            the selected compressed entry idx[t, s] of kv, exactly
  *                      as in dsa_sparse_mla (-1 = unused slot);
  *   k <= s < k+window: the raw (uncompressed) cache row
  *                      p = win_pos[t] - window + 1 + (s - k) of kv_win,
- *                      unused when p < 0,
+ *                      unused when p < 0;
+ *   k+window <= s < k+window+n_sink:
+ *                      the sink: raw row j = s - k - window of kv_win (the
+ *                      sequence's first rows), used only when
+ *                      j < win_pos[t] - window + 1, i.e. before the window's
+ *                      first row (so no raw row is attended twice, and none
+ *                      after the query),
  * and attention runs over all used slots together:
  *   out[t,h,:] = sum_s softmax_s(scale * q[t,h,:] . c_s[0:d_qk]) * c_s[0:d_v].
- * A window row is not deduplicated against a compressed entry that covers
- * it: the two are different vectors.
+ * A raw row is not deduplicated against a compressed entry that covers it:
+ * the two are different vectors.
  *
  *   kv_win   [batch, win_len, d_qk] contiguous raw cache of dtype, 16-byte
  *            aligned (the bf16 tensor-core path)
  *   win_pos  [rows] int32 raw position of each query (its window ends there);
  *            win_pos[t] >= win_len is skipped and reported by
  *            dsa_get_device_error
- *   window   rows per window, >= 0 (0: plain dsa_sparse_mla); k >= 0 and
- *            k + window >= 1; idx may be NULL when k = 0
+ *   window   rows per window, >= 0
+ *   n_sink   sink rows, 0 <= n_sink <= win_len (0: no sink; window = n_sink
+ *            = 0: plain dsa_sparse_mla); k >= 0 and k + window + n_sink >= 1;
+ *            idx may be NULL when k = 0; kv_win and win_pos are needed when
+ *            window + n_sink > 0
  * Other arguments, layouts, results and errors are those of dsa_sparse_mla;
- * the workspace is dsa_sparse_mla_workspace_size(rows, k + window, ...).
- * The pages name no window size and no attention sink: the caller chooses
- * the window, and no sink term is added.
+ * the workspace is dsa_sparse_mla_workspace_size(rows, k + window + n_sink, ...).
+ * The pages give neither the window size nor the number of sink rows: the
+ * caller chooses both.  The sink is read as the sequence's first raw rows,
+ * the form that pairs a sink with a sliding window (a learned per-head
+ * logit is another reading; the pages define neither).
  */
 DSA_API dsa_status_t csa_core_attention(const void* q, const void* kv, dsa_dtype_t dtype,
                             const int32_t* page_table, int page_size, int num_pages,
                             const int32_t* row_batch, const int32_t* idx, int k,
                             int rows, int batch, int ctx_len,
                             const void* kv_win, const int32_t* win_pos, int win_len, int window,
-                            int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
+                            int n_sink, int n_heads, int d_qk, int d_v, float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*

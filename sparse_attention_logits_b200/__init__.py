@@ -53,7 +53,7 @@ _SIGS = {
     "dsa_sparse_mla_noalloc": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                       _i32, _f32, _vp, _vp, _vp]),
     "csa_core_attention": (_i32, [_vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32,
-                                  _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+                                  _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
     "hca_attention": (_i32, [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
                              _vp]),
     "dsa_indexer_prepare_workspace_size": (_sz, [_i32, _i32, _i32, _i32]),
@@ -222,11 +222,12 @@ def sparse_mla(q: torch.Tensor, kv: torch.Tensor, idx: torch.Tensor, row_batch: 
 def csa_core_attention(q: torch.Tensor, kv: torch.Tensor, idx: Optional[torch.Tensor], row_batch: torch.Tensor,
                        scale: float, d_v: int, ctx_len: int, kv_win: torch.Tensor, win_pos: torch.Tensor, window: int,
                        page_table: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                       lse: Optional[torch.Tensor] = None,
-                       workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       n_sink: int = 0) -> Tuple[torch.Tensor, torch.Tensor]:
     """CSA core attention: the selected compressed entries idx of kv plus the
     window of `window` raw rows of kv_win [B, win_len, d_qk] ending at
-    win_pos[t] (out [rows, H, d_v], lse [rows, H] fp32)."""
+    win_pos[t] and the sink of the first `n_sink` raw rows (those before the
+    window) (out [rows, H, d_v], lse [rows, H] fp32)."""
     dev = _dev(q, kv, idx, row_batch, kv_win, win_pos, page_table, out, lse, workspace)
     rows, H, DK = q.shape
     k = 0 if idx is None else idx.shape[1]
@@ -244,14 +245,14 @@ def csa_core_attention(q: torch.Tensor, kv: torch.Tensor, idx: Optional[torch.Te
         out = torch.empty((rows, H, d_v), dtype=q.dtype, device=dev)
     if lse is None:
         lse = torch.empty((rows, H), dtype=torch.float32, device=dev)
-    need = sparse_mla_workspace_size(rows, k + window, H, DK, d_v, q.dtype)
+    need = sparse_mla_workspace_size(rows, k + window + n_sink, H, DK, d_v, q.dtype)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
     with torch.cuda.device(dev):
         _check(_lib.csa_core_attention(_ptr(q), _ptr(kv), _dt(q), _ptr(page_table), page_size, num_pages,
                                        _ptr(row_batch), _ptr(idx), k, rows, B, ctx_len, _ptr(kv_win), _ptr(win_pos),
-                                       kv_win.shape[1], window, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
+                                       kv_win.shape[1], window, n_sink, H, DK, d_v, float(scale), _ptr(out), _ptr(lse),
                                        _ptr(workspace), wsb, _stream(dev)), "csa_core_attention")
     return out, lse
 

@@ -327,16 +327,20 @@ dsa_status_t sparse_attention(const char* name, const void* q, const void* kv, d
                               int d_v, float scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                               void* stream, const dsa::KvExtra& x) {
     const int window = x.kv2 ? x.window : 0;
-    if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 0 || window < 0 || k + window < 1 || n_heads <= 0 ||
+    const int n_sink = x.kv2 ? x.n_sink : 0;
+    if (rows < 0 || batch <= 0 || ctx_len <= 0 || k < 0 || window < 0 || n_sink < 0 ||
+        (int64_t)k + window + n_sink < 1 || (int64_t)k + window + n_sink > (1 << 30) || n_heads <= 0 ||
         d_qk <= 0 || d_v <= 0 || d_v > d_qk)
         return fail(DSA_ERR_INVALID_ARG, "%s: bad sizes", name);
+    const bool raw = window + n_sink > 0;                   // a segment of raw rows
     if ((int64_t)batch * ctx_len >= ((int64_t)1 << 31) - 2 ||
-        (window > 0 && (int64_t)batch * x.len2 >= ((int64_t)1 << 31) - 2))
+        (raw && (int64_t)batch * x.len2 >= ((int64_t)1 << 31) - 2))
         return fail(DSA_ERR_UNSUPPORTED, "%s: a cache holds more than 2^31 - 2 rows", name);
     if (rows == 0) return DSA_OK;
     if (!q || !kv || !row_batch || !out || !lse || (k > 0 && !idx && !x.row_last))
         return fail(DSA_ERR_INVALID_ARG, "%s: null pointer", name);
-    if (window > 0 && (!x.pos2 || x.len2 <= 0)) return fail(DSA_ERR_INVALID_ARG, "%s: window needs win_pos and win_len", name);
+    if (raw && (!x.pos2 || x.len2 <= 0))
+        return fail(DSA_ERR_INVALID_ARG, "%s: a window or sink needs win_pos and win_len", name);
     if (dtype != DSA_BF16 && dtype != DSA_FP32) return fail(DSA_ERR_UNSUPPORTED, "%s: dtype must be bf16 or fp32", name);
     if (page_table) {
         if (page_size <= 0 || ctx_len % page_size)
@@ -351,9 +355,9 @@ dsa_status_t sparse_attention(const char* name, const void* q, const void* kv, d
     dsa_status_t st = make_launch(stream, &L);
     if (st != DSA_OK) return st;
     if (tc) {
-        if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || (window > 0 && !aligned(x.kv2, 16)))
+        if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || (raw && !aligned(x.kv2, 16)))
             return fail(DSA_ERR_INVALID_ARG, "%s: q, kv, the window cache and out must be 16-byte aligned", name);
-        const size_t need = dsa::mla_tc_workspace_bytes(rows, k + window, L.num_sms);
+        const size_t need = dsa::mla_tc_workspace_bytes(rows, k + window + n_sink, L.num_sms);
         if (need && (!workspace || workspace_bytes < need))
             return fail(DSA_ERR_INVALID_ARG, "%s: workspace of %zu bytes needed", name, need);
         return cuda_status(dsa::launch_mla_tc(L, q, kv, page_table, page_size, num_pages, row_batch, idx, k, rows,
@@ -383,15 +387,18 @@ dsa_status_t dsa_sparse_mla(const void* q, const void* kv, dsa_dtype_t dtype, co
 dsa_status_t csa_core_attention(const void* q, const void* kv, dsa_dtype_t dtype, const int32_t* page_table,
                                 int page_size, int num_pages, const int32_t* row_batch, const int32_t* idx, int k,
                                 int rows, int batch, int ctx_len, const void* kv_win, const int32_t* win_pos,
-                                int win_len, int window, int n_heads, int d_qk, int d_v, float scale, void* out,
-                                float* lse, void* workspace, size_t workspace_bytes, void* stream) {
-    if (window < 0 || (window > 0 && !kv_win)) return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: bad window");
+                                int win_len, int window, int n_sink, int n_heads, int d_qk, int d_v, float scale,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+    if (window < 0 || n_sink < 0 || (window + n_sink > 0 && !kv_win))
+        return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: bad window or sink");
+    if (n_sink > win_len) return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: n_sink above win_len");
     if (rows > 0 && k > 0 && !idx) return fail(DSA_ERR_INVALID_ARG, "csa_core_attention: null pointer");
     dsa::KvExtra x;
     x.kv2 = kv_win;
     x.pos2 = win_pos;
     x.len2 = win_len;
     x.window = window;
+    x.n_sink = n_sink;
     return sparse_attention("csa_core_attention", q, kv, dtype, page_table, page_size, num_pages, row_batch, idx, k,
                             rows, batch, ctx_len, n_heads, d_qk, d_v, scale, out, lse, workspace, workspace_bytes,
                             stream, x);

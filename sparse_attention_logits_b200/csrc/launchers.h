@@ -28,11 +28,15 @@ bool topk_supported(int ctx_len);
 //  - a window segment: slots [k, k + window) of row t are the raw cache rows
 //    pos2[t] - window + 1 .. pos2[t] of kv2 [batch, len2, d_qk] (positions
 //    below 0 are unused slots);
+//  - a sink segment: slots [k + window, k + window + n_sink) are the raw
+//    rows 0 .. n_sink - 1 of kv2, each used only when it lies before the
+//    window's first position pos2[t] - window + 1 (so no raw row is
+//    attended twice, and none after the query);
 //  - dense mode (idx == NULL): slot s < k is key s when s <= row_last[t].
 struct KvExtra {
     const void* kv2 = nullptr;
     const int32_t* pos2 = nullptr;
-    int len2 = 0, window = 0;
+    int len2 = 0, window = 0, n_sink = 0;
     const int32_t* row_last = nullptr;
 };
 

@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
     const T* __restrict__ q, const T* __restrict__ kv, const int32_t* __restrict__ page_table, int page_size,
     int pages_per_seq, int num_pages, const int32_t* __restrict__ row_batch, const int32_t* __restrict__ idx, int k,
     int batch, int ctx_len, int n_heads, float scale, T* __restrict__ out, float* __restrict__ lse, unsigned* err,
-    const T* __restrict__ kv2, const int32_t* __restrict__ pos2, int len2, int window,
+    const T* __restrict__ kv2, const int32_t* __restrict__ pos2, int len2, int window, int n_sink,
     const int32_t* __restrict__ row_last) {
     pdl_wait();
     constexpr int DK = QPL * 32, DV = VPL * 32;
@@ -51,16 +51,17 @@ __global__ void __launch_bounds__(256) mla_simt_kernel(
 
     const int32_t* sel = idx ? idx + (int64_t)t * k : nullptr;
     const int last = idx ? 0 : row_last[t];
-    const int wpos = window > 0 ? pos2[t] : 0;
-    const int ktot = k + window;
+    const int wfirst = window + n_sink > 0 ? pos2[t] - window + 1 : 0;   // the window's first raw position
+    const int ktot = k + window + n_sink;
     for (int j0 = 0; j0 < ktot; j0 += MLA_SIMT_TILE) {
         __syncthreads();
         // gather up to 16 slots (warp w loads slots w and w+8): selected keys
-        // (or every visible key in dense mode), then the window rows
+        // (or every visible key in dense mode), then the window rows, then
+        // the sink rows that lie before the window
         for (int r = warp; r < MLA_SIMT_TILE; r += 8) {
             const int j = j0 + r;
             if (j >= k && j < ktot) {
-                const int s = wpos - window + 1 + (j - k);
+                const int s = j - k < window ? wfirst + (j - k) : (j - k - window < wfirst ? j - k - window : -1);
                 const bool ok = row_ok && s >= 0 && s < len2;
                 if (s >= len2) record_error(err, DEV_ERR_BAD_INDEX);
                 const int64_t row = (int64_t)b * len2 + s;
@@ -124,7 +125,8 @@ static cudaError_t launch_t(const Launch& L, const void* q, const void* kv, cons
     cfg.numAttrs = 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_simt_kernel<T, QPL, VPL>, (const T*)q, (const T*)kv, pt, page_size,
                                              pages_per_seq, num_pages, rb, idx, k, batch, ctx, H, scale, (T*)out, lse,
-                                             L.err, (const T*)x.kv2, x.pos2, x.len2, x.kv2 ? x.window : 0, x.row_last);
+                                             L.err, (const T*)x.kv2, x.pos2, x.len2, x.kv2 ? x.window : 0,
+                                             x.kv2 ? x.n_sink : 0, x.row_last);
     count_launch();
     return e;
 }

@@ -110,14 +110,14 @@ struct MlaParams {
     const int32_t* row_last;
     const __nv_bfloat16* kv2;       // window segment: raw cache [batch, len2, DK]
     const int32_t* pos2;            // [rows] raw position of each query
-    int len2, window;
+    int len2, window, n_sink;
     __nv_bfloat16* out;
     float* lse;
     __nv_bfloat16* part_o;          // [rows, splits, H, DV] normalised partials when splits > 1
     float* part_lse;                // [rows, splits, H]
     unsigned* err;
     int page_size, pages_per_seq, num_pages;
-    int k, ktot, rows, batch, ctx, splits, per_split;   // ktot = k + window slots per row
+    int k, ktot, rows, batch, ctx, splits, per_split;   // ktot = k + window + n_sink slots per row
     int fuse2;                      // two key splits per row in one 4-CTA cluster, merged in the kernel
     float scale_log2;
 };
@@ -142,9 +142,10 @@ __device__ __forceinline__ Work work_of(const MlaParams& p) {
 
 // Key position held by slot `slot` of this row (-1: unused), before range
 // checks: selected (or, in dense mode, every visible) key for slot < k, raw
-// window position for k <= slot < ktot.
-// EXT = false compiles the plain selected-rows path (no window, no dense
-// mode) exactly as lean as it was before those existed.
+// window position for k <= slot < k + window, raw sink position (only before
+// the window's first position) for k + window <= slot < ktot.
+// EXT = false compiles the plain selected-rows path (no window, sink or
+// dense mode) exactly as lean as it was before those existed.
 template <bool EXT>
 __device__ __forceinline__ int slot_key(const MlaParams& p, const Work& w, int slot) {
     if (!EXT) return __ldg(p.idx + (int64_t)w.t * p.k + slot);
@@ -152,8 +153,10 @@ __device__ __forceinline__ int slot_key(const MlaParams& p, const Work& w, int s
         if (p.idx) return __ldg(p.idx + (int64_t)w.t * p.k + slot);
         return slot <= __ldg(p.row_last + w.t) ? slot : -1;
     }
-    const int s = __ldg(p.pos2 + w.t) - p.window + 1 + (slot - p.k);
-    return s < 0 ? -1 : s;
+    const int first = __ldg(p.pos2 + w.t) - p.window + 1;     // the window's first raw position
+    const int j = slot - p.k;
+    if (j < p.window) return first + j < 0 ? -1 : first + j;
+    return j - p.window < first ? j - p.window : -1;        // sink row j - window
 }
 
 // Row to gather for a slot: >= 0 a row of kv, <= -2 the row -2 - r of the
@@ -869,6 +872,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.pos2 = x.pos2;
     p.len2 = x.len2;
     p.window = x.kv2 ? x.window : 0;
+    p.n_sink = x.kv2 ? x.n_sink : 0;
     p.out = (__nv_bfloat16*)out;
     p.lse = lse;
     p.err = L.err;
@@ -876,7 +880,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.pages_per_seq = page_table ? ctx_len / page_size : 0;
     p.num_pages = page_table ? num_pages : 0;
     p.k = k;
-    p.ktot = k + p.window;
+    p.ktot = k + p.window + p.n_sink;
     p.rows = rows;
     p.batch = batch;
     p.ctx = ctx_len;
@@ -887,7 +891,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.part_o = nullptr;
     p.part_lse = nullptr;
-    const bool ext = p.window > 0 || !p.idx;
+    const bool ext = p.window > 0 || p.n_sink > 0 || !p.idx;
     auto kern = ext ? mla_tc_kernel<true> : mla_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
     if (e != cudaSuccess) return e;

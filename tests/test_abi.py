@@ -98,12 +98,16 @@ def test_v4_attention_arguments_rejected_before_launch(lib):
     vp, ci = ctypes.c_void_p, ctypes.c_int
     fake = vp(0x1000)      # never dereferenced: validation fails first
     lib.csa_core_attention.argtypes = [vp, vp, ci, vp, ci, ci, vp, vp, ci, ci, ci, ci, vp, vp, ci, ci, ci, ci, ci,
-                                       ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
+                                       ci, ctypes.c_float, vp, vp, vp, ctypes.c_size_t, vp]
 
-    def csa(idx, k, kv_win, win_pos, win_len, window, n_heads=128):
+    def csa(idx, k, kv_win, win_pos, win_len, window, n_heads=128, n_sink=0):
         return lib.csa_core_attention(fake, fake, 1, None, 0, 0, fake, idx, k, 4, 4, 1024, kv_win, win_pos, win_len,
-                                      window, n_heads, 576, 512, 0.04, fake, fake, None, 0, None)
+                                      window, n_sink, n_heads, 576, 512, 0.04, fake, fake, None, 0, None)
     assert csa(fake, 64, fake, fake, 4096, -1) == 1                  # negative window
+    assert csa(fake, 64, fake, fake, 4096, 128, n_sink=-1) == 1      # negative sink
+    assert csa(fake, 64, None, fake, 4096, 0, n_sink=4) == 1         # sink without its cache
+    assert csa(fake, 64, fake, None, 4096, 0, n_sink=4) == 1         # sink without positions
+    assert csa(fake, 64, fake, fake, 16, 8, n_sink=17) == 1          # more sink rows than the raw cache holds
     assert csa(fake, 64, None, fake, 4096, 128) == 1                 # window without its cache
     assert csa(fake, 64, fake, None, 4096, 128) == 1                 # window without positions
     assert csa(None, 0, fake, fake, 4096, 0) == 1                    # no slot at all

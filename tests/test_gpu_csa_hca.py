@@ -45,20 +45,27 @@ def _check(out, lse, ro, rl, dtype):
     assert lerr <= ATOL_LSE[key], lerr
 
 
-# (rows, B, raw length, k, window, window end, page size, dtype, heads, d_qk, d_v)
+# (rows, B, raw length, k, window, window end, page size, dtype, heads, d_qk, d_v, sink rows)
 CSA_CASES = {
-    "bf16_rows4_split": (4, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512),
-    "bf16_rows32_fused_splits": (32, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512),
-    "bf16_window_clipped": (4, 2, 2048, 192, 128, "early", 0, torch.bfloat16, 128, 576, 512),
-    "bf16_window_only": (3, 3, 1024, 0, 100, "end", 0, torch.bfloat16, 128, 576, 512),
-    "bf16_paged": (5, 2, 4096, 300, 64, "end", 64, torch.bfloat16, 128, 576, 512),
-    "fp32_small_heads": (6, 2, 256, 16, 32, "early", 0, torch.float32, 8, 64, 64),
+    "bf16_rows4_split": (4, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512, 0),
+    "bf16_rows32_fused_splits": (32, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512, 0),
+    "bf16_window_clipped": (4, 2, 2048, 192, 128, "early", 0, torch.bfloat16, 128, 576, 512, 0),
+    "bf16_window_only": (3, 3, 1024, 0, 100, "end", 0, torch.bfloat16, 128, 576, 512, 0),
+    "bf16_paged": (5, 2, 4096, 300, 64, "end", 64, torch.bfloat16, 128, 576, 512, 0),
+    "fp32_small_heads": (6, 2, 256, 16, 32, "early", 0, torch.float32, 8, 64, 64, 0),
+    # attention sink: the first raw rows beside the window
+    "bf16_sink_rows4_split": (4, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512, 4),
+    "bf16_sink_rows32_fused_splits": (32, 4, 4096, 256, 128, "end", 0, torch.bfloat16, 128, 576, 512, 64),
+    "bf16_sink_window_overlap": (6, 2, 2048, 192, 128, "overlap", 0, torch.bfloat16, 128, 576, 512, 100),
+    "bf16_sink_only": (3, 3, 1024, 0, 0, "overlap", 0, torch.bfloat16, 128, 576, 512, 70),
+    "bf16_sink_paged": (5, 2, 4096, 300, 64, "end", 64, torch.bfloat16, 128, 576, 512, 16),
+    "fp32_sink_small_heads": (6, 2, 256, 16, 32, "overlap", 0, torch.float32, 8, 64, 64, 20),
 }
 
 
 @pytest.mark.parametrize("case", list(CSA_CASES), ids=list(CSA_CASES))
 def test_csa_core_attention_matches_oracle(cuda_device, case):
-    rows, B, Lraw, k, W, end, page, dtype, H, DK, DV = CSA_CASES[case]
+    rows, B, Lraw, k, W, end, page, dtype, H, DK, DV, S = CSA_CASES[case]
     raw, g = _caches(B, Lraw, DK, dtype, seed=41)
     raw_d = raw.to(cuda_device)
     kvc = _pooled(raw_d, 4)
@@ -67,8 +74,11 @@ def test_csa_core_attention_matches_oracle(cuda_device, case):
     rb = (torch.arange(rows) % B).to(torch.int32)
     if end == "end":
         pos = torch.full((rows,), Lraw - 1, dtype=torch.int32)
-    else:                                   # windows that start before position 0
+    elif end == "early":                    # windows that start before position 0
         pos = torch.tensor([(7 * t) % W for t in range(rows)], dtype=torch.int32)
+    else:                                   # sink and window meet, overlap or the query sits inside the sink
+        pos = torch.tensor([[0, S // 2, S - 1, S + W - 2, S + W - 1, S + W + 37][t % 6] for t in range(rows)],
+                           dtype=torch.int32)
     idx = None
     if k:
         idx = torch.stack([torch.randperm(Lc, generator=g)[:k] for _ in range(rows)]).to(torch.int32)
@@ -85,9 +95,9 @@ def test_csa_core_attention_matches_oracle(cuda_device, case):
         kv_arg = pages
     out, lse = dsa.csa_core_attention(q.to(cuda_device), kv_arg, None if idx is None else idx.to(cuda_device),
                                       rb.to(cuda_device), scale, DV, Lc, raw_d, pos.to(cuda_device), W,
-                                      page_table=None if table is None else table.to(cuda_device))
-    dsa.get_device_error(cuda_device)
-    ro, rl = oracle.csa_core_attention(q, kvc.cpu(), idx, rb, scale, DV, Lc, raw, pos, W)
+                                      page_table=None if table is None else table.to(cuda_device), n_sink=S)
+    assert dsa.get_device_error(cuda_device) == dsa.DSA_OK
+    ro, rl = oracle.csa_core_attention(q, kvc.cpu(), idx, rb, scale, DV, Lc, raw, pos, W, n_sink=S)
     _check(out, lse, ro, rl, dtype)
 
 

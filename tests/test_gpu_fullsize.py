@@ -127,13 +127,14 @@ def test_full_size_sampled_rows(cuda_device, wl, sample):
 
 
 V4_WINDOW = 128
+V4_SINK = 4
 
 
 def test_full_size_v4_variants(cuda_device):
     """The 1M-token CSA shapes (4 sequences of 1,048,576 raw tokens) through
     the two variants of the attention step, in the bench's launch
     configuration: CSA core attention over 1024 seeded pooled entries plus a
-    128-row window of raw rows, and HCA over all 8,192 entries of the 128:1
+    128-row window and a 4-row sink of raw rows, and HCA over all 8,192 entries of the 128:1
     pooled cache.  Sampled rows are checked against the oracle, which pools
     the raw seeded rows itself."""
     wl = workloads.CSA_DECODE_1M
@@ -148,17 +149,19 @@ def test_full_size_v4_variants(cuda_device):
     g = torch.Generator().manual_seed(5)
     idx = torch.stack([torch.randperm(wl.ctx, generator=g)[:wl.topk] for _ in range(rows)]).to(torch.int32)
     out, lse = dsa.csa_core_attention(dv["q"], kv_c, idx.to(cuda_device), rb, wl.softmax_scale, wl.d_v, wl.ctx,
-                                      raw, pos, V4_WINDOW)
-    dsa.get_device_error()
+                                      raw, pos, V4_WINDOW, n_sink=V4_SINK)
+    assert dsa.get_device_error() == dsa.DSA_OK
     for t in (0, rows - 1):
         b = int(rb[t])
         sel = idx[t].long().to(cuda_device)
         raw_ids = (sel[:, None] * wl.compress_m + torch.arange(wl.compress_m, device=cuda_device)[None, :]).reshape(-1)
         pooled = oracle.csa_compress(raw[b, raw_ids].unsqueeze(0), wl.compress_m)            # [1, 1024, 576]
         pooled_t = torch.from_numpy(pooled.view(np.int16)).view(torch.bfloat16)
-        win = raw[b, Lraw - V4_WINDOW:].unsqueeze(0).cpu()
+        # the oracle's raw cache: the sink rows, then the window's rows (the query at its end)
+        win = torch.cat([raw[b, :V4_SINK], raw[b, Lraw - V4_WINDOW:]]).unsqueeze(0).cpu()
         ro, rl = oracle.csa_core_attention(dv["q"][t:t + 1].cpu(), pooled_t, torch.arange(wl.topk).view(1, -1), [0],
-                                           wl.softmax_scale, wl.d_v, wl.topk, win, [V4_WINDOW - 1], V4_WINDOW)
+                                           wl.softmax_scale, wl.d_v, wl.topk, win, [V4_SINK + V4_WINDOW - 1],
+                                           V4_WINDOW, n_sink=V4_SINK)
         assert np.abs(out[t].float().cpu().numpy() - ro[0]).max() <= ATOL_OUT["bf16"], f"csa row {t}"
         assert np.abs(lse[t].cpu().numpy() - rl[0]).max() <= ATOL_LSE["bf16"], f"csa row {t} lse"
     del kv_c, out, lse
