@@ -71,24 +71,36 @@ static_assert(PWARPS * 32 * REGS_LOW + 8 * 32 * REGS_SOFTMAX + 4 * 32 * REGS_LAU
               "register split exceeds launch");
 constexpr int KBLK = DK / 64;       // 9 dim blocks of 64 (128 B per row) per gathered row
 constexpr int VBLK = DV / 64;       // the value CTA gathers the first 8
-constexpr int KSTAGE = NK * DK * 2; // 73728 B
-constexpr int STAGES = 2;
-constexpr int REGION = STAGES * KSTAGE;  // [stage][dim block][64 rows x 128 B]
-constexpr int QBYTES = H * DK * 2;  // 147456: the Q tile, staged through the same region before the gather starts
-static_assert(QBYTES == REGION, "Q staging uses the gather region");
+constexpr int KSTAGE = NK * DK * 2; // 73728 B: one chunk's rows, [dim block][64 rows x 128 B]
+constexpr int SSTAGES = 3;          // score CTA: gather ring of full rows
+constexpr int VSTAGES = 2;          // value CTA: gather ring of value rows (KSTAGE-sized slots)
+constexpr int REGION = SSTAGES * KSTAGE;   // 221184: the role-specific part of shared memory
+constexpr int QBYTES = H * DK * 2;  // 147456: the Q tile
+constexpr int Q_OFF = KSTAGE;       // Q is staged in score stages 1-2, so chunk 0 is gathered into stage 0 at once
+static_assert(Q_OFF + QBYTES == REGION, "Q staging fills score stages 1 and 2");
 constexpr int EPI_BUF = 4096;       // epilogue: per-warp output staging tile (32 heads x 128 B), two per warp
 constexpr int PBYTES = H * NK * 2;  // 16384: P [128 heads x 64 keys] bf16
 constexpr int PSLOTS = 4;           // P ring depth (score CTA may run this many chunks ahead)
 constexpr int ABYTES = H * 4;       // rescale factor per head
 constexpr int SBYTES = 2 * H * 4;   // final running max and sum per head
+// value CTA: its V ring, then the P ring and the rescale factors that the
+// score CTA stores into it (st.async), inside the same region
+constexpr int PBUF_OFF = VSTAGES * KSTAGE;
+constexpr int ABUF_OFF = PBUF_OFF + PSLOTS * PBYTES;
+static_assert(ABUF_OFF + PSLOTS * ABYTES <= REGION, "value CTA layout");
+// the same offsets in every CTA: final statistics, scratch of the pair
+// meetings and fused merge, barriers (remote accesses use mapa)
+constexpr int SBUF_OFF = REGION;
+constexpr int XBUF_OFF = SBUF_OFF + SBYTES;
+constexpr int BARS_OFF = XBUF_OFF + 4 * H * 4;
 constexpr int S_COL = 320;          // score CTA: Q in TMEM columns [0, 288), S buffers at 320, 384
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between rescales)
 constexpr float LN2 = 0.6931471805599453f;
 
 struct Bars {                       // same offset in both CTAs of a cluster
-    uint64_t full[2];               // a stage's gathered rows have landed (cp.async arrivals)
-    uint64_t empty[2];              // the MMA is done reading a stage
+    uint64_t full[SSTAGES];         // a stage's gathered rows have landed (cp.async arrivals)
+    uint64_t empty[SSTAGES];        // the MMA is done reading a stage (score stages 1-2: first, Q has left)
     uint64_t sfull[2], sempty[2], pempty[PSLOTS], qready, statready, statack;
     // value CTA: P slot landed / rescaled, PV of chunk c done (ring of PSLOTS, so
     // that a parity wait never aliases), all PV done, final statistics landed
@@ -96,7 +108,7 @@ struct Bars {                       // same offset in both CTAs of a cluster
     uint64_t qfull;                 // score CTA: the Q tile has landed in shared memory
     uint64_t cfree, cstat, crecv;   // fused two-split merge (value CTAs): the other split's gather region is
                                     // drained / its statistics / its share of O have landed here
-    int flag[2][2][8];              // score CTA: per softmax warp "still ok" at the two pair barriers of a chunk
+    int flag[2][8];                 // score CTA: per softmax warp "still ok" at the pair meeting of a chunk
     uint32_t tmem;
     int abort;
 };
@@ -229,17 +241,22 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 
 // consecutive 16-byte pieces.  Many producer warps are used because the copy
 // throughput of an SM grows with the number of copies its threads keep in
 // flight.
-template <int NB, bool EXT>   // NB: dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
+//
+// Ring of NST stages, chunk c in stage c % NST.  Score CTA (NST = 3): stages
+// 1 and 2 first hold the Q tile, and their empty barrier's first phase is the
+// release of Q (after its copy to TMEM), so their gathers wait one phase
+// more than stage 0's, which starts at once.
+template <int NB, bool EXT, int NST>   // NB: dim blocks gathered per row (9: full 576-d rows; 8: the 512 value dims)
 __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, uint8_t* gbuf, Bars* bars, int warp,
                                             int lane, volatile int* abort_flag) {
     constexpr int RC = NB * 8;                           // 16-byte pieces per row
+    constexpr bool Q_IN_RING = NB == KBLK;               // score CTA
     const int my_slot = warp * ROWS_PER_PW + (lane % ROWS_PER_PW);
     int64_t next_row = key_row<EXT>(p, w, w.slot0 + my_slot);
-    // score CTA: the region holds the Q tile until it has been moved to TMEM
-    if (NB == KBLK && !mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)) return;
     for (int c = 0; c < w.nchunks; ++c) {
-        const int st = c & 1;
-        if (!mbar_wait(&bars->empty[st], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+        const int st = c % NST;
+        const uint32_t par = (uint32_t)((c / NST) & 1) ^ ((Q_IN_RING && st > 0) ? 0u : 1u);
+        if (!mbar_wait(&bars->empty[st], par, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
         const int myrow_lo = (int)next_row;     // row indices (and the window encoding) fit in 31 bits
         uint8_t* base = gbuf + (size_t)st * KSTAGE;
 #pragma unroll
@@ -272,12 +289,12 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* gbuf = smem;                                   // K (score CTA) or V (value CTA) stages
-    uint8_t* pbuf = gbuf + REGION;                          // [PSLOTS][PBYTES]
-    float* abuf = (float*)(pbuf + PSLOTS * PBYTES);         // [PSLOTS][H]
-    float* sbuf = abuf + PSLOTS * H;                        // [2*H]: running max, running sum
-    float* xbuf = sbuf + 2 * H;                             // [2][2][H]: partial maxima / sums of the two halves
+    uint8_t* pbuf = smem + PBUF_OFF;                        // value CTA: [PSLOTS][PBYTES]
+    float* abuf = (float*)(smem + ABUF_OFF);                // value CTA: [PSLOTS][H]
+    float* sbuf = (float*)(smem + SBUF_OFF);                // [2*H]: running max, running sum
+    float* xbuf = (float*)(smem + XBUF_OFF);                // [2][2][H]: partial maxima / sums of the two halves
                                                             // of a head (score CTA)
-    Bars* bars = (Bars*)(xbuf + 4 * H);
+    Bars* bars = (Bars*)(smem + BARS_OFF);
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -288,9 +305,11 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     const Work w = work_of(p);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < SSTAGES; ++i) {
             mbar_init(&bars->full[i], PWARPS * 32);
             mbar_init(&bars->empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sfull[i], 1);
             mbar_init(&bars->sempty[i], 8);
         }
@@ -319,10 +338,11 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         fence_mbar_init();
         if (role == 0) {
             // Q [128 heads x 576] of this row: 9 boxes of 128 rows x 64 dims,
-            // 128-byte swizzled, into the (still unused) gather region
+            // 128-byte swizzled, into gather stages 1-2 (not yet in use)
             tma_prefetch_desc(&q_map);
             mbar_arrive_expect_tx(&bars->qfull, QBYTES);
-            for (int b = 0; b < KBLK; ++b) tma_load_2d(gbuf + b * (H * 128), &q_map, b * 64, w.t * H, &bars->qfull);
+            for (int b = 0; b < KBLK; ++b)
+                tma_load_2d(gbuf + Q_OFF + b * (H * 128), &q_map, b * 64, w.t * H, &bars->qfull);
         } else {
             tma_prefetch_desc(&o_map);
         }
@@ -345,8 +365,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (role == 0) gather_rows<KBLK, EXT>(p, w, gbuf, bars, warp, lane, abort_flag);
-        else gather_rows<VBLK, EXT>(p, w, gbuf, bars, warp, lane, abort_flag);
+        if (role == 0) gather_rows<KBLK, EXT, SSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
+        else gather_rows<VBLK, EXT, VSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
     } else if (warp < SWARP0 + 8) {
       regs_inc<REGS_SOFTMAX>();
       if (role == 0) {
@@ -354,22 +374,24 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
         // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
         // of every chunk.  The two warps of a quarter (a "pair") meet at a
-        // named barrier twice per chunk: to combine their partial maxima, so
-        // both take the same rescaling decision, and once both halves of the
-        // quarter's P rows are in shared memory, after which one of them sends
-        // those rows and the quarter's rescale factors to the value CTA.  Each
-        // warp posts whether it is still ok at both meetings, so that the two
-        // always leave the loop together (a named barrier has no time limit).
+        // named barrier once per chunk to combine their partial maxima, so
+        // both take the same rescaling decision; each warp posts there whether
+        // its waits of the chunk succeeded, so that the two always leave the
+        // loop together (a named barrier has no time limit).  Every thread
+        // then stores its P row piece (and half 0 the head's rescale factor)
+        // straight into the value CTA's P slot with st.async, whose bytes are
+        // counted on the value CTA's barrier for that slot: the score CTA
+        // keeps no P ring, which leaves room for a third gather stage.
         const int sw = warp - SWARP0, half = sw >> 2, quarter = sw & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const int pair_bar = 1 + quarter;
-        volatile int* flag = &bars->flag[0][0][0];
+        volatile int* flag = &bars->flag[0][0];
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->qfull, 0, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag));
         if (ok) {   // Q row h -> TMEM lane h; this half writes the 16-column groups [9*half, 9*half + 9)
 #pragma unroll 1
             for (int g = 9 * half; g < 9 * half + 9; ++g) {
-                const uint8_t* row = gbuf + (g >> 1) * (H * 128) + h * 128;
+                const uint8_t* row = gbuf + Q_OFF + (g >> 1) * (H * 128) + h * 128;
                 uint32_t words[16];
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
@@ -384,8 +406,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->qready);
         float m_run = -INFINITY, l_run = 0.f;                   // l_run: this half's keys
-        const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);
-        const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);
+        const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);    // the value CTA's P ring
+        const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);    // and its rescale factors
         // whether this lane's key of a chunk is real: the raw index is loaded
         // one chunk ahead and only inspected in the next iteration
         int s_next = slot_index<EXT>(p, w, w.slot0 + 32 * half + lane);
@@ -410,6 +432,11 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 32; ++j) sv[j] = 0.f;
             }
+            const int pb = c % PSLOTS, pu = c / PSLOTS;
+            // the slot's previous P has been consumed by the value CTA's MMA
+            if (ok)
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER,
+                                                       abort_flag));
             float mx[16];
 #pragma unroll
             for (int j = 0; j < 32; ++j) sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
@@ -421,9 +448,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                 for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
             float* xb = xbuf + par * 2 * H;
             xb[half * H + h] = mx[0];
-            if (lane == 0) flag[(0 * 2 + par) * 8 + sw] = ok ? 1 : 0;
+            if (lane == 0) flag[par * 8 + sw] = ok ? 1 : 0;
             named_bar_sync(pair_bar, 64);
-            ok = ok && flag[(0 * 2 + par) * 8 + (sw ^ 4)] != 0;        // the same in both warps of the pair
+            ok = ok && flag[par * 8 + (sw ^ 4)] != 0;        // the same in both warps of the pair
             if (!ok) break;
             const float mc = fmaxf(mx[0], xb[(half ^ 1) * H + h]);
             float alpha = 1.f;
@@ -454,30 +481,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
 #pragma unroll
                 for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
             l_run += ls[0];
-            const int pb = c % PSLOTS, pu = c / PSLOTS;
-            // the slot's previous P has been consumed by the value CTA's MMA
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
-            if (ok) {
-                uint8_t* prow = pbuf + pb * PBYTES + (h >> 3) * 1024;
+            // P row h, keys [32 half, +32) (64 B, 128-B-swizzled K-major tile)
+            // and, from half 0, the head's rescale factor: 256 x 64 + 128 x 4
+            // bytes per chunk, the count the value CTA expects on pfull[pb]
+            const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
+            const uint32_t prow = peer_pbuf + (uint32_t)(pb * PBYTES + (h >> 3) * 1024);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    st_shared_v4(prow + sw128(h & 7, 4 * half + jj), pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2],
-                                 pk[4 * jj + 3]);
-                if (half == 0) abuf[pb * H + h] = alpha;
-                fence_proxy_async_smem();
-            }
-            if (lane == 0) flag[(1 * 2 + par) * 8 + sw] = ok ? 1 : 0;
-            named_bar_sync(pair_bar, 64);
-            ok = ok && flag[(1 * 2 + par) * 8 + (sw ^ 4)] != 0;
-            if (!ok) break;
-            if (half == 0 && lane == 0) {
-                // this quarter's 32 P rows (4 KB, contiguous) and 32 rescale factors
-                const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
-                const uint32_t poff = (uint32_t)(pb * PBYTES + quarter * 4096);
-                bulk_copy_s2cluster(peer_pbuf + poff, pbuf + poff, 4096, rbar);
-                bulk_copy_s2cluster(peer_abuf + pb * ABYTES + quarter * 128, abuf + pb * H + quarter * 32, 128, rbar);
-            }
+            for (int jj = 0; jj < 4; ++jj)
+                st_async_v4(prow + sw128(h & 7, 4 * half + jj), pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2],
+                            pk[4 * jj + 3], rbar);
+            if (half == 0) st_async_b32(peer_abuf + (uint32_t)(pb * ABYTES + h * 4), __float_as_uint(alpha), rbar);
         }
         // final statistics -> value CTA: running max (same in both halves) and
         // the sum of the two halves' running sums
@@ -518,7 +531,9 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         if (colhalf == 0) {
             for (int c = 0; c < w.nchunks && ok; ++c) {
                 const int pb = c % PSLOTS, pu = c / PSLOTS;
-                ok = mbar_wait(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
+                // P and the rescale factors arrive as st.async stores from the
+                // score CTA (release at cluster scope): acquire at cluster scope
+                ok = mbar_wait_cluster(&bars->pfull[pb], pu & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 if (!ok) break;
                 if (warp == SWARP0 && lane == 0 && c + PSLOTS < w.nchunks)
                     mbar_arrive_expect_tx(&bars->pfull[pb], PBYTES + ABYTES);     // arm this slot's next use
@@ -712,10 +727,15 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                 const uint32_t kbase = smem_u32(gbuf);
                 bool ok = mbar_wait(&bars->qready, 0, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag);
                 tc_fence_after();
+                if (ok) {
+                    // Q is in TMEM: gather stages 1 and 2 are free for their first chunks
+                    mbar_arrive(&bars->empty[1]);
+                    mbar_arrive(&bars->empty[2]);
+                }
                 for (int c = 0; c < w.nchunks && ok; ++c) {
-                    const int st = c & 1, sb = c & 1, par = (c >> 1) & 1;
-                    ok = mbar_wait(&bars->sempty[sb], par ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag) &&
-                         mbar_wait(&bars->full[st], par, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                    const int st = c % SSTAGES, sb = c & 1;
+                    ok = mbar_wait(&bars->sempty[sb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag) &&
+                         mbar_wait(&bars->full[st], (c / SSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                     if (!ok) break;
                     fence_proxy_async_smem();
                     tc_fence_after();
@@ -805,8 +825,11 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(const __nv_bfloat16* _
 
 namespace {
 
-constexpr size_t MLA_SMEM = 1024 + REGION + PSLOTS * (PBYTES + ABYTES) + SBYTES + 4 * H * 4 + 1024;
+// 1024 B of room to round the base up to 1024 (128-B swizzle atoms), the
+// region, the statistics and pair scratch, the barrier block
+constexpr size_t MLA_SMEM = 1024 + (size_t)BARS_OFF + 1024;
 static_assert(sizeof(Bars) <= 1024, "barrier block");
+static_assert(MLA_SMEM <= 232448, "above the 227 KB of shared memory a CTA may use");
 
 int choose_splits(int rows, int k, int num_sms) {
     const int clusters = num_sms / 2;

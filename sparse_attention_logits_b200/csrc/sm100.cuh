@@ -376,6 +376,23 @@ __device__ __forceinline__ void bulk_copy_s2cluster(uint32_t dst_cluster_addr, c
         : "memory");
 }
 
+// 16-byte store into another CTA's shared memory (cluster address from
+// mapa); when it lands, its 16 bytes are counted (complete_tx, release at
+// cluster scope) on that CTA's mbarrier `remote_bar`.
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(remote_addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
+                 : "memory");
+}
+
+// The same for one 32-bit word.
+__device__ __forceinline__ void st_async_b32(uint32_t remote_addr, uint32_t v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+                 ::"r"(remote_addr), "r"(v), "r"(remote_bar)
+                 : "memory");
+}
+
 // tcgen05.commit that arrives on the mbarrier at the same shared-memory
 // offset in every CTA of `cta_mask`.
 __device__ __forceinline__ void mma_commit_multicast(uint64_t* bar, uint16_t cta_mask) {
