@@ -108,7 +108,7 @@ struct Bars {                       // same offset in both CTAs of a cluster
     uint64_t qfull;                 // score CTA: the Q tile has landed in shared memory
     uint64_t cfree, cstat, crecv;   // fused two-split merge (value CTAs): the other split's gather region is
                                     // drained / its statistics / its share of O have landed here
-    int flag[2][8];                 // score CTA: per softmax warp "still ok" at the pair meeting of a chunk
+    int mdone[4];                   // score CTA: per quarter, last chunk whose running maximum is published
     uint32_t tmem;
     int abort;
 };
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->sfull[i], 1);
-            mbar_init(&bars->sempty[i], 8);
+            mbar_init(&bars->sempty[i], 4);     // the softmax group of this S buffer
         }
         for (int i = 0; i < PSLOTS; ++i) {
             mbar_init(&bars->pempty[i], 1);
@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         mbar_init(&bars->ofinal, 1);
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
+        for (int i = 0; i < 4; ++i) bars->mdone[i] = -1;
         if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
         mbar_init(&bars->cfree, 1);
         mbar_init(&bars->cstat, H);
@@ -371,26 +372,29 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
       regs_inc<REGS_SOFTMAX>();
       if (role == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
-        // Warp SWARP0 + 4*half + quarter: thread (quarter, lane) owns head
-        // h = 32*quarter + lane (its TMEM lane) and keys [32*half, 32*half+32)
-        // of every chunk.  The two warps of a quarter (a "pair") meet at a
-        // named barrier once per chunk to combine their partial maxima, so
-        // both take the same rescaling decision; each warp posts there whether
-        // its waits of the chunk succeeded, so that the two always leave the
-        // loop together (a named barrier has no time limit).  Every thread
-        // then stores its P row piece (and half 0 the head's rescale factor)
-        // straight into the value CTA's P slot with st.async, whose bytes are
-        // counted on the value CTA's barrier for that slot: the score CTA
-        // keeps no P ring, which leaves room for a third gather stage.
-        const int sw = warp - SWARP0, half = sw >> 2, quarter = sw & 3;
+        // Two groups of 4 warps take alternate chunks: group g = chunk & 1
+        // (warps SWARP0 + 4g .. +3, group g reads S buffer g).  Thread
+        // (quarter, lane) of a group owns head h = 32*quarter + lane (its TMEM
+        // lane) and all 64 keys of its group's chunks, so a chunk needs no
+        // meeting between warps.  The only sequential part of the online
+        // softmax is the running maximum: chunk c takes m(c-1) from the other
+        // group's warp of the same quarter (published in shared memory, with a
+        // per-quarter chunk counter), decides lazily whether it moves (only
+        // when a score exceeds it by 2^8) and publishes m(c); the exponentials,
+        // the packing and the transfer of P then overlap the other group's
+        // chunk.  Each group keeps its own running sum relative to the maximum
+        // it last used; the two are brought to the final maximum at the end.
+        // P rows (and the head's rescale factor) go straight into the value
+        // CTA's P slot with st.async, whose bytes are counted on the value
+        // CTA's barrier for that slot, so the score CTA keeps no P ring.
+        const int sw = warp - SWARP0, grp = sw >> 2, quarter = sw & 3;
         const int h = quarter * 32 + lane;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-        const int pair_bar = 1 + quarter;
-        volatile int* flag = &bars->flag[0][0];
+        float* mpub = xbuf;                                  // [2][H]: m(c) of the last chunk of group c & 1
         bool ok = __all_sync(0xffffffffu, mbar_wait(&bars->qfull, 0, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag));
-        if (ok) {   // Q row h -> TMEM lane h; this half writes the 16-column groups [9*half, 9*half + 9)
+        if (ok) {   // Q row h -> TMEM lane h; group g writes the 16-column groups [9g, 9g + 9)
 #pragma unroll 1
-            for (int g = 9 * half; g < 9 * half + 9; ++g) {
+            for (int g = 9 * grp; g < 9 * grp + 9; ++g) {
                 const uint8_t* row = gbuf + Q_OFF + (g >> 1) * (H * 128) + h * 128;
                 uint32_t words[16];
 #pragma unroll
@@ -405,103 +409,136 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->qready);
-        float m_run = -INFINITY, l_run = 0.f;                   // l_run: this half's keys
+        float m_own = -INFINITY, l_own = 0.f;     // this group's sum, relative to the maximum it last used
         const uint32_t peer_pbuf = mapa_shared(smem_u32(pbuf), peer);    // the value CTA's P ring
         const uint32_t peer_abuf = mapa_shared(smem_u32(abuf), peer);    // and its rescale factors
-        // whether this lane's key of a chunk is real: the raw index is loaded
-        // one chunk ahead and only inspected in the next iteration
-        int s_next = slot_index<EXT>(p, w, w.slot0 + 32 * half + lane);
-        for (int c = 0; c < w.nchunks; ++c) {
-            const int sb = c & 1, par = c & 1;
-            const uint32_t vmask = __ballot_sync(
-                0xffffffffu,
-                w.b_ok && s_next >= 0 && s_next < slot_limit<EXT>(p, w.slot0 + c * NK + 32 * half + lane));
-            if (c + 1 < w.nchunks) s_next = slot_index<EXT>(p, w, w.slot0 + (c + 1) * NK + 32 * half + lane);
-            float sv[32];
-            if (ok)
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag));
-            if (ok) {
-                tc_fence_after();
-                tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32 * half, sv);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->sempty[sb]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) sv[j] = 0.f;
+        // key positions of this lane's two keys (lane, 32 + lane) of the
+        // group's next chunk, loaded one group chunk ahead
+        int s_lo = grp < w.nchunks ? slot_index<EXT>(p, w, w.slot0 + grp * NK + lane) : -1;
+        int s_hi = grp < w.nchunks ? slot_index<EXT>(p, w, w.slot0 + grp * NK + 32 + lane) : -1;
+        for (int c = grp; c < w.nchunks; c += 2) {
+            const int sb = grp;
+            const int slot0 = w.slot0 + c * NK;
+            const uint32_t vm_lo = __ballot_sync(0xffffffffu, w.b_ok && s_lo >= 0 && s_lo < slot_limit<EXT>(p, slot0 + lane));
+            const uint32_t vm_hi =
+                __ballot_sync(0xffffffffu, w.b_ok && s_hi >= 0 && s_hi < slot_limit<EXT>(p, slot0 + 32 + lane));
+            if (c + 2 < w.nchunks) {
+                s_lo = slot_index<EXT>(p, w, slot0 + 2 * NK + lane);
+                s_hi = slot_index<EXT>(p, w, slot0 + 2 * NK + 32 + lane);
             }
-            const int pb = c % PSLOTS, pu = c / PSLOTS;
-            // the slot's previous P has been consumed by the value CTA's MMA
-            if (ok)
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER,
-                                                       abort_flag));
+            float sv[64];
+            ok = ok && __all_sync(0xffffffffu,
+                                  mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            tmem_ld32(tmem + lane_base + S_COL + sb * NK, *reinterpret_cast<float(*)[32]>(sv));
+            tmem_ld32(tmem + lane_base + S_COL + sb * NK + 32, *reinterpret_cast<float(*)[32]>(sv + 32));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->sempty[sb]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                sv[j] = ((vm_lo >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
+                sv[32 + j] = ((vm_hi >> j) & 1u) ? sv[32 + j] * p.scale_log2 : -INFINITY;
+            }
             float mx[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] = ((vmask >> j) & 1u) ? sv[j] * p.scale_log2 : -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(sv[2 * j], sv[2 * j + 1]);
+            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(fmaxf(sv[4 * j], sv[4 * j + 1]), fmaxf(sv[4 * j + 2], sv[4 * j + 3]));
 #pragma unroll
             for (int w2 = 8; w2 >= 1; w2 >>= 1)
 #pragma unroll
                 for (int j = 0; j < w2; ++j) mx[j] = fmaxf(mx[j], mx[j + w2]);
-            float* xb = xbuf + par * 2 * H;
-            xb[half * H + h] = mx[0];
-            if (lane == 0) flag[par * 8 + sw] = ok ? 1 : 0;
-            named_bar_sync(pair_bar, 64);
-            ok = ok && flag[par * 8 + (sw ^ 4)] != 0;        // the same in both warps of the pair
-            if (!ok) break;
-            const float mc = fmaxf(mx[0], xb[(half ^ 1) * H + h]);
-            float alpha = 1.f;
+            const float mc = mx[0];
+            // the running maximum after chunk c - 1 (the other group's chunk)
+            float m_prev = -INFINITY;
+            if (c > 0) {
+                bool got = true;
+                if (lane == 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    for (uint32_t it = 0; ld_acquire_cta(&bars->mdone[quarter]) < c - 1; ++it) {
+                        if ((it & 63u) == 63u) {
+                            if (*abort_flag) { got = false; break; }
+                            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                                record_error(p.err, DEV_ERR_TIMEOUT_PEER);
+                                *abort_flag = 1;
+                                got = false;
+                                break;
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                __syncwarp();                       // orders lane 0's acquire before the other lanes' reads
+                m_prev = ((volatile float*)mpub)[((c - 1) & 1) * H + h];
+            }
+            float m_new = m_prev, alpha = 1.f;
             if (mc > -INFINITY) {
-                if (m_run == -INFINITY) {
-                    m_run = mc;
-                } else if (mc > m_run + RESCALE_LOG2) {
-                    alpha = exp2f(m_run - mc);
-                    l_run *= alpha;
-                    m_run = mc;
+                if (m_prev == -INFINITY) {
+                    m_new = mc;
+                } else if (mc > m_prev + RESCALE_LOG2) {
+                    alpha = exp2f(m_prev - mc);
+                    m_new = mc;
                 }
             }
-            uint32_t pk[16];
-            float ls[8];
-            // exp2 of (score - running max): at most 2^8 (lazy rescale); -inf for
-            // unused keys, which ex2 maps to +0
-            const float mr = m_run == -INFINITY ? 0.f : m_run;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const __nv_bfloat162 pa = __floats2bfloat162_rn(fast_exp2(sv[4 * j] - mr), fast_exp2(sv[4 * j + 1] - mr));
-                const __nv_bfloat162 pb2 = __floats2bfloat162_rn(fast_exp2(sv[4 * j + 2] - mr), fast_exp2(sv[4 * j + 3] - mr));
-                ls[j] = (__low2float(pa) + __high2float(pa)) + (__low2float(pb2) + __high2float(pb2));
-                pk[2 * j] = *(const uint32_t*)&pa;
-                pk[2 * j + 1] = *(const uint32_t*)&pb2;
+            ((volatile float*)mpub)[(c & 1) * H + h] = m_new;
+            __syncwarp();                           // every lane's value is written before lane 0 publishes
+            if (lane == 0) st_release_cta(&bars->mdone[quarter], c);
+            if (m_new != m_own) {
+                l_own = m_own == -INFINITY ? 0.f : l_own * exp2f(m_own - m_new);
+                m_own = m_new;
             }
+            // the slot's previous P has been consumed by the value CTA's MMA
+            const int pb = c % PSLOTS, pu = c / PSLOTS;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&bars->pempty[pb], (pu & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag));
+            if (!ok) break;
+            // exp2 of (score - running max): at most 2^8 (lazy rescale); -inf for
+            // unused keys, which ex2 maps to +0.  P row h (128 B, 128-B-swizzled
+            // K-major tile) and the head's rescale factor: 128 x 128 + 128 x 4
+            // bytes per chunk, the count the value CTA expects on pfull[pb]
+            const float mr = m_new == -INFINITY ? 0.f : m_new;
+            const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
+            const uint32_t prow = peer_pbuf + (uint32_t)(pb * PBYTES + (h >> 3) * 1024);
+            float ls[8];
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8) {            // 16-byte piece q8: keys 8 q8 .. 8 q8 + 7
+                uint32_t pk[4];
+                float s2 = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 pr = __floats2bfloat162_rn(fast_exp2(sv[8 * q8 + 2 * e] - mr),
+                                                                    fast_exp2(sv[8 * q8 + 2 * e + 1] - mr));
+                    s2 += __low2float(pr) + __high2float(pr);
+                    pk[e] = *(const uint32_t*)&pr;
+                }
+                ls[q8] = s2;
+                st_async_v4(prow + sw128(h & 7, q8), pk[0], pk[1], pk[2], pk[3], rbar);
+            }
+            st_async_b32(peer_abuf + (uint32_t)(pb * ABYTES + h * 4), __float_as_uint(alpha), rbar);
 #pragma unroll
             for (int w2 = 4; w2 >= 1; w2 >>= 1)
 #pragma unroll
                 for (int j = 0; j < w2; ++j) ls[j] += ls[j + w2];
-            l_run += ls[0];
-            // P row h, keys [32 half, +32) (64 B, 128-B-swizzled K-major tile)
-            // and, from half 0, the head's rescale factor: 256 x 64 + 128 x 4
-            // bytes per chunk, the count the value CTA expects on pfull[pb]
-            const uint32_t rbar = mapa_shared(smem_u32(&bars->pfull[pb]), peer);
-            const uint32_t prow = peer_pbuf + (uint32_t)(pb * PBYTES + (h >> 3) * 1024);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                st_async_v4(prow + sw128(h & 7, 4 * half + jj), pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2],
-                            pk[4 * jj + 3], rbar);
-            if (half == 0) st_async_b32(peer_abuf + (uint32_t)(pb * ABYTES + h * 4), __float_as_uint(alpha), rbar);
+            l_own += ls[0];
         }
-        // final statistics -> value CTA: running max (same in both halves) and
-        // the sum of the two halves' running sums
-        if (ok) {
-            float* xb = xbuf + (w.nchunks & 1) * 2 * H;
-            xb[half * H + h] = l_run;
-            named_bar_sync(pair_bar, 64);
-            if (half == 0) {
-                sbuf[h] = m_run;
-                sbuf[H + h] = l_run + xb[H + h];
-            }
+        // final statistics -> value CTA: the last chunk's running maximum and
+        // the two groups' sums brought to it.  Every softmax warp reaches the
+        // barrier below (the loop has no unbounded wait), aborted or not.
+        float* gstat = xbuf + 2 * H;                          // [2][H]: group 1's (m, l)
+        if (grp == 1) {
+            gstat[h] = m_own;
+            gstat[H + h] = l_own;
+        }
+        named_bar_sync(1, 256);
+        if (grp == 0 && ok && !*abort_flag) {
+            const float m1 = gstat[h], l1 = gstat[H + h];
+            const float mf = fmaxf(m_own, m1);        // the last chunk's maximum: the largest one used
+            const float l0s = m_own == -INFINITY ? 0.f : l_own * exp2f(m_own - mf);
+            const float l1s = m1 == -INFINITY ? 0.f : l1 * exp2f(m1 - mf);
+            sbuf[h] = mf;
+            sbuf[H + h] = l0s + l1s;
         }
         fence_proxy_async_smem();
         __syncwarp();

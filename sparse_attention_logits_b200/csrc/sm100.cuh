@@ -402,6 +402,18 @@ __device__ __forceinline__ void mma_commit_multicast(uint64_t* bar, uint16_t cta
         : "memory");
 }
 
+// Shared-memory flag of this CTA: load with acquire / store with release at
+// CTA scope (publishing data written before the store to a thread that sees
+// the stored value).
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
 // Hardware named barrier `id` (1..15) over `count` threads (a multiple of 32).
 // Unbounded: every thread of the group must reach it on every path.
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
