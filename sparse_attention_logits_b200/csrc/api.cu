@@ -334,7 +334,8 @@ dsa_status_t sparse_attention(const char* name, const void* q, const void* kv, d
         return fail(DSA_ERR_INVALID_ARG, "%s: bad sizes", name);
     const bool raw = window + n_sink > 0;                   // a segment of raw rows
     if ((int64_t)batch * ctx_len >= ((int64_t)1 << 31) - 2 ||
-        (raw && (int64_t)batch * x.len2 >= ((int64_t)1 << 31) - 2))
+        (raw && (int64_t)batch * x.len2 >= ((int64_t)1 << 31) - 2) ||
+        (page_table && (int64_t)num_pages * page_size >= ((int64_t)1 << 31) - 2))
         return fail(DSA_ERR_UNSUPPORTED, "%s: a cache holds more than 2^31 - 2 rows", name);
     if (rows == 0) return DSA_OK;
     if (!q || !kv || !row_batch || !out || !lse || (k > 0 && !idx && !x.row_last))

@@ -28,6 +28,7 @@ using namespace sm100;
 namespace {
 
 constexpr int TOPK_THREADS = 1024;
+static_assert(TOPK_THREADS == 32 * 32, "the bin search sums over exactly 32 warps");
 constexpr int NBINS = 2048;                    // 11-bit digits
 constexpr int SLICE_CAP = 40960;               // keys per CTA kept in shared memory (160 KB)
 constexpr int MAX_PASSES = 3;                  // 11 + 10 + 10 bits: the range is exact after three passes
@@ -45,35 +46,6 @@ constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 
 constexpr int SMEM_ROUND = 128;
 static_assert(SMEM_FIXED % 16 == 0, "the key slice must start 16-byte aligned");
 static_assert((2 * NBINS * 4) % 8 == 0 && NBINS % 2 == 0, "cluster histograms: 8-byte aligned pairs");
-
-// Exclusive scan over the CTA (1024 threads = 32 warps); also returns the total.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_sums, uint32_t* total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_sums[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t s = warp_sums[lane];
-        uint32_t inc = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-        }
-        warp_sums[lane] = inc - s;
-        if (lane == 31) warp_sums[32] = inc;
-    }
-    __syncthreads();
-    uint32_t r = warp_sums[warp] + x - v;
-    *total = warp_sums[32];
-    __syncthreads();
-    return r;
-}
 
 template <int CL>
 __device__ __forceinline__ void cl_sync() {
@@ -220,14 +192,17 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     // (cnt4), so that every walk below reads 16 bytes per lane
     const int cnt4 = (cnt + 3) & ~3;
     for (int i = cnt + tid; i < cnt4; i += TOPK_THREADS) keys[i] = keys[0];
-    if (tid == 0) {
-        uint32_t a = 0xFFFFFFFFu, b = 0u;
-        for (int w2 = 0; w2 < TOPK_THREADS / 32; ++w2) {
-            a = min(a, merged[w2]);
-            b = max(b, merged[32 + w2]);
+    if (tid < 32) {                              // this CTA's key range: warp 0 reduces the 32 warps' ranges
+        uint32_t a = merged[tid], b = merged[32 + tid];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+            b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
         }
-        cta_counts[2] = a;
-        cta_counts[3] = b;
+        if (tid == 0) {
+            cta_counts[2] = a;
+            cta_counts[3] = b;
+        }
     }
     // every CTA's key range published, its cluster histograms zeroed
     cl_sync<CL>();
@@ -238,15 +213,27 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     // range's width), finds the bucket that holds the remaining-th largest
     // candidate and shrinks [lo, hi] to it.  Bucketing by the actual range
     // spreads keys over the bins even when all scores share one exponent.
-    if (tid == 0) {
+    if (tid < 32) {                              // the cluster's key range: lane r reads CTA r's, in parallel
         uint32_t a = 0xFFFFFFFFu, b = 0u;
-        for (int r = 0; r < CL; ++r) {
-            const uint32_t base = CL > 1 ? mapa_shared(smem_u32(cta_counts), (uint32_t)r) : smem_u32(cta_counts);
-            a = min(a, CL > 1 ? ld_cluster_u32(base + 8) : cta_counts[2]);
-            b = max(b, CL > 1 ? ld_cluster_u32(base + 12) : cta_counts[3]);
+        if (tid < CL) {
+            if (CL > 1) {
+                const uint32_t base = mapa_shared(smem_u32(cta_counts), (uint32_t)tid);
+                a = ld_cluster_u32(base + 8);
+                b = ld_cluster_u32(base + 12);
+            } else {
+                a = cta_counts[2];
+                b = cta_counts[3];
+            }
         }
-        shared_res[4] = a;
-        shared_res[5] = b;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+            b = max(b, __shfl_xor_sync(0xffffffffu, b, o));
+        }
+        if (tid == 0) {
+            shared_res[4] = a;
+            shared_res[5] = b;
+        }
     }
     __syncthreads();
     uint32_t lo_key = shared_res[4], hi_key = shared_res[5], remaining = (uint32_t)k;
@@ -285,16 +272,26 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
             h0 = hist[2 * tid];
             h1 = hist[2 * tid + 1];
         }
-        // keys in bins above each thread's pair: scan over reversed thread order
-        uint32_t tot;
-        merged[TOPK_THREADS - 1 - tid] = h0 + h1;
+        // keys in bins above each thread's pair (the pairs of higher
+        // threads): a suffix sum within the warp, then over the 32 warps
+        const int lane = tid & 31, warp = tid >> 5;
+        const uint32_t hs = h0 + h1;
+        uint32_t suf = hs;                       // this lane's pair and the pairs of higher lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += y;
+        }
+        if (lane == 0) warp_sums[warp] = suf;
         __syncthreads();
-        const uint32_t rev = merged[tid];
-        __syncthreads();
-        const uint32_t above_rev = block_excl_scan(rev, warp_sums, &tot);
-        merged[TOPK_THREADS - 1 - tid] = above_rev;
-        __syncthreads();
-        const uint32_t above = merged[tid];
+        const uint32_t wt = warp_sums[lane];
+        uint32_t ws = wt;                        // warps >= lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_down_sync(0xffffffffu, ws, o);
+            if (lane + o < 32) ws += y;
+        }
+        const uint32_t above = __shfl_sync(0xffffffffu, ws - wt, warp) + (suf - hs);
         if (above < remaining && above + h1 >= remaining) {
             shared_res[0] = 2u * tid + 1u;
             shared_res[1] = above;
@@ -319,7 +316,6 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
             const uint32_t n_addr = CL > 1 ? mapa_shared(smem_u32(cand_n), 0u) : smem_u32(cand_n);
             const uint32_t c_addr = CL > 1 ? mapa_shared(smem_u32(cand), 0u) : smem_u32(cand);
             const uint32_t s_addr = CL > 1 ? mapa_shared(smem_u32(cand_src), 0u) : smem_u32(cand_src);
-            const int lane = tid & 31, warp = tid >> 5;
             {
                 // this CTA's keys in bins above the chosen one: all of them are taken
                 uint32_t a = (2u * tid > bin ? hist[2 * tid] : 0u) + (2u * tid + 1u > bin ? hist[2 * tid + 1] : 0u);

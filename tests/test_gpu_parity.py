@@ -85,6 +85,19 @@ def test_topk_bit_exact_on_given_scores(cuda_device, rows, L, k, seed):
         assert np.array_equal(np.sort(got[r][got[r] >= 0]), np.sort(ref[r][ref[r] >= 0])), f"row {r}"
 
 
+def test_topk_rows_not_16_byte_aligned(cuda_device):
+    # ld = L + 3: most rows start off a 16-byte boundary, so every CTA of a
+    # row's cluster takes the scalar load path (L = 100,001 keys: 8 CTAs per row)
+    rows, L, k = 4, 100001, 2048
+    x = workloads.synthetic_scores(rows, L + 3, seed=8)
+    pos = torch.tensor([L - 1, L - 2, 70000, 5000], dtype=torch.int32)
+    got = dsa.topk(x.to(cuda_device), pos.to(cuda_device), k, ctx_len=L).cpu().numpy()
+    check_sorted_unique(got, pos.numpy() + 1)
+    ref = oracle.topk(x[:, :L], pos, k)
+    for r in range(rows):
+        assert np.array_equal(got[r][got[r] >= 0], np.sort(ref[r][ref[r] >= 0])), f"row {r}"
+
+
 def test_topk_edge_cases(cuda_device):
     L = 4100
     rows = []
