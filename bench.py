@@ -475,6 +475,10 @@ def run_kernel_only(args):
     if args.kernel_only == "prepare":
         return run_prepare_only(dsa, workloads, device, args)
     wl = workloads.BY_NAME[args.workload]
+    if args.prefill_tokens and wl.mode == "prefill":
+        # a shorter prompt of the same prefill workload (profiler captures
+        # that collect more than kernel durations stay a few GB in size)
+        wl = wl.with_(name=f"{wl.name}_T{args.prefill_tokens}", rows=args.prefill_tokens, ctx=args.prefill_tokens)
     inp = workloads.generate(wl, device=device, seed=0)
     step = DecodeStep(dsa, wl, inp, device)
     step.run()
@@ -1089,6 +1093,8 @@ def main(argv=None):
     ap.add_argument("--no-tiny", dest="tiny", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--prep-tokens", type=int, default=64, help="tokens of --kernel-only prepare")
+    ap.add_argument("--prefill-tokens", type=int, default=0,
+                    help="--kernel-only on the prefill workload: use a prompt of this many tokens")
     ap.add_argument("--kernel-only", choices=["indexer", "topk", "mla", "prepare"], default=None,
                     help="time one kernel of the step alone (for profiler captures)")
     args = ap.parse_args(argv)

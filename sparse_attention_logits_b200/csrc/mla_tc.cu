@@ -278,11 +278,42 @@ __device__ __forceinline__ void gather_rows(const MlaParams& p, const Work& w, u
     }
 }
 
+// Dense mode (every key of a contiguous range, no index list): the 64 keys
+// of a chunk are consecutive cache rows, so one thread loads them with TMA
+// tiles of 64 rows x 64 dims straight into the 128-B-swizzled stage layout
+// (NB tiles per chunk) instead of gathering them row by row.  Rows past the
+// cache are zero-filled by the tensor map; rows past the row's last visible
+// key are masked by the softmax (their P is 0).  Same stage ring and
+// barriers as gather_rows; each stage's full barrier counts the bytes.
+template <int NB, int NST>
+__device__ __forceinline__ void dense_loads(const MlaParams& p, const Work& w, const CUtensorMap* kv_map,
+                                            uint8_t* gbuf, Bars* bars, volatile int* abort_flag) {
+    constexpr bool Q_IN_RING = NB == KBLK;               // score CTA
+    const int row_base = w.b_ok ? w.b * p.ctx + w.slot0 : 0;
+    int issued = 0;
+    for (int c = 0; c < w.nchunks; ++c) {
+        const int st = c % NST;
+        const uint32_t par = (uint32_t)((c / NST) & 1) ^ ((Q_IN_RING && st > 0) ? 0u : 1u);
+        if (!mbar_wait(&bars->empty[st], par, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
+        mbar_arrive_expect_tx(&bars->full[st], NB * NK * 128);
+        uint8_t* base = gbuf + (size_t)st * KSTAGE;
+        for (int b = 0; b < NB; ++b) tma_load_2d(base + b * (NK * 128), kv_map, b * 64, row_base + c * NK, &bars->full[st]);
+        ++issued;
+    }
+    // after an abort, let the tiles already requested land before the CTA exits
+    if (*abort_flag)
+        for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
+            mbar_wait(&bars->full[j % NST], (j / NST) & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr);
+}
+
 }  // namespace
 
-template <bool EXT>
+// EXT: window / sink / dense slots; DENSE (implies EXT): every key of a
+// contiguous range, loaded with TMA tiles (kv_map) instead of row gathers.
+template <bool EXT, bool DENSE>
 __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constant__ CUtensorMap q_map,
                                                           const __grid_constant__ CUtensorMap o_map,
+                                                          const __grid_constant__ CUtensorMap kv_map,
                                                           const MlaParams p) {
     pdl_wait();                     // the indices of the previous kernel are visible from here on
     pdl_launch_dependents();
@@ -306,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < SSTAGES; ++i) {
-            mbar_init(&bars->full[i], PWARPS * 32);
+            mbar_init(&bars->full[i], DENSE ? 1 : PWARPS * 32);
             mbar_init(&bars->empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -366,8 +397,16 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         // together); the copy loop then walks the warp's rows with consecutive
         // lanes on consecutive 16-byte pieces of a row.  Several warps are
         // used because each keeps only a bounded number of copies in flight.
-        if (role == 0) gather_rows<KBLK, EXT, SSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
-        else gather_rows<VBLK, EXT, VSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
+        if (DENSE) {
+            if (warp == 0 && elect_one()) {
+                if (role == 0) dense_loads<KBLK, SSTAGES>(p, w, &kv_map, gbuf, bars, abort_flag);
+                else dense_loads<VBLK, VSTAGES>(p, w, &kv_map, gbuf, bars, abort_flag);
+            }
+        } else if (role == 0) {
+            gather_rows<KBLK, EXT, SSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
+        } else {
+            gather_rows<VBLK, EXT, VSTAGES>(p, w, gbuf, bars, warp, lane, abort_flag);
+        }
     } else if (warp < SWARP0 + 8) {
       regs_inc<REGS_SOFTMAX>();
       if (role == 0) {
@@ -894,9 +933,9 @@ int max_active_quads() {
         cfg.numAttrs = 1;
         int n = 0;
         // both kernel variants have the same shape; the attribute must be set on the one queried
-        if (cudaFuncSetAttribute(mla_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM) !=
+        if (cudaFuncSetAttribute(mla_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM) !=
                 cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<false>, &cfg) != cudaSuccess) {
+            cudaOccupancyMaxActiveClusters(&n, mla_tc_kernel<false, false>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -952,7 +991,10 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     p.part_o = nullptr;
     p.part_lse = nullptr;
     const bool ext = p.window > 0 || p.n_sink > 0 || !p.idx;
-    auto kern = ext ? mla_tc_kernel<true> : mla_tc_kernel<false>;
+    // every key of a contiguous cache range (no index list, window, sink or
+    // page table): TMA tiles instead of row gathers
+    const bool dense = !p.idx && p.window == 0 && p.n_sink == 0 && !page_table;
+    auto kern = dense ? mla_tc_kernel<true, true> : ext ? mla_tc_kernel<true, false> : mla_tc_kernel<false, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)MLA_SMEM);
     if (e != cudaSuccess) return e;
     // Two splits per row: merge them inside a 4-CTA cluster when all rows'
@@ -968,8 +1010,11 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     // Q as [rows*128, 576] bf16 in boxes of 128 heads x 64 dims; the output as
     // [rows*128, 512] bf16 in boxes of 32 heads x 64 columns, or the partials
     // as [rows*splits*128, 512] fp32 in boxes of 32 heads x 32 columns
-    CUtensorMap q_map, o_map;
+    CUtensorMap q_map, o_map, kv_map;
     bool ok = make_map_sw128(&q_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DK, (uint64_t)rows * H, 64, H);
+    // dense mode: the cache as [batch * ctx, 576] in tiles of 64 rows x 64 dims
+    kv_map = q_map;
+    if (dense) ok = ok && make_map_sw128(&kv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kv, DK, (uint64_t)batch * ctx_len, 64, NK);
     if (p.splits == 1 || p.fuse2)
         ok = ok && make_map_sw128(&o_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, DV, (uint64_t)rows * H, 64, 32);
     else
@@ -989,7 +1034,7 @@ cudaError_t launch_mla_tc(const Launch& L, const void* q, const void* kv, const 
     attr[1] = pdl_attr();
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, kern, q_map, o_map, p);
+    e = cudaLaunchKernelEx(&cfg, kern, q_map, o_map, kv_map, p);
     count_launch();
     if (e != cudaSuccess) return e;
     if (p.splits > 1 && !p.fuse2) {
