@@ -37,6 +37,9 @@ constexpr int CAND_CAP = 1024;                 // candidates ranked directly aft
 // candidate buffer, candidates' source CTAs, per-CTA counts (rank 0)
 constexpr int MAX_CL = 16;                     // CTAs per row (16 needs the non-portable cluster size)
 constexpr int SMEM_FIXED = ((2 + MAX_PASSES) * NBINS + 64 + 32 + 2 * CAND_CAP + 32 + 3 * MAX_CL + 16) * 4;
+// the per-pass range totals (MAX_PASSES x MAX_CL words) fit in the last 16 + 32 words of the fixed part
+static_assert((2 + MAX_PASSES) * NBINS + 40 + 8 + 16 + 2 * CAND_CAP + 3 * MAX_CL + MAX_PASSES * MAX_CL <=
+              SMEM_FIXED / 4, "fixed shared-memory layout");
 // Alignment of the vector accesses, by construction: the base is rounded up
 // to 128 B in the kernel (the launch reserves exactly that rounding room,
 // SMEM_ROUND), the key slice starts SMEM_FIXED bytes after it, and every
@@ -98,7 +101,8 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* tk_smem = (uint32_t*)(((uintptr_t)tk_smem_raw + SMEM_ROUND - 1) & ~(uintptr_t)(SMEM_ROUND - 1));
     uint32_t* hist = tk_smem;                    // [NBINS]   this CTA's histogram
     uint32_t* merged = hist + NBINS;             // [NBINS]   scratch for the suffix scan
-    uint32_t* cl_hist = merged + NBINS;          // [MAX_PASSES][NBINS] cluster-wide histograms (rank 0 holds them)
+    uint32_t* cl_hist = merged + NBINS;          // [MAX_PASSES][NBINS] cluster-wide histograms: CTA r holds the
+                                                 // merged counts of its own range of bins (NBINS / CL of them)
     uint32_t* warp_sums = cl_hist + MAX_PASSES * NBINS;   // [33]
     uint32_t* shared_res = warp_sums + 40;       // digit, count above
     uint32_t* cta_counts = shared_res + 8;       // gt, eq of this CTA (read by peers), key range, and [4..7]: the
@@ -107,6 +111,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
     uint32_t* cand = cta_counts + 16;            // [CAND_CAP] candidate keys (rank 0's is used)
     uint32_t* cand_src = cand + CAND_CAP;        // [CAND_CAP] the CTA each candidate comes from (rank 0's)
     uint32_t* cta_cnt = cand_src + CAND_CAP;     // [3][MAX_CL] per-CTA keys above the bin, candidates > T, == T (rank 0's)
+    uint32_t* rtot = cta_cnt + 3 * MAX_CL;       // [MAX_PASSES][MAX_CL] cluster-wide keys in each CTA's bin range
     uint32_t* keys = tk_smem + (SMEM_FIXED / 4); // [slice]
 
     pdl_wait();                     // the scores of the previous kernel are visible from here on
@@ -183,8 +188,10 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
         merged[tid >> 5] = kmin;
         merged[32 + (tid >> 5)] = kmax;
     }
-    if (CL > 1)
+    if (CL > 1) {
         for (int i = tid; i < MAX_PASSES * NBINS; i += TOPK_THREADS) cl_hist[i] = 0u;
+        if (tid < MAX_PASSES * MAX_CL) rtot[tid] = 0u;
+    }
     if (tid == 0) *cand_n = 0u;
     if (tid < 3 * MAX_CL) cta_cnt[tid] = 0u;
     __syncthreads();
@@ -256,25 +263,55 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
                 if (i + u < cnt && kq[u] >= lo_key && kq[u] <= hi_key) atomicAdd(&hist[(kq[u] - lo_key) >> sh], 1u);
         }
         __syncthreads();
-        // cluster-wide histogram: thread t owns bins 2t and 2t+1
-        uint32_t h0, h1;
+        // cluster-wide histogram: thread t owns bins 2t and 2t+1.  With a
+        // cluster, CTA r holds the merged counts of bins [r OWN, (r+1) OWN):
+        // every CTA adds its counts into the owner of each range, and its
+        // count per range into every CTA's range totals, so one cluster
+        // barrier suffices and no CTA is the target of all the traffic.  After
+        // it, every CTA finds (from the totals) the range that holds the
+        // remaining-th largest key and reads only that range's merged bins.
+        const int lane = tid & 31, warp = tid >> 5;
+        uint32_t h0, h1, above_r = 0u;
         if (CL > 1) {
-            // a fresh, zeroed buffer per pass: no CTA can add into a buffer
-            // another is still reading
-            const uint32_t lead = mapa_shared(smem_u32(cl_hist + pass * NBINS + 2 * tid), 0u);
-            if (hist[2 * tid]) red_cluster_add(lead, hist[2 * tid]);
-            if (hist[2 * tid + 1]) red_cluster_add(lead + 4, hist[2 * tid + 1]);
+            constexpr int OWN = NBINS / CL;                  // >= 128: a warp's 64 bins lie in one range
+            static_assert(NBINS % CL == 0 && OWN % 64 == 0, "bin ranges");
+            uint32_t* ch = cl_hist + pass * NBINS;
+            const uint32_t owner = (uint32_t)(64 * warp) / OWN;
+            const uint32_t dst = mapa_shared(smem_u32(ch + 2 * tid), owner);
+            if (hist[2 * tid]) red_cluster_add(dst, hist[2 * tid]);
+            if (hist[2 * tid + 1]) red_cluster_add(dst + 4, hist[2 * tid + 1]);
+            uint32_t wsum = hist[2 * tid] + hist[2 * tid + 1];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+            if (lane < CL && wsum) red_cluster_add(mapa_shared(smem_u32(rtot + pass * MAX_CL + owner), (uint32_t)lane), wsum);
             cl_sync<CL>();                       // all additions landed
-            const uint2 v = ld_cluster_v2(lead);
-            h0 = v.x;
-            h1 = v.y;
+            // the range R that holds the remaining-th key from the top (the
+            // same decision in every warp and CTA): keys in ranges above each
+            // range by a suffix sum over the lanes
+            const uint32_t tq = lane < CL ? rtot[pass * MAX_CL + lane] : 0u;
+            uint32_t sq = tq;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_down_sync(0xffffffffu, sq, o);
+                if (lane + o < 32) sq += y;
+            }
+            const uint32_t abv = sq - tq;
+            const uint32_t hit = __ballot_sync(0xffffffffu, lane < CL && abv < remaining && remaining <= sq);
+            const int R = hit ? __ffs(hit) - 1 : 0;
+            above_r = __shfl_sync(0xffffffffu, abv, R);
+            h0 = h1 = 0u;
+            if (2 * tid >= R * OWN && 2 * tid < (R + 1) * OWN) {
+                const uint2 v = ld_cluster_v2(mapa_shared(smem_u32(ch + 2 * tid), (uint32_t)R));
+                h0 = v.x;
+                h1 = v.y;
+            }
         } else {
             h0 = hist[2 * tid];
             h1 = hist[2 * tid + 1];
         }
         // keys in bins above each thread's pair (the pairs of higher
-        // threads): a suffix sum within the warp, then over the 32 warps
-        const int lane = tid & 31, warp = tid >> 5;
+        // threads, plus the ranges above R): a suffix sum within the warp,
+        // then over the 32 warps
         const uint32_t hs = h0 + h1;
         uint32_t suf = hs;                       // this lane's pair and the pairs of higher lanes
 #pragma unroll
@@ -291,7 +328,7 @@ __global__ void __launch_bounds__(TOPK_THREADS, 1) topk_cluster_kernel(
             const uint32_t y = __shfl_down_sync(0xffffffffu, ws, o);
             if (lane + o < 32) ws += y;
         }
-        const uint32_t above = __shfl_sync(0xffffffffu, ws - wt, warp) + (suf - hs);
+        const uint32_t above = above_r + __shfl_sync(0xffffffffu, ws - wt, warp) + (suf - hs);
         if (above < remaining && above + h1 >= remaining) {
             shared_res[0] = 2u * tid + 1u;
             shared_res[1] = above;
