@@ -93,7 +93,7 @@ static_assert(ABUF_OFF + PSLOTS * ABYTES <= REGION, "value CTA layout");
 constexpr int SBUF_OFF = REGION;
 constexpr int XBUF_OFF = SBUF_OFF + SBYTES;
 constexpr int BARS_OFF = XBUF_OFF + 4 * H * 4;
-constexpr int S_COL = 320;          // score CTA: Q in TMEM columns [0, 288), S buffers at 320, 384
+constexpr int S_COL = 320;          // score CTA: Q in TMEM columns [0, 288), S buffers at 320, 384, 448
 constexpr int TMEM_COLS = 512;
 constexpr float RESCALE_LOG2 = 8.f; // lazy rescale threshold (P <= 2^8 between rescales)
 constexpr float LN2 = 0.6931471805599453f;
@@ -101,7 +101,7 @@ constexpr float LN2 = 0.6931471805599453f;
 struct Bars {                       // same offset in both CTAs of a cluster
     uint64_t full[SSTAGES];         // a stage's gathered rows have landed (cp.async arrivals)
     uint64_t empty[SSTAGES];        // the MMA is done reading a stage (score stages 1-2: first, Q has left)
-    uint64_t sfull[2], sempty[2], pempty[PSLOTS], qready, statready, statack;
+    uint64_t sfull[3], sempty[3], pempty[PSLOTS], qready, statready, statack;
     // value CTA: P slot landed / rescaled, PV of chunk c done (ring of PSLOTS, so
     // that a parity wait never aliases), all PV done, final statistics landed
     uint64_t pfull[PSLOTS], ready[PSLOTS], odone[PSLOTS], ofinal, statfull;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             mbar_init(&bars->full[i], DENSE ? 1 : PWARPS * 32);
             mbar_init(&bars->empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 3; ++i) {
             mbar_init(&bars->sfull[i], 1);
             mbar_init(&bars->sempty[i], 4);     // the softmax group of this S buffer
         }
@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
         int s_lo = grp < w.nchunks ? slot_index<EXT>(p, w, w.slot0 + grp * NK + lane) : -1;
         int s_hi = grp < w.nchunks ? slot_index<EXT>(p, w, w.slot0 + grp * NK + 32 + lane) : -1;
         for (int c = grp; c < w.nchunks; c += 2) {
-            const int sb = grp;
+            const int sb = c % 3;
             const int slot0 = w.slot0 + c * NK;
             const uint32_t vm_lo = __ballot_sync(0xffffffffu, w.b_ok && s_lo >= 0 && s_lo < slot_limit<EXT>(p, slot0 + lane));
             const uint32_t vm_hi =
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             }
             float sv[64];
             ok = ok && __all_sync(0xffffffffu,
-                                  mbar_wait(&bars->sfull[sb], (c >> 1) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag));
+                                  mbar_wait(&bars->sfull[sb], (c / 3) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag));
             if (!ok) break;
             tc_fence_after();
             tmem_ld32(tmem + lane_base + S_COL + sb * NK, *reinterpret_cast<float(*)[32]>(sv));
@@ -809,8 +809,8 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
                     mbar_arrive(&bars->empty[2]);
                 }
                 for (int c = 0; c < w.nchunks && ok; ++c) {
-                    const int st = c % SSTAGES, sb = c & 1;
-                    ok = mbar_wait(&bars->sempty[sb], ((c >> 1) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag) &&
+                    const int st = c % SSTAGES, sb = c % 3;
+                    ok = mbar_wait(&bars->sempty[sb], ((c / 3) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag) &&
                          mbar_wait(&bars->full[st], (c / SSTAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                     if (!ok) break;
                     fence_proxy_async_smem();
