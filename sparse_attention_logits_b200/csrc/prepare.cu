@@ -10,31 +10,37 @@
 //   k_I[t, :]    = RoPE( W_k . h[t] )  -> key cache row slot[t] (bf16, or
 //                  fp8 e4m3 / fp4 e2m1 codes with one fp32 scale per row)
 //
+// prepare_norm_kernel -- one warp per token: the token's sum of squares of
+// c_q (fp32) gives 1/RMS, and c_q * gain is rounded once to bf16 into the
+// workspace; every query tile then reads that operand as it is, instead of
+// each of them scaling the same latent again.  It also clears the per
+// token-tile arrival counters of the projection kernel.
+//
 // indexer_prepare_kernel -- all three projections in one launch on the
-// tcgen05 tensor cores.  Every CTA computes one tile of 128 tokens x 64
+// tcgen05 tensor cores, launched right after the norm kernel (programmatic
+// dependent launch).  Every CTA computes one tile of 128 tokens x 64
 // features (256 for query tiles when there are many tokens)
 // D = A . B^T (M = 128 tokens, N = 64 or 256 features, K streamed 64 at a time
 // through a 4-stage TMA ring of one or two 64-wide chunks per stage, fp32
 // accumulator in TMEM):
-//   query tiles  A = c_q, B = 64 rows of W_qb.  While a stage is in shared
-//                memory the four epilogue warps add up each token's squares
-//                (the RMS) and multiply the stage by the norm gain in place;
-//                1/RMS is a per-token factor applied in the epilogue, which
-//                also turns the rotary pairs and stores bf16 q_I.
+//   query tiles  A = the scaled latent, B = rows of W_qb.  The weight boxes of
+//                the first ring's worth of stages are requested before the
+//                norm kernel has finished (they do not depend on it); the
+//                epilogue multiplies by 1/RMS, turns the rotary pairs (the
+//                tile's cosine / sine rows are staged in shared memory while
+//                the main loop runs) and stores bf16 q_I.
 //   key/weight tiles  A = h, B = 64 rows of [W_k ; W_w], with K split over S
 //                CTAs when the token count is small (so that the long
 //                d_model reduction is spread over as many SMs as the query
 //                tiles use).  Each writes its fp32 partial tile to the
-//                workspace.
+//                workspace and counts itself in its token tile's counter; the
+//                last of a token tile's key / weight CTAs adds the partials
+//                up in split order (the result does not depend on
+//                scheduling), writes the head weights, turns the key's
+//                rotary pairs and writes the key row into the cache.
 // Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and
-// TMEM owner), warps 4-7 norm pass and epilogue (warp 4+q owns TMEM lanes
-// 32q .. 32q+31 = tokens of the tile).  The norm gain is copied to shared
-// memory once per CTA.
-//
-// prepare_finish_kernel -- launched right after (programmatic dependent
-// launch), one warp per token: adds the S partials in split order (the
-// result does not depend on scheduling), writes the head weights, turns the
-// key's rotary pairs and writes the key row into the cache.
+// TMEM owner), warps 4-7 epilogue (warp 4+q owns TMEM lanes 32q .. 32q+31 =
+// tokens of the tile).
 //
 // key_append_kernel -- the key-cache write alone for keys that are already
 // projected (for instance compressed CSA keys): one warp per key row, lane l
@@ -63,24 +69,26 @@ constexpr int A_BYTES = PT * PK * 2;            // 16 KB (stage room; a 64-token
 constexpr int PTHREADS = 256;
 constexpr int KDIM = 128;                       // indexer head dim (key row length)
 // Shared-memory layout for a ring of STG stages of NSUB reduction chunks
-// each (A boxes then B boxes): stages, barriers / TMEM address / abort flag,
-// then the norm gain (d_c floats).  Three variants: few tokens (the grid fits
-// on the SMs at one CTA each): query tiles 64 wide, two chunks per stage (256
-// contiguous bytes of every weight row per stage, half the hand-offs); many
-// tokens: query tiles 256 wide, one chunk per stage (each c_q tile feeds four
-// times the features: half the bytes an SM takes in per multiply-add); in
-// between: 64-wide tiles, one chunk per stage, two CTAs per SM.
+// each (A boxes then B boxes): stages, barriers / TMEM address / flags, then
+// (query tiles with rotary columns, when it fits) the tile's cosine and sine
+// rows, [d_rope / 2][128 tokens] each.  Three variants: few tokens (the grid
+// fits on the SMs at one CTA each): query tiles 64 wide, two chunks per
+// stage (256 contiguous bytes of every weight row per stage, half the
+// hand-offs); many tokens: query tiles 256 wide, one chunk per stage (each
+// latent tile feeds four times the features: half the bytes an SM takes in
+// per multiply-add); in between: 64-wide tiles, one chunk per stage, two
+// CTAs per SM (no staged rotary rows).
 template <int STG, int NSUB, int QN>
 struct Ring {
     static constexpr int B_ROOM = QN * PK * 2;                                 // one B box (query tiles are QN wide)
     static constexpr size_t SLOT = (size_t)NSUB * (A_BYTES + B_ROOM);          // one stage: NSUB A boxes, NSUB B boxes
     static constexpr size_t BAR_OFF = (size_t)STG * SLOT;
-    static constexpr size_t GAIN_OFF = (BAR_OFF + (3 * STG + 1) * 8 + 16 + 15) & ~(size_t)15;
-    static constexpr size_t SMEM_BASE = 1024 + GAIN_OFF;
-    static_assert(GAIN_OFF % 16 == 0, "gain alignment");
+    static constexpr size_t TAB_OFF = (BAR_OFF + (2 * STG + 2) * 8 + 16 + 15) & ~(size_t)15;
+    static constexpr size_t SMEM_BASE = 1024 + TAB_OFF;
+    static_assert(TAB_OFF % 16 == 0, "table alignment");
 };
 constexpr size_t SMEM_LIMIT = 227 * 1024;
-constexpr int MAX_DC = 16384;                   // the gain (d_c floats) is held in shared memory
+constexpr int MAX_DC = 16384;
 
 struct KeyOut {
     void* cache;          // [cache_rows, 128] bf16 / [cache_rows, 128] e4m3 / [cache_rows, 64] e2m1 pairs
@@ -91,18 +99,29 @@ struct KeyOut {
     int d_rope, max_pos, fmt;   // fmt: DSA_BF16, DSA_FP8_E4M3 or DSA_FP4_E2M1
 };
 
+struct NormParams {
+    const __nv_bfloat16* c_q;   // [T, d_c]
+    const float* gamma;         // [d_c]
+    __nv_bfloat16* cqn;         // [T, d_c] c_q * gain, rounded once
+    float* inv_rms;             // [T]
+    unsigned* arrivals;         // [n_tt] cleared here
+    float eps;
+    int T, d_c, n_tt;
+};
+
 struct PrepParams {
-    const float* gamma;   // [d_c] norm gain
     const int32_t* pos;   // [T]
     const int64_t* slot;  // [T]
     __nv_bfloat16* q_out; // [T, H, 128]
     float* w_out;         // [T, H]
     float* ws;            // [S][n_tt * 128][kwc] partial sums of the key / weight tiles
+    const float* inv_rms; // [T] (norm kernel)
+    unsigned* arrivals;   // [n_tt] key / weight CTAs done per token tile (cleared by the norm kernel)
     KeyOut ko;
-    float eps;
-    int T, d_c, n_heads;
+    int T, n_heads;
     int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
     int a_bytes;          // bytes of one A box (64 or 128 token rows)
+    int tab;              // query tiles stage their rotary rows in shared memory
     unsigned* err;
 };
 
@@ -158,18 +177,10 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
     return r;
 }
 
-// One warp writes one key row: lane l holds dims 4l .. 4l+3 (binary32);
-// rotary pairs of dims below d_rope turned at position `ps`, then stored at
-// row `row` of the cache in its format.
-__device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, int64_t row, const KeyOut& o) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const int d0 = 4 * lane + 2 * e;
-        if (d0 < o.d_rope) {
-            const int64_t ti = (int64_t)ps * (o.d_rope >> 1) + (d0 >> 1);
-            rope_pair(x[2 * e], x[2 * e + 1], __ldg(o.cos + ti), __ldg(o.sin + ti));
-        }
-    }
+// One warp writes one key row: lane l holds dims 4l .. 4l+3 (binary32),
+// already turned by the rotary pairs; stored at row `row` of the cache in
+// its format.
+__device__ __forceinline__ void write_key_row(float (&x)[4], int lane, int64_t row, const KeyOut& o) {
     if (o.fmt == DSA_BF16) {
         __nv_bfloat162 a = __floats2bfloat162_rn(x[0], x[1]), b = __floats2bfloat162_rn(x[2], x[3]);
         uint2 u;
@@ -196,9 +207,141 @@ __device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, i
     if (lane == 0) o.scale[row] = sc;
 }
 
-__device__ __forceinline__ void bar_epilogue() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The rotary pairs of dims below d_rope of lane l's dims 4l .. 4l+3 turned at
+// position `ps`, then the row written.
+__device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, int64_t row, const KeyOut& o) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        const int d0 = 4 * lane + 2 * e;
+        if (d0 < o.d_rope) {
+            const int64_t ti = (int64_t)ps * (o.d_rope >> 1) + (d0 >> 1);
+            rope_pair(x[2 * e], x[2 * e + 1], __ldg(o.cos + ti), __ldg(o.sin + ti));
+        }
+    }
+    write_key_row(x, lane, row, o);
+}
+
+// The last key / weight CTA of token tile `tt` finishes its keys and
+// weights, `cap` tokens at a time, in the drained ring (`buf`): the S
+// partial sums of each token's 128 key and n_heads weight columns arrive by
+// bulk copies, [S][cap][kwc], while the threads fetch the tokens' slots,
+// positions and cosine / sine rows ([2][d_rope / 2][cap]); then one warp
+// per token adds the partials in split order (the result does not depend on
+// scheduling), writes the weights, turns the key's rotary pairs and writes
+// the key row in the cache's format.
+__device__ __forceinline__ size_t finish_bytes_per_token(const PrepParams& p) {
+    return (size_t)p.S * p.kwc * sizeof(float) + sizeof(int64_t) + sizeof(int) + (size_t)p.ko.d_rope * sizeof(float);
+}
+
+__device__ __forceinline__ void finish_tile(const PrepParams& p, int tt, uint8_t* buf, int cap, uint64_t* bar) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t0 = tt * PT;
+    const int rows = min(PT, p.T - t0);
+    const int half = p.ko.d_rope >> 1;
+    const int kv4 = p.kwc / 4;                                  // float4 per token row
+    float* part = (float*)buf;                                  // [S][cap][kwc]
+    int64_t* sl_s = (int64_t*)(buf + (size_t)p.S * cap * p.kwc * sizeof(float));
+    int* ps_s = (int*)(sl_s + cap);
+    float* tab = (float*)(ps_s + cap);                          // [2][half][cap]: cos, then sin
+    bool ok = true;
+    for (int c0 = 0, it = 0; c0 < rows && ok; c0 += cap, ++it) {
+        const int nr = min(cap, rows - c0);
+        if (threadIdx.x == 0) {
+            fence_proxy_async_global();                         // the other CTAs' partials, acquired above
+            fence_proxy_async_smem();                           // the previous tokens' reads of the buffer
+            const uint32_t bytes = (uint32_t)(nr * p.kwc * sizeof(float));
+            mbar_arrive_expect_tx(bar, bytes * (uint32_t)p.S);
+            for (int sp = 0; sp < p.S; ++sp)
+                bulk_load(part + (size_t)sp * cap * p.kwc, p.ws + ((int64_t)sp * p.n_tt * PT + t0 + c0) * p.kwc, bytes,
+                          bar);
+        }
+        for (int i = threadIdx.x; i < nr; i += PTHREADS) {
+            sl_s[i] = __ldg(p.slot + t0 + c0 + i);
+            ps_s[i] = half > 0 ? __ldg(p.pos + t0 + c0 + i) : 0;
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < nr * half; i += PTHREADS) {
+            const int r = i / half, j = i - r * half;
+            const int ps = ps_s[r];
+            if (sl_s[r] >= 0 && ps >= 0 && ps < p.ko.max_pos) {
+                tab[j * cap + r] = __ldg(p.ko.cos + (int64_t)ps * half + j);
+                tab[(half + j) * cap + r] = __ldg(p.ko.sin + (int64_t)ps * half + j);
+            }
+        }
+        ok = __syncthreads_and(mbar_wait(bar, it & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
+        if (!ok) break;
+        for (int rr = warp; rr < nr; rr += PTHREADS / 32) {
+            const int t = t0 + c0 + rr;
+            for (int j = lane; j < p.n_heads; j += 32) {
+                float acc = part[(size_t)rr * p.kwc + KDIM + j];
+                for (int sp = 1; sp < p.S; ++sp) acc += part[((size_t)sp * cap + rr) * p.kwc + KDIM + j];
+                p.w_out[(int64_t)t * p.n_heads + j] = acc;
+            }
+            const int64_t sl = sl_s[rr];
+            if (sl < 0) continue;                                 // token not stored
+            const int ps = ps_s[rr];
+            if (sl >= p.ko.cache_rows || (half > 0 && (ps < 0 || ps >= p.ko.max_pos))) {
+                if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
+                continue;
+            }
+            float4 a = ((const float4*)part)[(size_t)rr * kv4 + lane];
+            for (int sp = 1; sp < p.S; ++sp) {
+                const float4 v = ((const float4*)part)[((size_t)sp * cap + rr) * kv4 + lane];
+                a.x += v.x;
+                a.y += v.y;
+                a.z += v.z;
+                a.w += v.w;
+            }
+            float x[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int pr = 2 * lane + e;                        // the pair of dims 4 lane + 2 e, + 1
+                if (pr < half) rope_pair(x[2 * e], x[2 * e + 1], tab[pr * cap + rr], tab[(half + pr) * cap + rr]);
+            }
+            write_key_row(x, lane, sl, p.ko);
+        }
+        __syncthreads();                                          // the buffers are reused by the next tokens
+    }
+}
 
 }  // namespace
+
+// One warp per token: 1/RMS of the latent and the latent times the gain,
+// rounded once to bf16 (the projection kernel's A operand of query tiles).
+// Block 0 also clears the projection kernel's arrival counters.
+__global__ void __launch_bounds__(256) prepare_norm_kernel(const NormParams n) {
+    pdl_wait();
+    pdl_launch_dependents();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < n.n_tt; i += blockDim.x) n.arrivals[i] = 0u;
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= n.T) return;
+    const uint4* src = (const uint4*)(n.c_q + (int64_t)t * n.d_c);
+    uint4* dst = (uint4*)(n.cqn + (int64_t)t * n.d_c);
+    const float4* g4 = (const float4*)n.gamma;
+    float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 2
+    for (int i = lane; i < n.d_c / 8; i += 32) {
+        const uint4 xv = __ldg(src + i);
+        const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
+        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+        uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
+            ss0 = fmaf(lo, lo, ss0);
+            ss1 = fmaf(hi, hi, ss1);
+            const __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
+            xs[e] = *(const uint32_t*)&v;
+        }
+        dst[i] = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+    }
+    float ss = ss0 + ss1;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+    if (lane == 0) n.inv_rms[t] = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)n.d_c), n.eps)));
+}
 
 template <int STG, int NSUB, int QN>
 __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __grid_constant__ CUtensorMap tm_cq,
@@ -211,12 +354,13 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* full = (uint64_t*)(smem + R::BAR_OFF);                      // [STG] stage landed
-    uint64_t* conv = full + STG;                                           // [STG] query stage scaled by the gain
-    uint64_t* empty = conv + STG;                                          // [STG] stage consumed by the MMA
+    uint64_t* empty = full + STG;                                          // [STG] stage consumed by the MMA
     uint64_t* accfull = empty + STG;                                       // accumulator complete
-    uint32_t* tmem_slot = (uint32_t*)(accfull + 1);
+    uint64_t* finbar = accfull + 1;                                        // bulk copies of the tile finishing
+    uint32_t* tmem_slot = (uint32_t*)(finbar + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-    float* gain = (float*)(smem + R::GAIN_OFF);                            // [d_c] (query tiles)
+    volatile int* last_flag = abort_flag + 1;                              // this CTA finishes its token tile
+    float* tab = (float*)(smem + R::TAB_OFF);                              // [2][d_rope / 2][PT]: cos, then sin
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Job jb = job_of(p, blockIdx.x);
@@ -226,11 +370,12 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     if (threadIdx.x == 0) {
         for (int i = 0; i < STG; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&conv[i], 4);
             mbar_init(&empty[i], 1);
         }
         mbar_init(accfull, 1);
+        mbar_init(finbar, 1);
         *abort_flag = 0;
+        *last_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -241,7 +386,11 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();
+    // Only the query tiles' latent operand, 1/RMS and the arrival counters
+    // come from the norm kernel; the weights, h, positions and rotary tables
+    // are inputs that the kernels before it had finished writing when it
+    // started (it waits for them before letting this grid start), so they
+    // are read before pdl_wait().
     pdl_launch_dependents();
 
     if (warp == 0) {
@@ -253,7 +402,24 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             const uint32_t b_bytes = (uint32_t)(jb.q ? QN : PN) * PK * 2;
             tma_prefetch_desc(am);
             tma_prefetch_desc(bm);
-            int i = 0;
+            // query tiles: the weight boxes of the first ring's worth of
+            // stages before waiting for the norm kernel, then their latent boxes
+            const int npre = jb.q ? min(STG, nst) : 0;
+            for (int i = 0; i < npre; ++i) {
+                const int ns = min(NSUB, nch - i * NSUB);
+                mbar_arrive_expect_tx(&full[i], (uint32_t)ns * ((uint32_t)p.a_bytes + b_bytes));
+                for (int j = 0; j < ns; ++j)
+                    tma_load_2d(smem + i * R::SLOT + NSUB * A_BYTES + j * R::B_ROOM, bm, (jb.c0 + i * NSUB + j) * PK,
+                                brow, &full[i]);
+            }
+            if (jb.q) pdl_wait();
+            for (int i = 0; i < npre; ++i) {
+                const int ns = min(NSUB, nch - i * NSUB);
+                for (int j = 0; j < ns; ++j)
+                    tma_load_2d(smem + i * R::SLOT + j * A_BYTES, am, (jb.c0 + i * NSUB + j) * PK, jb.tt * PT,
+                                &full[i]);
+            }
+            int i = npre;
             for (; i < nst; ++i) {
                 const int st = i % STG;
                 if (!mbar_wait(&empty[st], ((i / STG) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
@@ -279,8 +445,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             bool ok = true;
             for (int i = 0; i < nst; ++i) {
                 const int st = i % STG;
-                ok = jb.q ? mbar_wait(&conv[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_PEER, abort_flag)
-                          : mbar_wait(&full[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
+                ok = mbar_wait(&full[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const int ns = min(NSUB, nch - i * NSUB);
@@ -297,73 +462,33 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             if (ok) mma_commit(accfull);
         }
     } else if (warp >= 4) {
-        // ------------------------------------- norm pass and epilogue ----
+        // ------------------------------------------------------ epilogue ----
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                  // token of the tile = TMEM lane
         const int t = jb.tt * PT + r;
-        float ss = 0.f;
-        bool ok = true;
-        // query tiles: the token's position now, and its rotary factors into L1,
-        // so that the epilogue does not wait on them
-        const int col0 = jb.f * QN, o = col0 % KDIM;    // query tiles: first feature, its dim in the head
-        const bool rot = jb.q && o < p.ko.d_rope;
-        const int ps = (jb.q && t < p.T) ? __ldg(p.pos + t) : 0;
-        const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
-        if (rot && pos_ok && t < p.T) {
-            const int64_t ti = (int64_t)ps * (p.ko.d_rope >> 1) + (o >> 1);
-            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.cos + ti));
-            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.sin + ti));
-        }
-        if (jb.q) {
-            for (int c = threadIdx.x - 128; c < p.d_c / 4; c += 128)
-                ((float4*)gain)[c] = __ldg((const float4*)p.gamma + c);
-            bar_epilogue();
-            // every stage of c_q: this token's squares, then times the gain in place
-            for (int i = 0; i < nst && ok; ++i) {
-                const int st = i % STG;
-                ok = mbar_wait(&full[st], (i / STG) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag);
-                if (!ok) break;
-                const int ns = min(NSUB, nch - i * NSUB);
-                for (int j = 0; j < ns; ++j) {
-                    uint8_t* row = smem + st * R::SLOT + j * A_BYTES + r * 128;
-                    const float4* g4 = (const float4*)(gain + (jb.c0 + i * NSUB + j) * PK);
-                    // the whole 128-byte row first, then the arithmetic, then the
-                    // stores: no load waits behind a store it might alias
-                    uint4 xv[8];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) xv[c] = *(const uint4*)(row + ((c ^ (r & 7)) << 4));   // 128-byte swizzle
-                    float s2[2] = {0.f, 0.f};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 ga = g4[2 * c], gb = g4[2 * c + 1];
-                        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                        uint32_t xs[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
-                            s2[e & 1] = fmaf(lo, lo, s2[e & 1]);
-                            s2[e & 1] = fmaf(hi, hi, s2[e & 1]);
-                            __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
-                            xs[e] = *(uint32_t*)&v;
-                        }
-                        xv[c] = make_uint4(xs[0], xs[1], xs[2], xs[3]);
-                    }
-                    ss += s2[0] + s2[1];
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) *(uint4*)(row + ((c ^ (r & 7)) << 4)) = xv[c];
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&conv[st]);
-            }
-        }
-        ok = ok && mbar_wait(accfull, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
-        if (ok) tc_fence_after();
         const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
         if (jb.q) {
-            if (ok && t < p.T && !pos_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
-            const float inv = __frcp_rn(__fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)p.d_c), p.eps)));
+            const int col0 = jb.f * QN, o = col0 % KDIM;    // first feature, its dim in the head
+            const bool rot = o < p.ko.d_rope;
             const int half = p.ko.d_rope >> 1;
+            const int ps = t < p.T ? __ldg(p.pos + t) : 0;
+            const bool pos_ok = !rot || (ps >= 0 && ps < p.ko.max_pos);
+            if (rot && p.tab && t < p.T && pos_ok) {
+                // this token's cosine / sine row while the main loop runs; the
+                // thread reads back only its own column, so no barrier is needed
+                const float* cr = p.ko.cos + (int64_t)ps * half;
+                const float* sr = p.ko.sin + (int64_t)ps * half;
+#pragma unroll 8
+                for (int i = 0; i < half; ++i) {
+                    tab[i * PT + r] = __ldg(cr + i);
+                    tab[(half + i) * PT + r] = __ldg(sr + i);
+                }
+            }
+            pdl_wait();                                     // 1/RMS of the norm kernel
+            const float inv = t < p.T ? __ldcg(p.inv_rms + t) : 0.f;
+            const bool ok = mbar_wait(accfull, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+            if (ok) tc_fence_after();
+            if (ok && t < p.T && !pos_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
 #pragma unroll 1
             for (int hh = 0; hh < QN / 32 && ok; ++hh) {
                 float v[32];
@@ -378,8 +503,16 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                     for (int c = 0; c < 32; c += 2) {
                         const int d = o32 + c;                          // dim within the head
                         if (d < p.ko.d_rope) {
-                            const int64_t ti = (int64_t)ps * half + (d >> 1);
-                            rope_pair(v[c], v[c + 1], __ldg(p.ko.cos + ti), __ldg(p.ko.sin + ti));
+                            float cs, sn;
+                            if (p.tab) {
+                                cs = tab[(d >> 1) * PT + r];
+                                sn = tab[(half + (d >> 1)) * PT + r];
+                            } else {
+                                const int64_t ti = (int64_t)ps * half + (d >> 1);
+                                cs = __ldg(p.ko.cos + ti);
+                                sn = __ldg(p.ko.sin + ti);
+                            }
+                            rope_pair(v[c], v[c + 1], cs, sn);
                         }
                     }
                 }
@@ -395,18 +528,23 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                     dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
-        } else if (ok) {
+        } else {
             // partial tile of this split -> workspace (rows past T hold zeros)
-            float4* dst = (float4*)(p.ws + ((int64_t)jb.s * p.n_tt * PT + t) * p.kwc + jb.f * PN);
+            const bool ok = mbar_wait(accfull, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                float4* dst = (float4*)(p.ws + ((int64_t)jb.s * p.n_tt * PT + t) * p.kwc + jb.f * PN);
 #pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float v[32];
-                tmem_ld32(taddr + hh * 32, v);
-                tmem_ld_wait();
+                for (int hh = 0; hh < 2; ++hh) {
+                    float v[32];
+                    tmem_ld32(taddr + hh * 32, v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    dst[hh * 8 + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    for (int c = 0; c < 8; ++c)
+                        dst[hh * 8 + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                }
             }
+            __threadfence();                                // the partial is visible before the tile's count moves
         }
     }
 
@@ -416,47 +554,21 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         tc_fence_after();
         tmem_dealloc(tmem, QN);
     }
-}
-
-__global__ void __launch_bounds__(256) prepare_finish_kernel(const PrepParams p) {
-    pdl_wait();                     // the partials of the projection kernel are visible from here on
-    pdl_launch_dependents();
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (t >= p.T) return;
-    // independent loads first: slot, position and this lane's rotary factors
-    const int64_t sl = __ldg(p.slot + t);
-    const int ps = __ldg(p.pos + t);
-    const bool pos_ok = p.ko.d_rope == 0 || (ps >= 0 && ps < p.ko.max_pos);
-    if (pos_ok && p.ko.d_rope > 0 && 4 * lane < p.ko.d_rope) {
-        const int64_t ti = (int64_t)ps * (p.ko.d_rope >> 1) + 2 * lane;
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.cos + ti));
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(p.ko.sin + ti));
+    if (!jb.q) {
+        // the last of the token tile's key / weight CTAs finishes its keys and
+        // weights (the ring is free: every copy into it has landed)
+        if (threadIdx.x == 0) {
+            pdl_wait();                                     // the counters were cleared by the norm kernel
+            const unsigned before = atomicAdd(p.arrivals + jb.tt, 1u);
+            __threadfence();
+            *last_flag = before == (unsigned)(p.n_kwf * p.S - 1) ? 1 : 0;
+        }
+        __syncthreads();
+        if (*last_flag) {
+            const int cap = min(PT, (int)((size_t)STG * R::SLOT / finish_bytes_per_token(p)));
+            finish_tile(p, jb.tt, smem, cap, finbar);
+        }
     }
-    const int64_t split_stride = (int64_t)p.n_tt * PT * p.kwc;
-    const float* src = p.ws + (int64_t)t * p.kwc;
-    float4 a = __ldcg((const float4*)src + lane);
-#pragma unroll 4
-    for (int s = 1; s < p.S; ++s) {
-        const float4 b = __ldcg((const float4*)(src + s * split_stride) + lane);
-        a.x += b.x;
-        a.y += b.y;
-        a.z += b.z;
-        a.w += b.w;
-    }
-    for (int j = lane; j < p.n_heads; j += 32) {
-        float acc = __ldcg(src + KDIM + j);
-#pragma unroll 4
-        for (int s = 1; s < p.S; ++s) acc += __ldcg(src + s * split_stride + KDIM + j);
-        p.w_out[(int64_t)t * p.n_heads + j] = acc;
-    }
-    if (sl < 0) return;                                   // token not stored
-    if (sl >= p.ko.cache_rows || !pos_ok) {
-        if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
-        return;
-    }
-    float x[4] = {a.x, a.y, a.z, a.w};
-    store_key_row(x, lane, ps, sl, p.ko);
 }
 
 __global__ void __launch_bounds__(256) key_append_kernel(const void* k, int k_fp32, int n, const int32_t* pos,
@@ -497,8 +609,10 @@ namespace {
 
 struct PrepShape {
     int n_tt, qn, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
-    size_t ws_bytes;
+    size_t cqn_off, inv_off, arr_off, ws_bytes;   // workspace: partials | scaled latent | 1/RMS | counters
 };
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Tiles and the split of the d_model reduction.  When the tiles alone fill
 // the GPU (two CTAs per SM) nothing is split; otherwise each key / weight
@@ -508,8 +622,7 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
     PrepShape s;
     s.n_tt = ceil_div(T, PT);
     // 256-wide query tiles when they alone give at least one CTA per SM
-    const bool wide = (n_heads * KDIM) % 256 == 0 && s.n_tt * (n_heads * KDIM / 256) >= num_sms &&
-                      Ring<4, 1, 256>::SMEM_BASE + (size_t)d_c * sizeof(float) <= SMEM_LIMIT;
+    const bool wide = (n_heads * KDIM) % 256 == 0 && s.n_tt * (n_heads * KDIM / 256) >= num_sms;
     s.qn = wide ? 256 : PN;
     s.n_qf = n_heads * KDIM / s.qn;
     s.n_kwf = KDIM / PN + ceil_div(n_heads, PN);
@@ -528,13 +641,14 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
     }
     if (S > s.kc_kw) S = s.kc_kw;
     s.S = S;
-    s.ws_bytes = (size_t)S * s.n_tt * PT * s.kwc * sizeof(float);
+    s.cqn_off = align256((size_t)S * s.n_tt * PT * s.kwc * sizeof(float));
+    s.inv_off = align256(s.cqn_off + (size_t)T * d_c * 2);
+    s.arr_off = align256(s.inv_off + (size_t)T * sizeof(float));
+    s.ws_bytes = s.arr_off + (size_t)s.n_tt * sizeof(unsigned);
     return s;
 }
 
 }  // namespace
-
-static_assert(Ring<4, 1, PN>::SMEM_BASE + MAX_DC * sizeof(float) <= SMEM_LIMIT, "shared memory");
 
 int indexer_prepare_max_dc() { return MAX_DC; }
 
@@ -547,26 +661,36 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     if (a.T == 0) return cudaSuccess;
     const PrepShape s = prep_shape(a.T, a.n_heads, a.d_c, a.d_model, L.num_sms);
     if (ws_bytes < s.ws_bytes) return cudaErrorInvalidValue;
+    uint8_t* ws = (uint8_t*)workspace;
+    NormParams n;
+    n.c_q = (const __nv_bfloat16*)a.c_q;
+    n.gamma = a.gamma;
+    n.cqn = (__nv_bfloat16*)(ws + s.cqn_off);
+    n.inv_rms = (float*)(ws + s.inv_off);
+    n.arrivals = (unsigned*)(ws + s.arr_off);
+    n.eps = a.eps;
+    n.T = a.T;
+    n.d_c = a.d_c;
+    n.n_tt = s.n_tt;
     CUtensorMap m_cq, m_h, m_wqb, m_wk, m_ww;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint32_t a_rows = a.T <= 64 ? 64 : PT;     // rows past the box feed accumulator rows never stored
-    bool ok = make_map_sw128(&m_cq, BF, 2, a.c_q, a.d_c, a.T, PK, a_rows);
+    bool ok = make_map_sw128(&m_cq, BF, 2, n.cqn, a.d_c, a.T, PK, a_rows);
     ok = ok && make_map_sw128(&m_h, BF, 2, a.h, a.d_model, a.T, PK, a_rows);
     ok = ok && make_map_sw128(&m_wqb, BF, 2, a.wq_b, a.d_c, (uint64_t)a.n_heads * KDIM, PK, (uint32_t)s.qn);
     ok = ok && make_map_sw128(&m_wk, BF, 2, a.wk, a.d_model, KDIM, PK, PN);
     ok = ok && make_map_sw128(&m_ww, BF, 2, a.w_proj, a.d_model, a.n_heads, PK, PN);
     if (!ok) return cudaErrorInvalidValue;
     PrepParams p;
-    p.gamma = a.gamma;
     p.pos = a.pos;
     p.slot = a.slot;
     p.q_out = (__nv_bfloat16*)a.q_out;
     p.w_out = a.w_out;
     p.ws = (float*)workspace;
+    p.inv_rms = n.inv_rms;
+    p.arrivals = n.arrivals;
     p.ko = KeyOut{a.k_cache, a.k_scale, a.rope_cos, a.rope_sin, a.cache_rows, a.d_rope, a.max_pos, (int)a.k_fmt};
-    p.eps = a.eps;
     p.T = a.T;
-    p.d_c = a.d_c;
     p.n_heads = a.n_heads;
     p.n_tt = s.n_tt;
     p.n_qf = s.n_qf;
@@ -578,31 +702,34 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     p.a_bytes = (int)a_rows * PK * 2;
     p.err = L.err;
     const int grid = s.n_tt * (s.n_qf + s.n_kwf * s.S);
-    const size_t gain_bytes = (size_t)a.d_c * sizeof(float);
-    const bool deep = s.qn == PN && grid <= L.num_sms && Ring<4, 2, PN>::SMEM_BASE + gain_bytes <= SMEM_LIMIT;
-    const size_t smem = (s.qn == 256 ? Ring<4, 1, 256>::SMEM_BASE
-                         : deep      ? Ring<4, 2, PN>::SMEM_BASE
-                                     : Ring<4, 1, PN>::SMEM_BASE) + gain_bytes;
+    const bool deep = s.qn == PN && grid <= L.num_sms;
+    // the rotary rows of a query tile in shared memory with one CTA per SM
+    // (few or many tokens), when they fit beside the ring
+    const size_t tab_bytes = (size_t)PT * a.d_rope * sizeof(float);
+    const size_t base_smem = s.qn == 256 ? Ring<4, 1, 256>::SMEM_BASE
+                           : deep        ? Ring<4, 2, PN>::SMEM_BASE
+                                         : Ring<4, 1, PN>::SMEM_BASE;
+    p.tab = (s.qn == 256 || deep) && a.d_rope > 0 && base_smem + tab_bytes <= SMEM_LIMIT;
+    const size_t smem = base_smem + (p.tab ? tab_bytes : 0);
     auto kern = s.qn == 256 ? indexer_prepare_kernel<4, 1, 256>
               : deep        ? indexer_prepare_kernel<4, 2, PN>
                             : indexer_prepare_kernel<4, 1, PN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(PTHREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = L.stream;
     cudaLaunchAttribute attr[1] = {pdl_attr()};
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, m_cq, m_h, m_wqb, m_wk, m_ww, p);
-    count_launch();
-    if (e != cudaSuccess) return e;
+    cfg.stream = L.stream;
     cfg.gridDim = dim3(ceil_div(a.T, 8));
     cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    e = cudaLaunchKernelEx(&cfg, prepare_finish_kernel, p);
+    e = cudaLaunchKernelEx(&cfg, prepare_norm_kernel, n);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(PTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    e = cudaLaunchKernelEx(&cfg, kern, m_cq, m_h, m_wqb, m_wk, m_ww, p);
     count_launch();
     return e;
 }

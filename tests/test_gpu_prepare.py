@@ -200,6 +200,29 @@ def test_prepare_v3_sizes(tokens, fmt):
     _run_prepare(workloads.PrepareShape(tokens, 1536, 7168, cache_rows=4096), fmt, seed=tokens)
 
 
+@pytest.mark.parametrize("tokens", [64, 200])
+def test_prepare_reuses_one_workspace(tokens):
+    # Two calls on one workspace that starts out filled with 0xFF bytes (the
+    # per token-tile arrival counters read 0xFFFFFFFF): the norm kernel clears
+    # the counters on every call, so each call's last key / weight CTA of a tile
+    # finishes exactly that call's keys and weights.  64 tokens: one CTA per SM,
+    # rotary rows staged in shared memory; 200 tokens: two CTAs per SM.
+    dev = torch.device("cuda:0")
+    shape = workloads.PrepareShape(tokens, 1536, 7168, cache_rows=4096)
+    ws = torch.full((dsa.indexer_prepare_workspace_size(tokens, 64, 1536, 7168),), 0xFF, dtype=torch.uint8,
+                    device=dev)
+    for seed in (31, 32):
+        inp = workloads.make_prepare_inputs(shape, seed)
+        d = {k: v.to(dev) for k, v in inp.items()}
+        cache, scale = _cache("fp8", shape.cache_rows, dev)
+        q_g, w_g = dsa.indexer_prepare(d["c_q"], d["gamma"], d["wq_b"], d["h"], d["wk"], d["w_proj"], d["pos"],
+                                       d["slot"], cache, scale, d.get("rope_cos"), d.get("rope_sin"), eps=1e-6,
+                                       workspace=ws)
+        assert dsa.get_device_error() == 0
+        _verify(inp, q_g.cpu(), w_g.cpu(), cache, scale, shape, "fp8")
+        _check_untouched(cache, scale, inp["slot"].numpy(), "fp8", shape.cache_rows)
+
+
 @pytest.mark.parametrize("n_heads,d_rope", [(16, 0), (24, 32), (96, 128)])
 def test_prepare_other_geometries(n_heads, d_rope):
     # partial head-weight tiles, no / short / full rotary parts, ragged token tiles
