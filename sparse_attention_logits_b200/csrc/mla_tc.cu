@@ -14,11 +14,11 @@
 //                       Per chunk of 64 selected keys: gather the 576-d rows
 //                       into 128-B-swizzled shared memory (cp.async), S = Q K^T
 //                       (tcgen05, M=128 heads, N=64 keys, K=576) into one of
-//                       two TMEM buffers, online softmax in base 2 with lazy
+//                       three TMEM buffers, online softmax in base 2 with lazy
 //                       rescaling (the running max moves only when a score
 //                       exceeds it by more than 2^8), P rounded to bf16 and
-//                       bulk-copied with its per-head rescale factors into the
-//                       value CTA's shared memory (DSMEM).
+//                       sent with its per-head rescale factors into the value
+//                       CTA's shared memory by 16-byte st.async remote stores.
 //   value CTA (rank 1)  gathers the first 512 dims of the same rows (the MMA
 //                       reads them as an MN-major B operand), rescales O only
 //                       for chunks whose max moved, accumulates
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
       if (role == 0) {
         // ------------------------------------- score CTA: Q load + softmax ----
         // Two groups of 4 warps take alternate chunks: group g = chunk & 1
-        // (warps SWARP0 + 4g .. +3, group g reads S buffer g).  Thread
+        // (warps SWARP0 + 4g .. +3; chunk c's S is in buffer c mod 3).  Thread
         // (quarter, lane) of a group owns head h = 32*quarter + lane (its TMEM
         // lane) and all 64 keys of its group's chunks, so a chunk needs no
         // meeting between warps.  The only sequential part of the online

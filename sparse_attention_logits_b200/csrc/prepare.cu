@@ -19,7 +19,7 @@
 // indexer_prepare_kernel -- all three projections in one launch on the
 // tcgen05 tensor cores, launched right after the norm kernel (programmatic
 // dependent launch).  Every CTA computes one tile of 128 tokens x 64
-// features (256 for query tiles when there are many tokens)
+// features (up to 256 when there are many tokens)
 // D = A . B^T (M = 128 tokens, N = 64 or 256 features, K streamed 64 at a time
 // through a 4-stage TMA ring of one or two 64-wide chunks per stage, fp32
 // accumulator in TMEM):
@@ -29,8 +29,10 @@
 //                epilogue multiplies by 1/RMS, turns the rotary pairs (the
 //                tile's cosine / sine rows are staged in shared memory while
 //                the main loop runs) and stores bf16 q_I.
-//   key/weight tiles  A = h, B = 64 rows of [W_k ; W_w], with K split over S
-//                CTAs when the token count is small (so that the long
+//   key/weight tiles  A = h, B = as many 64-row blocks of [W_k ; W_w] as a
+//                query tile is wide (up to 256 rows, so that with many
+//                tokens h crosses into the SMs once per token tile), with K
+//                split over S CTAs when the token count is small (so that the long
 //                d_model reduction is spread over as many SMs as the query
 //                tiles use).  Each writes its fp32 partial tile to the
 //                workspace and counts itself in its token tile's counter; the
@@ -83,7 +85,7 @@ struct Ring {
     static constexpr int B_ROOM = QN * PK * 2;                                 // one B box (query tiles are QN wide)
     static constexpr size_t SLOT = (size_t)NSUB * (A_BYTES + B_ROOM);          // one stage: NSUB A boxes, NSUB B boxes
     static constexpr size_t BAR_OFF = (size_t)STG * SLOT;
-    static constexpr size_t TAB_OFF = (BAR_OFF + (2 * STG + 2) * 8 + 16 + 15) & ~(size_t)15;
+    static constexpr size_t TAB_OFF = (BAR_OFF + (2 * STG + 4) * 8 + 16 + 15) & ~(size_t)15;
     static constexpr size_t SMEM_BASE = 1024 + TAB_OFF;
     static_assert(TAB_OFF % 16 == 0, "table alignment");
 };
@@ -119,7 +121,7 @@ struct PrepParams {
     unsigned* arrivals;   // [n_tt] key / weight CTAs done per token tile (cleared by the norm kernel)
     KeyOut ko;
     int T, n_heads;
-    int n_tt, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    int n_tt, n_qf, n_kwf, n_kwt, S, kc_q, kc_kw, kwc;   // n_kwf 64-row blocks of [W_k ; W_w] in n_kwt tiles
     int a_bytes;          // bytes of one A box (64 or 128 token rows)
     int tab;              // query tiles stage their rotary rows in shared memory
     unsigned* err;
@@ -134,11 +136,11 @@ struct Job {
 // Key / weight tiles come first in the grid: they are the longer ones.
 __device__ __forceinline__ Job job_of(const PrepParams& p, int b) {
     Job j;
-    const int kw = p.n_tt * p.n_kwf * p.S;
+    const int kw = p.n_tt * p.n_kwt * p.S;
     if (b < kw) {
         j.q = false;
-        j.tt = b / (p.n_kwf * p.S);
-        const int r = b - j.tt * p.n_kwf * p.S;
+        j.tt = b / (p.n_kwt * p.S);
+        const int r = b - j.tt * p.n_kwt * p.S;
         j.f = r / p.S;
         j.s = r - j.f * p.S;
         j.c0 = (int)((int64_t)p.kc_kw * j.s / p.S);
@@ -221,39 +223,94 @@ __device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, i
     write_key_row(x, lane, row, o);
 }
 
+// Eight lanes write one key row: lane g (0..7 within its aligned group of
+// 8) holds dims 16g .. 16g+15 (binary32, already turned by the rotary pairs).
+// Every lane of the warp takes part in the shuffles; only lanes with
+// `store` write.
+__device__ __forceinline__ void write_key_group(float (&x)[16], int g, bool store, int64_t row, const KeyOut& o) {
+    if (o.fmt == DSA_BF16) {
+        if (!store) return;
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x[2 * k], x[2 * k + 1]);
+            w[k] = *(const uint32_t*)&b2;
+        }
+        uint4* dst = (uint4*)o.cache + row * (KDIM / 8) + 2 * g;
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        return;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
+#pragma unroll
+    for (int m = 4; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
+    const bool fp8 = o.fmt == DSA_FP8_E4M3;
+    const float sc = amax > 0.f ? __fdiv_rn(amax, fp8 ? 448.f : 6.f) : 1.f;
+    if (!store) return;
+    float y[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) y[k] = __fdiv_rn(x[k], sc);
+    if (fp8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = f32x2_to_e4m3x2(y[4 * k], y[4 * k + 1]) | (f32x2_to_e4m3x2(y[4 * k + 2], y[4 * k + 3]) << 16);
+        ((uint4*)o.cache)[row * (KDIM / 16) + g] = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        uint32_t w[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            w[k] = f32x2_to_e2m1x2(y[8 * k], y[8 * k + 1]) | (f32x2_to_e2m1x2(y[8 * k + 2], y[8 * k + 3]) << 8) |
+                   (f32x2_to_e2m1x2(y[8 * k + 4], y[8 * k + 5]) << 16) |
+                   (f32x2_to_e2m1x2(y[8 * k + 6], y[8 * k + 7]) << 24);
+        ((uint2*)o.cache)[row * (KDIM / 16) + g] = make_uint2(w[0], w[1]);
+    }
+    if (g == 0) o.scale[row] = sc;
+}
+
 // The last key / weight CTA of token tile `tt` finishes its keys and
 // weights, `cap` tokens at a time, in the drained ring (`buf`): the S
 // partial sums of each token's 128 key and n_heads weight columns arrive by
-// bulk copies, [S][cap][kwc], while the threads fetch the tokens' slots,
-// positions and cosine / sine rows ([2][d_rope / 2][cap]); then one warp
-// per token adds the partials in split order (the result does not depend on
-// scheduling), writes the weights, turns the key's rotary pairs and writes
-// the key row in the cache's format.
+// bulk copies, split 0 into the sums [cap][kwc] and the others through two
+// staging buffers, and are added in split order (the result does not depend
+// on scheduling) while the threads fetch the tokens' slots, positions and
+// cosine / sine rows ([2][d_rope / 2][cap]).  Then eight lanes per token
+// write the weights, turn the key's rotary pairs and write the key row in the
+// cache's format (four tokens per warp at a time).
 __device__ __forceinline__ size_t finish_bytes_per_token(const PrepParams& p) {
-    return (size_t)p.S * p.kwc * sizeof(float) + sizeof(int64_t) + sizeof(int) + (size_t)p.ko.d_rope * sizeof(float);
+    return (size_t)3 * p.kwc * sizeof(float) + sizeof(int64_t) + sizeof(int) + (size_t)p.ko.d_rope * sizeof(float);
 }
 
-__device__ __forceinline__ void finish_tile(const PrepParams& p, int tt, uint8_t* buf, int cap, uint64_t* bar) {
+__device__ __forceinline__ void finish_tile(const PrepParams& p, int tt, uint8_t* buf, int cap, uint64_t* bars) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = tt * PT;
     const int rows = min(PT, p.T - t0);
     const int half = p.ko.d_rope >> 1;
     const int kv4 = p.kwc / 4;                                  // float4 per token row
-    float* part = (float*)buf;                                  // [S][cap][kwc]
-    int64_t* sl_s = (int64_t*)(buf + (size_t)p.S * cap * p.kwc * sizeof(float));
+    const size_t rowf = (size_t)cap * p.kwc;                    // floats of one [cap][kwc] buffer
+    float* acc = (float*)buf;
+    float* stg = acc + rowf;                                    // [2][cap][kwc]
+    int64_t* sl_s = (int64_t*)(stg + 2 * rowf);
     int* ps_s = (int*)(sl_s + cap);
     float* tab = (float*)(ps_s + cap);                          // [2][half][cap]: cos, then sin
+    const int64_t split = (int64_t)p.n_tt * PT * p.kwc;        // floats between two splits' partials
+    uint32_t use0 = 0u, use1 = 0u, use2 = 0u;                   // completed phases of bars[0..2]
     bool ok = true;
-    for (int c0 = 0, it = 0; c0 < rows && ok; c0 += cap, ++it) {
+    for (int c0 = 0; c0 < rows && ok; c0 += cap) {
         const int nr = min(cap, rows - c0);
+        const uint32_t bytes = (uint32_t)(nr * p.kwc * sizeof(float));
+        const float* src = p.ws + (int64_t)(t0 + c0) * p.kwc;
         if (threadIdx.x == 0) {
             fence_proxy_async_global();                         // the other CTAs' partials, acquired above
-            fence_proxy_async_smem();                           // the previous tokens' reads of the buffer
-            const uint32_t bytes = (uint32_t)(nr * p.kwc * sizeof(float));
-            mbar_arrive_expect_tx(bar, bytes * (uint32_t)p.S);
-            for (int sp = 0; sp < p.S; ++sp)
-                bulk_load(part + (size_t)sp * cap * p.kwc, p.ws + ((int64_t)sp * p.n_tt * PT + t0 + c0) * p.kwc, bytes,
-                          bar);
+            fence_proxy_async_smem();                           // earlier reads of these buffers
+            mbar_arrive_expect_tx(&bars[0], bytes);
+            bulk_load(acc, src, bytes, &bars[0]);
+            for (int sp = 1; sp < p.S && sp < 3; ++sp) {
+                mbar_arrive_expect_tx(&bars[sp], bytes);
+                bulk_load(stg + (sp - 1) * rowf, src + sp * split, bytes, &bars[sp]);
+            }
         }
         for (int i = threadIdx.x; i < nr; i += PTHREADS) {
             sl_s[i] = __ldg(p.slot + t0 + c0 + i);
@@ -268,37 +325,61 @@ __device__ __forceinline__ void finish_tile(const PrepParams& p, int tt, uint8_t
                 tab[(half + j) * cap + r] = __ldg(p.ko.sin + (int64_t)ps * half + j);
             }
         }
-        ok = __syncthreads_and(mbar_wait(bar, it & 1, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
+        ok = __syncthreads_and(mbar_wait(&bars[0], use0 & 1u, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
+        ++use0;
+        for (int sp = 1; sp < p.S && ok; ++sp) {
+            const int b = 1 + ((sp - 1) & 1);
+            float* sb = stg + ((sp - 1) & 1) * rowf;
+            const uint32_t par = (b == 1 ? use1 : use2) & 1u;
+            ok = __syncthreads_and(mbar_wait(&bars[b], par, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
+            if (b == 1) ++use1; else ++use2;
+            if (!ok) break;
+            for (int i = threadIdx.x; i < nr * kv4; i += PTHREADS) {
+                float4 x = ((float4*)acc)[i];
+                const float4 v = ((const float4*)sb)[i];
+                x.x += v.x;
+                x.y += v.y;
+                x.z += v.z;
+                x.w += v.w;
+                ((float4*)acc)[i] = x;
+            }
+            __syncthreads();                                    // the staging buffer is free again
+            if (threadIdx.x == 0 && sp + 2 < p.S) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&bars[b], bytes);
+                bulk_load(sb, src + (sp + 2) * split, bytes, &bars[b]);
+            }
+        }
         if (!ok) break;
-        for (int rr = warp; rr < nr; rr += PTHREADS / 32) {
-            const int t = t0 + c0 + rr;
-            for (int j = lane; j < p.n_heads; j += 32) {
-                float acc = part[(size_t)rr * p.kwc + KDIM + j];
-                for (int sp = 1; sp < p.S; ++sp) acc += part[((size_t)sp * cap + rr) * p.kwc + KDIM + j];
-                p.w_out[(int64_t)t * p.n_heads + j] = acc;
-            }
-            const int64_t sl = sl_s[rr];
-            if (sl < 0) continue;                                 // token not stored
-            const int ps = ps_s[rr];
-            if (sl >= p.ko.cache_rows || (half > 0 && (ps < 0 || ps >= p.ko.max_pos))) {
-                if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
-                continue;
-            }
-            float4 a = ((const float4*)part)[(size_t)rr * kv4 + lane];
-            for (int sp = 1; sp < p.S; ++sp) {
-                const float4 v = ((const float4*)part)[((size_t)sp * cap + rr) * kv4 + lane];
-                a.x += v.x;
-                a.y += v.y;
-                a.z += v.z;
-                a.w += v.w;
-            }
-            float x[4] = {a.x, a.y, a.z, a.w};
+        for (int base = warp * 4; base < nr; base += (PTHREADS / 32) * 4) {
+            const int rr = base + (lane >> 3), g = lane & 7;
+            const bool act = rr < nr;
+            const int rc = act ? rr : base;                     // every lane takes part in the shuffles
+            const float* row = acc + (size_t)rc * p.kwc;
+            const int t = t0 + c0 + rc;
+            if (act)
+                for (int j = g; j < p.n_heads; j += 8) p.w_out[(int64_t)t * p.n_heads + j] = row[KDIM + j];
+            const int64_t sl = sl_s[rc];
+            const int ps = ps_s[rc];
+            const bool bad = sl >= p.ko.cache_rows || (half > 0 && (ps < 0 || ps >= p.ko.max_pos));
+            if (act && sl >= 0 && bad && g == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
+            float x[16];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int pr = 2 * lane + e;                        // the pair of dims 4 lane + 2 e, + 1
-                if (pr < half) rope_pair(x[2 * e], x[2 * e + 1], tab[pr * cap + rr], tab[(half + pr) * cap + rr]);
+            for (int k = 0; k < 4; ++k) {
+                const float4 v = ((const float4*)row)[4 * g + k];
+                x[4 * k] = v.x;
+                x[4 * k + 1] = v.y;
+                x[4 * k + 2] = v.z;
+                x[4 * k + 3] = v.w;
             }
-            write_key_row(x, lane, sl, p.ko);
+            if (!bad) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int pr = 8 * g + i;                       // the pair of dims 16 g + 2 i, + 1
+                    if (pr < half) rope_pair(x[2 * i], x[2 * i + 1], tab[pr * cap + rc], tab[(half + pr) * cap + rc]);
+                }
+            }
+            write_key_group(x, g, act && sl >= 0 && !bad, sl, p.ko);
         }
         __syncthreads();                                          // the buffers are reused by the next tokens
     }
@@ -320,22 +401,37 @@ __global__ void __launch_bounds__(256) prepare_norm_kernel(const NormParams n) {
     const uint4* src = (const uint4*)(n.c_q + (int64_t)t * n.d_c);
     uint4* dst = (uint4*)(n.cqn + (int64_t)t * n.d_c);
     const float4* g4 = (const float4*)n.gamma;
+    const int nv = n.d_c / 8;
     float ss0 = 0.f, ss1 = 0.f;
-#pragma unroll 2
-    for (int i = lane; i < n.d_c / 8; i += 32) {
-        const uint4 xv = __ldg(src + i);
-        const float4 ga = __ldg(g4 + 2 * i), gb = __ldg(g4 + 2 * i + 1);
-        const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-        uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+    for (int base = lane; base < nv; base += 32 * 8) {
+        // eight 16-byte pieces of the row (and their gains) requested together
+        uint4 xv[8];
+        float4 ga[8], gb[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
-            ss0 = fmaf(lo, lo, ss0);
-            ss1 = fmaf(hi, hi, ss1);
-            const __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
-            xs[e] = *(const uint32_t*)&v;
+        for (int k = 0; k < 8; ++k) {
+            const int i = base + 32 * k;
+            if (i < nv) {
+                xv[k] = __ldg(src + i);
+                ga[k] = __ldg(g4 + 2 * i);
+                gb[k] = __ldg(g4 + 2 * i + 1);
+            }
         }
-        dst[i] = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = base + 32 * k;
+            if (i >= nv) break;
+            const float g[8] = {ga[k].x, ga[k].y, ga[k].z, ga[k].w, gb[k].x, gb[k].y, gb[k].z, gb[k].w};
+            uint32_t xs[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xFFFF0000u);
+                ss0 = fmaf(lo, lo, ss0);
+                ss1 = fmaf(hi, hi, ss1);
+                const __nv_bfloat162 v = __floats2bfloat162_rn(lo * g[2 * e], hi * g[2 * e + 1]);
+                xs[e] = *(const uint32_t*)&v;
+            }
+            dst[i] = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+        }
     }
     float ss = ss0 + ss1;
 #pragma unroll
@@ -356,8 +452,8 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     uint64_t* full = (uint64_t*)(smem + R::BAR_OFF);                      // [STG] stage landed
     uint64_t* empty = full + STG;                                          // [STG] stage consumed by the MMA
     uint64_t* accfull = empty + STG;                                       // accumulator complete
-    uint64_t* finbar = accfull + 1;                                        // bulk copies of the tile finishing
-    uint32_t* tmem_slot = (uint32_t*)(finbar + 1);
+    uint64_t* finbar = accfull + 1;                                        // [3] bulk copies of the tile finishing
+    uint32_t* tmem_slot = (uint32_t*)(finbar + 3);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     volatile int* last_flag = abort_flag + 1;                              // this CTA finishes its token tile
     float* tab = (float*)(smem + R::TAB_OFF);                              // [2][d_rope / 2][PT]: cos, then sin
@@ -366,6 +462,9 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     const Job jb = job_of(p, blockIdx.x);
     const int nch = jb.c1 - jb.c0;                  // reduction chunks of 64
     const int nst = (nch + NSUB - 1) / NSUB;        // stages (the last may hold fewer chunks)
+    // key / weight tiles: 64-row blocks [blk0, blk0 + nblk) of [W_k ; W_w] (QN / 64 at most)
+    const int blk0 = jb.q ? 0 : jb.f * (QN / PN);
+    const int nblk = jb.q ? 0 : min(QN / PN, p.n_kwf - blk0);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STG; ++i) {
@@ -373,7 +472,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             mbar_init(&empty[i], 1);
         }
         mbar_init(accfull, 1);
-        mbar_init(finbar, 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&finbar[i], 1);
         *abort_flag = 0;
         *last_flag = 0;
         fence_mbar_init();
@@ -397,11 +496,26 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         // ------------------------------------------------ TMA producer ----
         if (elect_one()) {
             const CUtensorMap* am = jb.q ? &tm_cq : &tm_h;
-            const CUtensorMap* bm = jb.q ? &tm_wqb : (jb.f < 2 ? &tm_wk : &tm_ww);
-            const int brow = jb.q ? jb.f * QN : (jb.f < 2 ? jb.f : jb.f - 2) * PN;
-            const uint32_t b_bytes = (uint32_t)(jb.q ? QN : PN) * PK * 2;
+            const uint32_t b_bytes = (uint32_t)(jb.q ? QN : nblk * PN) * PK * 2;
             tma_prefetch_desc(am);
-            tma_prefetch_desc(bm);
+            if (jb.q) {
+                tma_prefetch_desc(&tm_wqb);
+            } else {
+                tma_prefetch_desc(&tm_wk);
+                tma_prefetch_desc(&tm_ww);
+            }
+            // B of one chunk: QN rows of W_qb, or the tile's 64-row blocks of [W_k ; W_w]
+            auto load_b = [&](uint8_t* dst, int kx, uint64_t* bar) {
+                if (jb.q) {
+                    tma_load_2d(dst, &tm_wqb, kx, jb.f * QN, bar);
+                } else {
+                    for (int bb = 0; bb < nblk; ++bb) {
+                        const int blk = blk0 + bb;
+                        tma_load_2d(dst + bb * PN * 128, blk < 2 ? &tm_wk : &tm_ww, kx, (blk < 2 ? blk : blk - 2) * PN,
+                                    bar);
+                    }
+                }
+            };
             // query tiles: the weight boxes of the first ring's worth of
             // stages before waiting for the norm kernel, then their latent boxes
             const int npre = jb.q ? min(STG, nst) : 0;
@@ -409,8 +523,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                 const int ns = min(NSUB, nch - i * NSUB);
                 mbar_arrive_expect_tx(&full[i], (uint32_t)ns * ((uint32_t)p.a_bytes + b_bytes));
                 for (int j = 0; j < ns; ++j)
-                    tma_load_2d(smem + i * R::SLOT + NSUB * A_BYTES + j * R::B_ROOM, bm, (jb.c0 + i * NSUB + j) * PK,
-                                brow, &full[i]);
+                    load_b(smem + i * R::SLOT + NSUB * A_BYTES + j * R::B_ROOM, (jb.c0 + i * NSUB + j) * PK, &full[i]);
             }
             if (jb.q) pdl_wait();
             for (int i = 0; i < npre; ++i) {
@@ -429,7 +542,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                 for (int j = 0; j < ns; ++j) {
                     const int kx = (jb.c0 + i * NSUB + j) * PK;
                     tma_load_2d(dst + j * A_BYTES, am, kx, jb.tt * PT, &full[st]);
-                    tma_load_2d(dst + NSUB * A_BYTES + j * R::B_ROOM, bm, kx, brow, &full[st]);
+                    load_b(dst + NSUB * A_BYTES + j * R::B_ROOM, kx, &full[st]);
                 }
             }
             if (*abort_flag) {
@@ -440,7 +553,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     } else if (warp == 1) {
         // ------------------------------------------------- MMA issuer ----
         if (elect_one()) {
-            const uint32_t idesc = jb.q ? idesc_bf16_f32(PT, QN, 0, 0) : idesc_bf16_f32(PT, PN, 0, 0);
+            const uint32_t idesc = idesc_bf16_f32(PT, jb.q ? QN : nblk * PN, 0, 0);
             const uint32_t base = smem_u32(smem);
             bool ok = true;
             for (int i = 0; i < nst; ++i) {
@@ -533,9 +646,9 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             const bool ok = mbar_wait(accfull, 0, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag);
             if (ok) {
                 tc_fence_after();
-                float4* dst = (float4*)(p.ws + ((int64_t)jb.s * p.n_tt * PT + t) * p.kwc + jb.f * PN);
+                float4* dst = (float4*)(p.ws + ((int64_t)jb.s * p.n_tt * PT + t) * p.kwc + blk0 * PN);
 #pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
+                for (int hh = 0; hh < 2 * nblk; ++hh) {
                     float v[32];
                     tmem_ld32(taddr + hh * 32, v);
                     tmem_ld_wait();
@@ -561,7 +674,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             pdl_wait();                                     // the counters were cleared by the norm kernel
             const unsigned before = atomicAdd(p.arrivals + jb.tt, 1u);
             __threadfence();
-            *last_flag = before == (unsigned)(p.n_kwf * p.S - 1) ? 1 : 0;
+            *last_flag = before == (unsigned)(p.n_kwt * p.S - 1) ? 1 : 0;
         }
         __syncthreads();
         if (*last_flag) {
@@ -608,7 +721,7 @@ __global__ void __launch_bounds__(256) key_append_kernel(const void* k, int k_fp
 namespace {
 
 struct PrepShape {
-    int n_tt, qn, n_qf, n_kwf, S, kc_q, kc_kw, kwc;
+    int n_tt, qn, n_qf, n_kwf, n_kwt, S, kc_q, kc_kw, kwc;
     size_t cqn_off, inv_off, arr_off, ws_bytes;   // workspace: partials | scaled latent | 1/RMS | counters
 };
 
@@ -629,12 +742,13 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
     s.kc_q = d_c / PK;
     s.kc_kw = d_model / PK;
     s.kwc = s.n_kwf * PN;
+    s.n_kwt = ceil_div(s.n_kwf, s.qn / PN);           // key / weight tiles as wide as the query tiles
     const int slots = 2 * num_sms;
-    const int base = s.n_tt * (s.n_qf + s.n_kwf);
+    const int base = s.n_tt * (s.n_qf + s.n_kwt);
     int S = 1;
     if (base < slots) {
         S = ceil_div(s.kc_kw, s.kc_q > 0 ? s.kc_q : 1);
-        const int room = (slots - s.n_tt * s.n_qf) / (s.n_tt * s.n_kwf);
+        const int room = (slots - s.n_tt * s.n_qf) / (s.n_tt * s.n_kwt);
         if (S > room) S = room;
         if (S > 16) S = 16;
         if (S < 1) S = 1;
@@ -695,13 +809,14 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     p.n_tt = s.n_tt;
     p.n_qf = s.n_qf;
     p.n_kwf = s.n_kwf;
+    p.n_kwt = s.n_kwt;
     p.S = s.S;
     p.kc_q = s.kc_q;
     p.kc_kw = s.kc_kw;
     p.kwc = s.kwc;
     p.a_bytes = (int)a_rows * PK * 2;
     p.err = L.err;
-    const int grid = s.n_tt * (s.n_qf + s.n_kwf * s.S);
+    const int grid = s.n_tt * (s.n_qf + s.n_kwt * s.S);
     const bool deep = s.qn == PN && grid <= L.num_sms;
     // the rotary rows of a query tile in shared memory with one CTA per SM
     // (few or many tokens), when they fit beside the ring

@@ -237,6 +237,15 @@ def test_prepare_prefill_many_token_tiles(fmt):
     _run_prepare(workloads.PrepareShape(2400, 512, 1024, cache_rows=4096), fmt, seed=5)
 
 
+@pytest.mark.parametrize("n_heads,d_rope", [(96, 128), (200, 32)])
+def test_prepare_prefill_wide_key_weight_tiles(n_heads, d_rope):
+    # 256-wide tiles: [W_k ; W_w] in one tile of 256 rows (96 heads; rotary rows
+    # too long to stage in shared memory) or in tiles of 256 and 128 rows
+    # (200 heads, the last weight block partly past the head count)
+    _run_prepare(workloads.PrepareShape(2400, 512, 1024, n_heads=n_heads, d_rope=d_rope, cache_rows=4096), "fp8",
+                 seed=n_heads + d_rope)
+
+
 def test_prepare_then_indexer_scores_the_new_keys():
     # the prepared queries / weights and the fp8 cache feed the indexer directly
     dev = torch.device("cuda:0")
