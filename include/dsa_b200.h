@@ -311,8 +311,8 @@ DSA_API size_t dsa_indexer_prepare_workspace_size(int tokens, int n_heads, int d
  * projected up, the result split into a part with and a part without rotary
  * position encoding, the former turned by apply_rotary_emb, and weights_proj
  * gives the per-head weights; section 1.3: a learned linear map takes query
- * and key to 128 dims), in two launches: the latent's norm, then the three
- * projections on the tensor cores:
+ * and key to 128 dims), in three launches: the latent's norm, the three
+ * projections on the tensor cores, the key-cache write:
  *
  *   q_out[t, j, :] = RoPE( W_qb[j*128 .. j*128+127] . RMSNorm(c_q[t]) )
  *   w_out[t, :]    = W_w . h[t]
@@ -343,9 +343,9 @@ DSA_API size_t dsa_indexer_prepare_workspace_size(int tokens, int n_heads, int d
  *                 all of it in binary32 with every operation rounded on its own
  *   workspace     dsa_indexer_prepare_workspace_size() bytes, 256-byte aligned; no
  *                 part of it needs to hold anything on entry (it carries the scaled
- *                 latent and 1/RMS of each token, the fp32 partial sums of the key
- *                 and weight projections, which the last CTA of each token tile
- *                 adds up in a fixed order, and that tile's arrival counter)
+ *                 latent and 1/RMS of each token and the fp32 partial sums of the
+ *                 key and weight projections, which the last kernel adds up in a
+ *                 fixed order)
  * The projections multiply bf16 operands with fp32 accumulation; the norm's
  * gain is applied to c_q in bf16 (c_q * gain rounded once) and 1/RMS (fp32)
  * to the product.  head_dim must be 128; d_c and d_model multiples of 64,

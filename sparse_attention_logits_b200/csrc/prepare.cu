@@ -13,8 +13,7 @@
 // prepare_norm_kernel -- one warp per token: the token's sum of squares of
 // c_q (fp32) gives 1/RMS, and c_q * gain is rounded once to bf16 into the
 // workspace; every query tile then reads that operand as it is, instead of
-// each of them scaling the same latent again.  It also clears the per
-// token-tile arrival counters of the projection kernel.
+// each of them scaling the same latent again.
 //
 // indexer_prepare_kernel -- all three projections in one launch on the
 // tcgen05 tensor cores, launched right after the norm kernel (programmatic
@@ -35,14 +34,17 @@
 //                split over S CTAs when the token count is small (so that the long
 //                d_model reduction is spread over as many SMs as the query
 //                tiles use).  Each writes its fp32 partial tile to the
-//                workspace and counts itself in its token tile's counter; the
-//                last of a token tile's key / weight CTAs adds the partials
-//                up in split order (the result does not depend on
-//                scheduling), writes the head weights, turns the key's
-//                rotary pairs and writes the key row into the cache.
+//                workspace.
 // Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and
 // TMEM owner), warps 4-7 epilogue (warp 4+q owns TMEM lanes 32q .. 32q+31 =
 // tokens of the tile).
+//
+// prepare_finish_kernel -- launched right after (programmatic dependent
+// launch), one warp per token: its slot, position and rotary factors are
+// read before the projections finish; then it adds the S partials in split
+// order (the result does not depend on scheduling), writes the head
+// weights, turns the key's rotary pairs and writes the key row in the
+// cache's format.
 //
 // key_append_kernel -- the key-cache write alone for keys that are already
 // projected (for instance compressed CSA keys): one warp per key row, lane l
@@ -85,7 +87,7 @@ struct Ring {
     static constexpr int B_ROOM = QN * PK * 2;                                 // one B box (query tiles are QN wide)
     static constexpr size_t SLOT = (size_t)NSUB * (A_BYTES + B_ROOM);          // one stage: NSUB A boxes, NSUB B boxes
     static constexpr size_t BAR_OFF = (size_t)STG * SLOT;
-    static constexpr size_t TAB_OFF = (BAR_OFF + (2 * STG + 4) * 8 + 16 + 15) & ~(size_t)15;
+    static constexpr size_t TAB_OFF = (BAR_OFF + (2 * STG + 1) * 8 + 16 + 15) & ~(size_t)15;
     static constexpr size_t SMEM_BASE = 1024 + TAB_OFF;
     static_assert(TAB_OFF % 16 == 0, "table alignment");
 };
@@ -106,9 +108,8 @@ struct NormParams {
     const float* gamma;         // [d_c]
     __nv_bfloat16* cqn;         // [T, d_c] c_q * gain, rounded once
     float* inv_rms;             // [T]
-    unsigned* arrivals;         // [n_tt] cleared here
     float eps;
-    int T, d_c, n_tt;
+    int T, d_c;
 };
 
 struct PrepParams {
@@ -118,7 +119,6 @@ struct PrepParams {
     float* w_out;         // [T, H]
     float* ws;            // [S][n_tt * 128][kwc] partial sums of the key / weight tiles
     const float* inv_rms; // [T] (norm kernel)
-    unsigned* arrivals;   // [n_tt] key / weight CTAs done per token tile (cleared by the norm kernel)
     KeyOut ko;
     int T, n_heads;
     int n_tt, n_qf, n_kwf, n_kwt, S, kc_q, kc_kw, kwc;   // n_kwf 64-row blocks of [W_k ; W_w] in n_kwt tiles
@@ -223,178 +223,13 @@ __device__ __forceinline__ void store_key_row(float (&x)[4], int lane, int ps, i
     write_key_row(x, lane, row, o);
 }
 
-// Eight lanes write one key row: lane g (0..7 within its aligned group of
-// 8) holds dims 16g .. 16g+15 (binary32, already turned by the rotary pairs).
-// Every lane of the warp takes part in the shuffles; only lanes with
-// `store` write.
-__device__ __forceinline__ void write_key_group(float (&x)[16], int g, bool store, int64_t row, const KeyOut& o) {
-    if (o.fmt == DSA_BF16) {
-        if (!store) return;
-        uint32_t w[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x[2 * k], x[2 * k + 1]);
-            w[k] = *(const uint32_t*)&b2;
-        }
-        uint4* dst = (uint4*)o.cache + row * (KDIM / 8) + 2 * g;
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        return;
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(x[k]));
-#pragma unroll
-    for (int m = 4; m > 0; m >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, m));
-    const bool fp8 = o.fmt == DSA_FP8_E4M3;
-    const float sc = amax > 0.f ? __fdiv_rn(amax, fp8 ? 448.f : 6.f) : 1.f;
-    if (!store) return;
-    float y[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) y[k] = __fdiv_rn(x[k], sc);
-    if (fp8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[k] = f32x2_to_e4m3x2(y[4 * k], y[4 * k + 1]) | (f32x2_to_e4m3x2(y[4 * k + 2], y[4 * k + 3]) << 16);
-        ((uint4*)o.cache)[row * (KDIM / 16) + g] = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-        uint32_t w[2];
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-            w[k] = f32x2_to_e2m1x2(y[8 * k], y[8 * k + 1]) | (f32x2_to_e2m1x2(y[8 * k + 2], y[8 * k + 3]) << 8) |
-                   (f32x2_to_e2m1x2(y[8 * k + 4], y[8 * k + 5]) << 16) |
-                   (f32x2_to_e2m1x2(y[8 * k + 6], y[8 * k + 7]) << 24);
-        ((uint2*)o.cache)[row * (KDIM / 16) + g] = make_uint2(w[0], w[1]);
-    }
-    if (g == 0) o.scale[row] = sc;
-}
-
-// The last key / weight CTA of token tile `tt` finishes its keys and
-// weights, `cap` tokens at a time, in the drained ring (`buf`): the S
-// partial sums of each token's 128 key and n_heads weight columns arrive by
-// bulk copies, split 0 into the sums [cap][kwc] and the others through two
-// staging buffers, and are added in split order (the result does not depend
-// on scheduling) while the threads fetch the tokens' slots, positions and
-// cosine / sine rows ([2][d_rope / 2][cap]).  Then eight lanes per token
-// write the weights, turn the key's rotary pairs and write the key row in the
-// cache's format (four tokens per warp at a time).
-__device__ __forceinline__ size_t finish_bytes_per_token(const PrepParams& p) {
-    return (size_t)3 * p.kwc * sizeof(float) + sizeof(int64_t) + sizeof(int) + (size_t)p.ko.d_rope * sizeof(float);
-}
-
-__device__ __forceinline__ void finish_tile(const PrepParams& p, int tt, uint8_t* buf, int cap, uint64_t* bars) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = tt * PT;
-    const int rows = min(PT, p.T - t0);
-    const int half = p.ko.d_rope >> 1;
-    const int kv4 = p.kwc / 4;                                  // float4 per token row
-    const size_t rowf = (size_t)cap * p.kwc;                    // floats of one [cap][kwc] buffer
-    float* acc = (float*)buf;
-    float* stg = acc + rowf;                                    // [2][cap][kwc]
-    int64_t* sl_s = (int64_t*)(stg + 2 * rowf);
-    int* ps_s = (int*)(sl_s + cap);
-    float* tab = (float*)(ps_s + cap);                          // [2][half][cap]: cos, then sin
-    const int64_t split = (int64_t)p.n_tt * PT * p.kwc;        // floats between two splits' partials
-    uint32_t use0 = 0u, use1 = 0u, use2 = 0u;                   // completed phases of bars[0..2]
-    bool ok = true;
-    for (int c0 = 0; c0 < rows && ok; c0 += cap) {
-        const int nr = min(cap, rows - c0);
-        const uint32_t bytes = (uint32_t)(nr * p.kwc * sizeof(float));
-        const float* src = p.ws + (int64_t)(t0 + c0) * p.kwc;
-        if (threadIdx.x == 0) {
-            fence_proxy_async_global();                         // the other CTAs' partials, acquired above
-            fence_proxy_async_smem();                           // earlier reads of these buffers
-            mbar_arrive_expect_tx(&bars[0], bytes);
-            bulk_load(acc, src, bytes, &bars[0]);
-            for (int sp = 1; sp < p.S && sp < 3; ++sp) {
-                mbar_arrive_expect_tx(&bars[sp], bytes);
-                bulk_load(stg + (sp - 1) * rowf, src + sp * split, bytes, &bars[sp]);
-            }
-        }
-        for (int i = threadIdx.x; i < nr; i += PTHREADS) {
-            sl_s[i] = __ldg(p.slot + t0 + c0 + i);
-            ps_s[i] = half > 0 ? __ldg(p.pos + t0 + c0 + i) : 0;
-        }
-        __syncthreads();
-        for (int i = threadIdx.x; i < nr * half; i += PTHREADS) {
-            const int r = i / half, j = i - r * half;
-            const int ps = ps_s[r];
-            if (sl_s[r] >= 0 && ps >= 0 && ps < p.ko.max_pos) {
-                tab[j * cap + r] = __ldg(p.ko.cos + (int64_t)ps * half + j);
-                tab[(half + j) * cap + r] = __ldg(p.ko.sin + (int64_t)ps * half + j);
-            }
-        }
-        ok = __syncthreads_and(mbar_wait(&bars[0], use0 & 1u, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
-        ++use0;
-        for (int sp = 1; sp < p.S && ok; ++sp) {
-            const int b = 1 + ((sp - 1) & 1);
-            float* sb = stg + ((sp - 1) & 1) * rowf;
-            const uint32_t par = (b == 1 ? use1 : use2) & 1u;
-            ok = __syncthreads_and(mbar_wait(&bars[b], par, p.err, DEV_ERR_TIMEOUT_TMA, nullptr) ? 1 : 0) != 0;
-            if (b == 1) ++use1; else ++use2;
-            if (!ok) break;
-            for (int i = threadIdx.x; i < nr * kv4; i += PTHREADS) {
-                float4 x = ((float4*)acc)[i];
-                const float4 v = ((const float4*)sb)[i];
-                x.x += v.x;
-                x.y += v.y;
-                x.z += v.z;
-                x.w += v.w;
-                ((float4*)acc)[i] = x;
-            }
-            __syncthreads();                                    // the staging buffer is free again
-            if (threadIdx.x == 0 && sp + 2 < p.S) {
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&bars[b], bytes);
-                bulk_load(sb, src + (sp + 2) * split, bytes, &bars[b]);
-            }
-        }
-        if (!ok) break;
-        for (int base = warp * 4; base < nr; base += (PTHREADS / 32) * 4) {
-            const int rr = base + (lane >> 3), g = lane & 7;
-            const bool act = rr < nr;
-            const int rc = act ? rr : base;                     // every lane takes part in the shuffles
-            const float* row = acc + (size_t)rc * p.kwc;
-            const int t = t0 + c0 + rc;
-            if (act)
-                for (int j = g; j < p.n_heads; j += 8) p.w_out[(int64_t)t * p.n_heads + j] = row[KDIM + j];
-            const int64_t sl = sl_s[rc];
-            const int ps = ps_s[rc];
-            const bool bad = sl >= p.ko.cache_rows || (half > 0 && (ps < 0 || ps >= p.ko.max_pos));
-            if (act && sl >= 0 && bad && g == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
-            float x[16];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 v = ((const float4*)row)[4 * g + k];
-                x[4 * k] = v.x;
-                x[4 * k + 1] = v.y;
-                x[4 * k + 2] = v.z;
-                x[4 * k + 3] = v.w;
-            }
-            if (!bad) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int pr = 8 * g + i;                       // the pair of dims 16 g + 2 i, + 1
-                    if (pr < half) rope_pair(x[2 * i], x[2 * i + 1], tab[pr * cap + rc], tab[(half + pr) * cap + rc]);
-                }
-            }
-            write_key_group(x, g, act && sl >= 0 && !bad, sl, p.ko);
-        }
-        __syncthreads();                                          // the buffers are reused by the next tokens
-    }
-}
-
 }  // namespace
 
 // One warp per token: 1/RMS of the latent and the latent times the gain,
 // rounded once to bf16 (the projection kernel's A operand of query tiles).
-// Block 0 also clears the projection kernel's arrival counters.
 __global__ void __launch_bounds__(256) prepare_norm_kernel(const NormParams n) {
     pdl_wait();
     pdl_launch_dependents();
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < n.n_tt; i += blockDim.x) n.arrivals[i] = 0u;
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= n.T) return;
@@ -452,10 +287,8 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     uint64_t* full = (uint64_t*)(smem + R::BAR_OFF);                      // [STG] stage landed
     uint64_t* empty = full + STG;                                          // [STG] stage consumed by the MMA
     uint64_t* accfull = empty + STG;                                       // accumulator complete
-    uint64_t* finbar = accfull + 1;                                        // [3] bulk copies of the tile finishing
-    uint32_t* tmem_slot = (uint32_t*)(finbar + 3);
+    uint32_t* tmem_slot = (uint32_t*)(accfull + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;                              // this CTA finishes its token tile
     float* tab = (float*)(smem + R::TAB_OFF);                              // [2][d_rope / 2][PT]: cos, then sin
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -472,9 +305,7 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
             mbar_init(&empty[i], 1);
         }
         mbar_init(accfull, 1);
-        for (int i = 0; i < 3; ++i) mbar_init(&finbar[i], 1);
         *abort_flag = 0;
-        *last_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -657,7 +488,6 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
                         dst[hh * 8 + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
                 }
             }
-            __threadfence();                                // the partial is visible before the tile's count moves
         }
     }
 
@@ -667,21 +497,63 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
         tc_fence_after();
         tmem_dealloc(tmem, QN);
     }
-    if (!jb.q) {
-        // the last of the token tile's key / weight CTAs finishes its keys and
-        // weights (the ring is free: every copy into it has landed)
-        if (threadIdx.x == 0) {
-            pdl_wait();                                     // the counters were cleared by the norm kernel
-            const unsigned before = atomicAdd(p.arrivals + jb.tt, 1u);
-            __threadfence();
-            *last_flag = before == (unsigned)(p.n_kwt * p.S - 1) ? 1 : 0;
-        }
-        __syncthreads();
-        if (*last_flag) {
-            const int cap = min(PT, (int)((size_t)STG * R::SLOT / finish_bytes_per_token(p)));
-            finish_tile(p, jb.tt, smem, cap, finbar);
+}
+
+// One warp per token (eight per CTA).
+__global__ void __launch_bounds__(256) prepare_finish_kernel(const PrepParams p) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // inputs first (the projections do not write them): slot, position and
+    // this lane's rotary factors (dims 4 lane .. 4 lane + 3: pairs 2 lane, 2 lane + 1)
+    int64_t sl = -1;
+    int ps = 0;
+    bool pos_ok = true;
+    const int half = p.ko.d_rope >> 1;
+    float cs[2] = {1.f, 1.f}, sn[2] = {0.f, 0.f};
+    if (t < p.T) {
+        sl = __ldg(p.slot + t);
+        ps = half > 0 ? __ldg(p.pos + t) : 0;
+        pos_ok = half == 0 || (ps >= 0 && ps < p.ko.max_pos);
+        if (sl >= 0 && pos_ok) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                if (2 * lane + e < half) {
+                    cs[e] = __ldg(p.ko.cos + (int64_t)ps * half + 2 * lane + e);
+                    sn[e] = __ldg(p.ko.sin + (int64_t)ps * half + 2 * lane + e);
+                }
+            }
         }
     }
+    pdl_wait();                     // the partials of the projection kernel are visible from here on
+    pdl_launch_dependents();
+    if (t >= p.T) return;
+    const int64_t split_stride = (int64_t)p.n_tt * PT * p.kwc;
+    const float* src = p.ws + (int64_t)t * p.kwc;
+    float4 a = __ldcg((const float4*)src + lane);
+#pragma unroll 4
+    for (int sp = 1; sp < p.S; ++sp) {
+        const float4 b = __ldcg((const float4*)(src + sp * split_stride) + lane);
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+    }
+    for (int j = lane; j < p.n_heads; j += 32) {
+        float acc = __ldcg(src + KDIM + j);
+#pragma unroll 4
+        for (int sp = 1; sp < p.S; ++sp) acc += __ldcg(src + sp * split_stride + KDIM + j);
+        p.w_out[(int64_t)t * p.n_heads + j] = acc;
+    }
+    if (sl < 0) return;                                   // token not stored
+    if (sl >= p.ko.cache_rows || !pos_ok) {
+        if (lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
+        return;
+    }
+    float x[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+        if (2 * lane + e < half) rope_pair(x[2 * e], x[2 * e + 1], cs[e], sn[e]);
+    write_key_row(x, lane, sl, p.ko);
 }
 
 __global__ void __launch_bounds__(256) key_append_kernel(const void* k, int k_fp32, int n, const int32_t* pos,
@@ -722,7 +594,7 @@ namespace {
 
 struct PrepShape {
     int n_tt, qn, n_qf, n_kwf, n_kwt, S, kc_q, kc_kw, kwc;
-    size_t cqn_off, inv_off, arr_off, ws_bytes;   // workspace: partials | scaled latent | 1/RMS | counters
+    size_t cqn_off, inv_off, ws_bytes;   // workspace: partials | scaled latent | 1/RMS
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -757,8 +629,7 @@ PrepShape prep_shape(int T, int n_heads, int d_c, int d_model, int num_sms) {
     s.S = S;
     s.cqn_off = align256((size_t)S * s.n_tt * PT * s.kwc * sizeof(float));
     s.inv_off = align256(s.cqn_off + (size_t)T * d_c * 2);
-    s.arr_off = align256(s.inv_off + (size_t)T * sizeof(float));
-    s.ws_bytes = s.arr_off + (size_t)s.n_tt * sizeof(unsigned);
+    s.ws_bytes = s.inv_off + (size_t)T * sizeof(float);
     return s;
 }
 
@@ -781,11 +652,9 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     n.gamma = a.gamma;
     n.cqn = (__nv_bfloat16*)(ws + s.cqn_off);
     n.inv_rms = (float*)(ws + s.inv_off);
-    n.arrivals = (unsigned*)(ws + s.arr_off);
     n.eps = a.eps;
     n.T = a.T;
     n.d_c = a.d_c;
-    n.n_tt = s.n_tt;
     CUtensorMap m_cq, m_h, m_wqb, m_wk, m_ww;
     const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint32_t a_rows = a.T <= 64 ? 64 : PT;     // rows past the box feed accumulator rows never stored
@@ -802,7 +671,6 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     p.w_out = a.w_out;
     p.ws = (float*)workspace;
     p.inv_rms = n.inv_rms;
-    p.arrivals = n.arrivals;
     p.ko = KeyOut{a.k_cache, a.k_scale, a.rope_cos, a.rope_sin, a.cache_rows, a.d_rope, a.max_pos, (int)a.k_fmt};
     p.T = a.T;
     p.n_heads = a.n_heads;
@@ -845,6 +713,12 @@ cudaError_t launch_indexer_prepare(const Launch& L, const PrepareArgs& a, void* 
     cfg.blockDim = dim3(PTHREADS);
     cfg.dynamicSmemBytes = smem;
     e = cudaLaunchKernelEx(&cfg, kern, m_cq, m_h, m_wqb, m_wk, m_ww, p);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3(ceil_div(a.T, 8));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    e = cudaLaunchKernelEx(&cfg, prepare_finish_kernel, p);
     count_launch();
     return e;
 }

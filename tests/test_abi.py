@@ -163,8 +163,7 @@ def test_indexer_prepare_workspace_sizes(lib):
     # no device here: the size is taken for a 1024-SM GPU (the most splits).
     # Layout: fp32 partials of 128 key + 64 weight columns for 128 token rows
     # per split and token tile | the scaled latent, [tokens, d_c] bf16 |
-    # 1/RMS, [tokens] fp32 | one arrival counter per token tile, each part
-    # starting on a 256-byte boundary.
+    # 1/RMS, [tokens] fp32, each part starting on a 256-byte boundary.
     lib.dsa_indexer_prepare_workspace_size.restype = ctypes.c_size_t
     lib.dsa_indexer_prepare_workspace_size.argtypes = [ctypes.c_int] * 4
 
@@ -175,13 +174,13 @@ def test_indexer_prepare_workspace_sizes(lib):
         tiles = (T + 127) // 128
         part = splits * tiles * 128 * 192 * 4
         inv = up(up(part) + T * d_c * 2)
-        return up(inv + T * 4) + tiles * 4
+        return inv + T * 4
 
     # 64 tokens: one token tile, the 112-chunk d_model reduction split 5 ways
     # (about the 24 chunks of a query tile)
-    assert lib.dsa_indexer_prepare_workspace_size(64, 64, 1536, 7168) == size(64, 1536, 5) == 688388
+    assert lib.dsa_indexer_prepare_workspace_size(64, 64, 1536, 7168) == size(64, 1536, 5) == 688384
     # 16384 tokens: 256-wide query tiles fill the GPU, no split
-    assert lib.dsa_indexer_prepare_workspace_size(16384, 64, 1536, 7168) == size(16384, 1536, 1) == 62980608
+    assert lib.dsa_indexer_prepare_workspace_size(16384, 64, 1536, 7168) == size(16384, 1536, 1) == 62980096
     assert lib.dsa_indexer_prepare_workspace_size(0, 64, 1536, 7168) == 0
 
 

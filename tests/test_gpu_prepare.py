@@ -202,11 +202,10 @@ def test_prepare_v3_sizes(tokens, fmt):
 
 @pytest.mark.parametrize("tokens", [64, 200])
 def test_prepare_reuses_one_workspace(tokens):
-    # Two calls on one workspace that starts out filled with 0xFF bytes (the
-    # per token-tile arrival counters read 0xFFFFFFFF): the norm kernel clears
-    # the counters on every call, so each call's last key / weight CTA of a tile
-    # finishes exactly that call's keys and weights.  64 tokens: one CTA per SM,
-    # rotary rows staged in shared memory; 200 tokens: two CTAs per SM.
+    # Two calls on one workspace that starts out filled with 0xFF bytes: nothing
+    # in it is read before this call writes it, so each call gives its own
+    # keys and weights.  64 tokens: one CTA per SM, rotary rows staged in shared
+    # memory; 200 tokens: two CTAs per SM.
     dev = torch.device("cuda:0")
     shape = workloads.PrepareShape(tokens, 1536, 7168, cache_rows=4096)
     ws = torch.full((dsa.indexer_prepare_workspace_size(tokens, 64, 1536, 7168),), 0xFF, dtype=torch.uint8,
