@@ -336,6 +336,17 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     const Work w = work_of(p);
 
     if (threadIdx.x == 0) {
+        if (role == 0) {
+            // Q [128 heads x 576] of this row first (it needs no load of the
+            // row's batch index): 9 boxes of 128 rows x 64 dims, 128-byte
+            // swizzled, into gather stages 1-2 (not yet in use)
+            mbar_init(&bars->qfull, 1);
+            fence_mbar_init();
+            tma_prefetch_desc(&q_map);
+            mbar_arrive_expect_tx(&bars->qfull, QBYTES);
+            for (int b = 0; b < KBLK; ++b)
+                tma_load_2d(gbuf + Q_OFF + b * (H * 128), &q_map, b * 64, w.t * H, &bars->qfull);
+        }
         for (int i = 0; i < SSTAGES; ++i) {
             mbar_init(&bars->full[i], DENSE ? 1 : PWARPS * 32);
             mbar_init(&bars->empty[i], 1);
@@ -351,14 +362,12 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             mbar_init(&bars->odone[i], 1);
         }
         mbar_init(&bars->qready, 8);
-        mbar_init(&bars->qfull, 1);
         mbar_init(&bars->statready, 8);
         mbar_init(&bars->statack, 4);
         mbar_init(&bars->ofinal, 1);
         mbar_init(&bars->statfull, 1);
         bars->abort = 0;
         for (int i = 0; i < 4; ++i) bars->mdone[i] = -1;
-        if (!w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
         mbar_init(&bars->cfree, 1);
         mbar_init(&bars->cstat, H);
         mbar_init(&bars->crecv, 8 * 32);
@@ -368,16 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
             mbar_arrive_expect_tx(&bars->statfull, SBYTES);
         }
         fence_mbar_init();
-        if (role == 0) {
-            // Q [128 heads x 576] of this row: 9 boxes of 128 rows x 64 dims,
-            // 128-byte swizzled, into gather stages 1-2 (not yet in use)
-            tma_prefetch_desc(&q_map);
-            mbar_arrive_expect_tx(&bars->qfull, QBYTES);
-            for (int b = 0; b < KBLK; ++b)
-                tma_load_2d(gbuf + Q_OFF + b * (H * 128), &q_map, b * 64, w.t * H, &bars->qfull);
-        } else {
-            tma_prefetch_desc(&o_map);
-        }
+        if (role == 1) tma_prefetch_desc(&o_map);
     }
     if (warp == MWARP) {
         tmem_alloc(&bars->tmem, TMEM_COLS);
@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(THREADS, 1) mla_tc_kernel(const __grid_constan
     tc_fence_after();
     const uint32_t tmem = bars->tmem;
     const uint32_t peer = cluster_ctarank() ^ 1u;
+    if (threadIdx.x == 0 && !w.b_ok) record_error(p.err, DEV_ERR_BAD_INDEX);
 
     if (warp < PWARPS) {
         // ------------------------------------------------ gather producers ----
