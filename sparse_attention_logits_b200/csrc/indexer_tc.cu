@@ -58,18 +58,27 @@ template <int NQ, int KF>
 struct Cfg {
     static constexpr bool FP8 = KF != KF_BF16;      // narrow keys: widened into TMEM, scaled in the epilogue
     static constexpr int N = NQ * HI;
-    static constexpr int STAGES = KF == KF_FP4 ? 16 : KF == KF_FP8 ? 8 : (NQ == 1 ? 6 : 3);
-    static constexpr int KBYTES = KF == KF_FP4 ? KT * DI / 2 : KF == KF_FP8 ? KT * DI : KT * DI * 2;  // one key tile
+    // Narrow-key decode takes 256 keys per unit (two 128-key MMA tiles behind one
+    // TMA box, one widening pass, one MMA commit and one epilogue hand-off): every
+    // hand-off of the unit pipeline costs about the same per unit whatever its
+    // size, so a 16 KB fp8 / 8 KB fp4 unit of 128 keys left the stream at half
+    // the rate the same ring reaches when nothing else runs.
+    static constexpr int SUB = (FP8 && NQ == 1) ? 2 : 1;            // 128-key MMA tiles per unit
+    static constexpr int KTU = SUB * KT;                             // keys per unit
+    static constexpr int STAGES = KF == KF_FP4 ? (SUB == 2 ? 12 : 16) : KF == KF_FP8 ? (SUB == 2 ? 6 : 8) : (NQ == 1 ? 6 : 3);
+    static constexpr int KBYTES = KF == KF_FP4 ? KTU * DI / 2 : KF == KF_FP8 ? KTU * DI : KTU * DI * 2;  // one unit
     static constexpr int QBYTES = N * DI * 2;                        // one query tile (bf16)
-    static constexpr int ACC_COLS = N;
-    // accumulator ring: decode has 4 (two epilogue groups take alternate
-    // tiles, so the per-tile epilogue never throttles the key stream)
-    static constexpr int NACC = NQ == 1 ? 4 : 2;
-    static constexpr int A_COL0 = NACC * ACC_COLS;                  // fp8: bf16 key tiles in TMEM
-    static constexpr int A_COLS = DI / 2;                            // 128 bf16 = 64 columns
+    static constexpr int ACC_COLS = SUB * N;
+    // accumulator ring: bf16 decode has 4 (two epilogue groups take alternate
+    // tiles, so the per-tile epilogue never throttles the key stream), narrow-key
+    // decode 2 units of two tiles each
+    static constexpr int NACC = NQ == 1 ? 4 / SUB : 2;
+    static constexpr int A_COL0 = NACC * ACC_COLS;                  // fp8: f16 key tiles in TMEM
+    static constexpr int A_COLS = SUB * DI / 2;                      // 128 f16 = 64 columns per tile
     // fp8: ring of widened key tiles in TMEM (as deep as the columns allow,
     // so that the widening warps can run ahead of the MMA)
     static constexpr int NA = FP8 ? (512 - NACC * ACC_COLS) / A_COLS < 4 ? (512 - NACC * ACC_COLS) / A_COLS : 4 : 2;
+    static_assert(KTU <= 256, "one TMA box per unit (at most 256 rows)");
     static constexpr int TMEM_NEED = NACC * ACC_COLS + (FP8 ? NA * A_COLS : 0);
     static_assert(!FP8 || NA >= 2, "fp8 needs at least two widened key tiles in TMEM");
     static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
@@ -105,8 +114,9 @@ __device__ __forceinline__ int last_visible(const Params& p, int t) {
     return pos < p.ctx - 1 ? pos : p.ctx - 1;     // may be < 0 (nothing visible)
 }
 
-// Deterministic schedule, walked identically by every warp role.
-template <int NQ>
+// Deterministic schedule, walked identically by every warp role (units of
+// KTU keys).
+template <int NQ, int KTU>
 struct Sched {
     // flat (NQ == 1)
     int64_t u, u_end;
@@ -116,7 +126,7 @@ struct Sched {
 
     __device__ void init(const Params& p) {
         if (NQ == 1) {
-            tpr = (p.ctx + KT - 1) / KT;
+            tpr = (p.ctx + KTU - 1) / KTU;
             const int64_t total = (int64_t)p.rows * tpr;
             u = total * blockIdx.x / gridDim.x;
             u_end = total * (blockIdx.x + 1) / gridDim.x;
@@ -133,7 +143,7 @@ struct Sched {
         if (NQ == 1) {
             while (u < u_end) {
                 const int t = (int)(u / tpr), j = (int)(u - (int64_t)t * tpr);
-                const int nt = last_visible(p, t) / KT + 1;          // 0 if nothing visible
+                const int nt = last_visible(p, t) / KTU + 1;         // 0 if nothing visible
                 if (last_visible(p, t) < 0 || j >= nt) {             // rest of this row is invisible
                     u = (int64_t)(t + 1) * tpr;
                     continue;
@@ -165,7 +175,7 @@ struct Sched {
                 int mp = -1;
                 for (int r = 0; r < NQ; ++r)
                     if (g * NQ + r < p.rows) mp = max(mp, last_visible(p, g * NQ + r));
-                ntiles = mp < 0 ? 0 : mp / KT + 1;
+                ntiles = mp < 0 ? 0 : mp / KTU + 1;
                 tile = 0;
             }
         }
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     pdl_wait();                     // inputs written by earlier kernels are visible from here on
     pdl_launch_dependents();
 
-    Sched<NQ> sch;
+    Sched<NQ, C::KTU> sch;
     Unit un;
 
     if (warp == 0) {
@@ -285,7 +295,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                 if (!mbar_wait(&kempty[st], ((i / C::STAGES) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
                 mbar_arrive_expect_tx(&kfull[st], C::KBYTES);
                 const int b = __ldg(p.row_batch + un.t0);
-                const int row = b * p.ctx + un.tile * KT;
+                const int row = b * p.ctx + un.tile * C::KTU;
                 uint8_t* kdst = kbuf + (size_t)st * C::KBYTES;
                 if (NQ == 1) {       // decode: every key is read once -> stream it past L2
                     tma_load_2d_hint(kdst, &tmap_k, 0, row, &kfull[st], pol_stream);
@@ -334,7 +344,10 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                     const uint32_t koff = (uint32_t)((kk >> 2) * (C::N * 128) + (kk & 3) * 32);
                     const uint64_t bdesc = desc_sw128(qaddr + koff, 1024);
                     if (FP8) {
-                        mma_ts(d, tmem + C::A_COL0 + ab * C::A_COLS + kk * 8, bdesc, idesc, kk > 0);
+#pragma unroll
+                        for (int sb = 0; sb < C::SUB; ++sb)          // the unit's 128-key tiles
+                            mma_ts(d + sb * C::N, tmem + C::A_COL0 + ab * C::A_COLS + sb * (DI / 2) + kk * 8, bdesc,
+                                   idesc, kk > 0);
                     } else {
                         const uint32_t aoff = (uint32_t)(st * C::KBYTES + (kk >> 2) * (KT * 128) + (kk & 3) * 32);
                         mma_ss(d, desc_sw128(kbase + aoff, 1024), bdesc, idesc, kk > 0);
@@ -350,7 +363,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
     } else if (FP8 && warp >= 4 && warp < 8) {
         // ------------------------- fp8 -> f16 key widening into TMEM ----
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;                  // key row of the tile = TMEM lane
+        const int r0 = quarter * 32 + lane;                 // key row of a 128-key tile = TMEM lane
         sch.init(p);
         int i = 0, qe = -1;
         while (sch.next(p, un)) {
@@ -376,7 +389,11 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
             if (!mbar_wait(&kfull[st], (i / C::STAGES) & 1, p.err, DEV_ERR_TIMEOUT_TMA, abort_flag)) break;
             if (!mbar_wait(&aempty[ab], ((i / C::NA) & 1) ^ 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + ab * C::A_COLS;
+#pragma unroll 1
+            for (int sb = 0; sb < C::SUB; ++sb) {
+            // tile sb of the unit: smem rows sb*128 + r, TMEM columns [64 sb, +64) of the slot
+            const int r = sb * KT + r0;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + C::A_COL0 + ab * C::A_COLS + sb * (DI / 2);
             if (KF == KF_FP4) {
                 // a 64-byte row of e2m1 pairs (64-byte swizzle: chunk c of row r
                 // sits at chunk c ^ ((r >> 1) & 3)); 16 bytes -> 32 dims -> 16 columns
@@ -415,6 +432,7 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
                 tmem_st16(taddr + half * 32 + 16, hi);
             }
             }
+            }
             tmem_st_wait();
             __syncwarp();
             tc_fence_before();
@@ -435,52 +453,87 @@ __global__ void __launch_bounds__(THREADS, 1) indexer_tc_kernel(const __grid_con
         while (sch.next(p, un)) {
             if (NQ == 1 && (i & 1) != eg) { ++i; continue; }
             const int acc = i % C::NACC;
-            const int key = un.tile * KT + quarter * 32 + lane;
-            // the key's row and (fp8) dequantisation scale are loaded before
-            // the wait for the accumulator, so their latency is hidden
+            // the keys' row and (fp8 / fp4) dequantisation scales are loaded
+            // before the wait for the accumulator, so their latency is hidden;
+            // thread (quarter, lane) owns key quarter*32 + lane of each 128-key tile
             const int b = __ldg(p.row_batch + un.t0);
             const bool b_ok = b >= 0 && b < p.batch;
-            float ks = 1.f;
-            if (FP8 && b_ok && key < p.ctx) ks = __ldg(p.k_scale + (int64_t)b * p.ctx + key);
+            const int key0 = un.tile * C::KTU + quarter * 32 + lane;     // key of tile sb: key0 + 128 sb
+            float ks[C::SUB];
+#pragma unroll
+            for (int sb = 0; sb < C::SUB; ++sb) {
+                ks[sb] = 1.f;
+                if (FP8 && b_ok && key0 + sb * KT < p.ctx) ks[sb] = __ldg(p.k_scale + (int64_t)b * p.ctx + key0 + sb * KT);
+            }
             if (!mbar_wait(&accfull[acc], (i / C::NACC) & 1, p.err, DEV_ERR_TIMEOUT_MMA, abort_flag)) break;
             tc_fence_after();
             const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * C::ACC_COLS;
             constexpr int QPW = NQ == 1 ? 1 : 2;           // query rows per epilogue warp
-            float score[QPW];
+            static_assert(C::SUB == 1 || QPW == 1, "two-tile units only with one query row per warp");
+            float score[QPW], score1 = 0.f;                 // score1: the unit's second tile
+#pragma unroll 1
+            for (int sb = 0; sb < C::SUB; ++sb) {           // one tile at a time (register budget)
 #pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
                 const int qi = NQ == 1 ? 0 : eg * 2 + qq;  // query within the group
-                float v0[32], v1[32];
-                tmem_ld32(tbase + qi * HI, v0);
-                tmem_ld32(tbase + qi * HI + 32, v1);
                 const int t = min(un.t0 + qi, p.rows - 1);
                 const float4* wr = (const float4*)(p.w + (int64_t)t * HI);
-                tmem_ld_wait();
                 // four independent partial sums (the weights are read as float4)
                 float s4[4] = {0.f, 0.f, 0.f, 0.f};
+                if (C::SUB == 1) {
+                    float v0[32], v1[32];
+                    tmem_ld32(tbase + qi * HI, v0);
+                    tmem_ld32(tbase + qi * HI + 32, v1);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int h4 = 0; h4 < 8; ++h4) {
-                    const float4 wa = __ldg(wr + h4), wb = __ldg(wr + 8 + h4);
-                    s4[0] = fmaf(wa.x, fmaxf(v0[4 * h4], 0.f), s4[0]);
-                    s4[1] = fmaf(wa.y, fmaxf(v0[4 * h4 + 1], 0.f), s4[1]);
-                    s4[2] = fmaf(wa.z, fmaxf(v0[4 * h4 + 2], 0.f), s4[2]);
-                    s4[3] = fmaf(wa.w, fmaxf(v0[4 * h4 + 3], 0.f), s4[3]);
-                    s4[0] = fmaf(wb.x, fmaxf(v1[4 * h4], 0.f), s4[0]);
-                    s4[1] = fmaf(wb.y, fmaxf(v1[4 * h4 + 1], 0.f), s4[1]);
-                    s4[2] = fmaf(wb.z, fmaxf(v1[4 * h4 + 2], 0.f), s4[2]);
-                    s4[3] = fmaf(wb.w, fmaxf(v1[4 * h4 + 3], 0.f), s4[3]);
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 wa = __ldg(wr + h4), wb = __ldg(wr + 8 + h4);
+                        s4[0] = fmaf(wa.x, fmaxf(v0[4 * h4], 0.f), s4[0]);
+                        s4[1] = fmaf(wa.y, fmaxf(v0[4 * h4 + 1], 0.f), s4[1]);
+                        s4[2] = fmaf(wa.z, fmaxf(v0[4 * h4 + 2], 0.f), s4[2]);
+                        s4[3] = fmaf(wa.w, fmaxf(v0[4 * h4 + 3], 0.f), s4[3]);
+                        s4[0] = fmaf(wb.x, fmaxf(v1[4 * h4], 0.f), s4[0]);
+                        s4[1] = fmaf(wb.y, fmaxf(v1[4 * h4 + 1], 0.f), s4[1]);
+                        s4[2] = fmaf(wb.z, fmaxf(v1[4 * h4 + 2], 0.f), s4[2]);
+                        s4[3] = fmaf(wb.w, fmaxf(v1[4 * h4 + 3], 0.f), s4[3]);
+                    }
+                } else {
+                    // two-tile units: the 64 head columns in two loads of 32
+                    // (register budget), the same four partial sums
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        float v[32];
+                        tmem_ld32(tbase + sb * C::N + qi * HI + hf * 32, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h4 = 0; h4 < 8; ++h4) {
+                            const float4 wa = __ldg(wr + hf * 8 + h4);
+                            s4[0] = fmaf(wa.x, fmaxf(v[4 * h4], 0.f), s4[0]);
+                            s4[1] = fmaf(wa.y, fmaxf(v[4 * h4 + 1], 0.f), s4[1]);
+                            s4[2] = fmaf(wa.z, fmaxf(v[4 * h4 + 2], 0.f), s4[2]);
+                            s4[3] = fmaf(wa.w, fmaxf(v[4 * h4 + 3], 0.f), s4[3]);
+                        }
+                    }
                 }
-                score[qq] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                const float sc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+                if (sb == 0) score[qq] = sc;
+                else score1 = sc;
+            }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
             if (!b_ok && lane == 0) record_error(p.err, DEV_ERR_BAD_INDEX);
 #pragma unroll
+            for (int sb = 0; sb < C::SUB; ++sb) {
+#pragma unroll
             for (int qq = 0; qq < QPW; ++qq) {
                 const int t = un.t0 + (NQ == 1 ? 0 : eg * 2 + qq);
+                const float sc = sb == 0 ? score[qq] : score1;
+                const int key = key0 + sb * KT;
                 if (b_ok && t < p.rows && key <= last_visible(p, t))
-                    p.logits[(int64_t)t * p.ld + key] = FP8 ? score[qq] * ks : score[qq];
+                    p.logits[(int64_t)t * p.ld + key] = FP8 ? sc * ks[sb] : sc;
+            }
             }
             ++i;
         }
@@ -503,9 +556,9 @@ cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Para
     using C = Cfg<NQ, KF>;
     CUtensorMap mk, mq;
     const uint64_t krows = (uint64_t)p.batch * p.ctx;
-    bool ok = KF == KF_FP4 ? make_map_swizzled(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI / 2, krows, 64, KT,
+    bool ok = KF == KF_FP4 ? make_map_swizzled(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI / 2, krows, 64, C::KTU,
                                                CU_TENSOR_MAP_SWIZZLE_64B)
-            : KF == KF_FP8 ? make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, KT)
+            : KF == KF_FP8 ? make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, DI, krows, 128, C::KTU)
                   : make_map_sw128(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, DI, krows, 64, KT);
     ok = ok && make_map_sw128(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DI, (uint64_t)p.rows * HI, 64, NQ * HI);
     if (!ok) return cudaErrorInvalidValue;
@@ -513,7 +566,7 @@ cudaError_t launch_cfg(const Launch& L, const void* q, const void* k, const Para
                                          (int)C::SMEM);
     if (e != cudaSuccess) return e;
     int64_t units;
-    if (NQ == 1) units = (int64_t)p.rows * ((p.ctx + KT - 1) / KT);
+    if (NQ == 1) units = (int64_t)p.rows * ((p.ctx + C::KTU - 1) / C::KTU);
     else units = (p.rows + NQ - 1) / NQ;
     const int grid = (int)(units < L.num_sms ? units : L.num_sms);
     cudaLaunchConfig_t cfg = {};

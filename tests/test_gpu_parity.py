@@ -192,6 +192,22 @@ def test_sparse_mla_all_slots_unused(cuda_device):
     assert np.abs(o[1] - row[None, :]).max() <= 1e-2
 
 
+@pytest.mark.parametrize("kd", ["fp8", "fp4", "bf16"])
+def test_indexer_partial_visibility(cuda_device, kd):
+    # decode rows that see only a prefix of their sequence's keys: the narrow-key
+    # path takes keys in units of 256, so prefixes ending inside, at and just past
+    # a unit are all present; rows share sequences
+    wl = workloads.DECODE_128K_FP8_PAGED.with_(batch=3, rows=8, ctx=777, idx_key_dtype=kd)
+    inp = workloads.generate(wl, parts=("indexer",))
+    inp["row_pos"] = torch.tensor([776, 0, 127, 255, 256, 511, 600, 1], dtype=torch.int32)
+    dv = _cuda(inp, cuda_device)
+    got = dsa.indexer_logits(dv["q_idx"], dv["w"], dv["k_idx"], dv["row_batch"], dv["row_pos"],
+                             k_scale=dv.get("k_scale")).cpu().numpy()
+    ref = oracle.index_scores(inp["q_idx"], inp["w"], inp["k_idx"], inp["row_batch"], inp["row_pos"],
+                              k_scale=inp.get("k_scale"))
+    _logits_close(got, ref, inp["row_pos"].numpy())
+
+
 # ----------------------------------------------------------- whole chain ----
 
 @pytest.mark.parametrize("wl", [
