@@ -4,13 +4,15 @@
 // sum):
 //   logits[t, s] = sum_{j<64} w[t, j] * ReLU(q[t, j, :] . k[b, s, :])
 //
-// Per work unit (a group of NQ query rows x a tile of 128 cached keys):
+// Per work unit (a group of NQ query rows x a tile of 128 cached keys; two
+// such tiles, 256 keys, for fp8 / fp4 keys in decode):
 //   D[128 keys, NQ*64 (query,head)] = K_tile[128 x 128] . Q[NQ*64 x 128]^T
-// one tcgen05.mma chain (M=128, N=NQ*64, K=128) with the fp32 accumulator in
-// TMEM, then an epilogue in which each thread owns one key (one TMEM lane)
-// and reduces its NQ*64 columns to NQ scores: ReLU, times w, sum over heads
-// (times the key's dequantisation scale for fp8 keys).  Scores are written
-// coalesced (32 consecutive keys per warp store).
+// one tcgen05.mma chain per tile (M=128, N=NQ*64, K=128) with the fp32
+// accumulator in TMEM, then an epilogue in which each thread owns one key of
+// each tile (one TMEM lane) and reduces its NQ*64 columns to NQ scores: ReLU,
+// times w, sum over heads (times the key's dequantisation scale for fp8 /
+// fp4 keys).  Scores are written coalesced (32 consecutive keys per warp
+// store).
 //
 // Warp roles (512 threads, one CTA per SM, persistent):
 //   warp 0      TMA producer: key tiles (ring of STAGES), query tiles (x2)

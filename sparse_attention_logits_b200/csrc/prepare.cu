@@ -316,8 +316,8 @@ __global__ void __launch_bounds__(PTHREADS, 2) indexer_prepare_kernel(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // Only the query tiles' latent operand, 1/RMS and the arrival counters
-    // come from the norm kernel; the weights, h, positions and rotary tables
+    // Only the query tiles' latent operand and 1/RMS come from the norm
+    // kernel; the weights, h, positions and rotary tables
     // are inputs that the kernels before it had finished writing when it
     // started (it waits for them before letting this grid start), so they
     // are read before pdl_wait().
