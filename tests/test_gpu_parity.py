@@ -98,6 +98,21 @@ def test_topk_rows_not_16_byte_aligned(cuda_device):
         assert np.array_equal(got[r][got[r] >= 0], np.sort(ref[r][ref[r] >= 0])), f"row {r}"
 
 
+@pytest.mark.parametrize("rows,L,ld_pad,k,seed", [(40, 131079, 0, 2048, 21), (80, 50000, 0, 1024, 22),
+                                                    (40, 90001, 3, 2048, 23)])
+def test_topk_clusters_in_several_waves(cuda_device, rows, L, ld_pad, k, seed):
+    # more rows' clusters (2 to 4 CTAs per row) than a B200 holds at once, so the
+    # launch runs in waves; ld = L + 3 puts most rows off a 16-byte boundary
+    # (the scalar load path)
+    x = workloads.synthetic_scores(rows, L + ld_pad, seed=seed)
+    pos = torch.tensor([L - 1 - (r * 997) % (L // 2) for r in range(rows)], dtype=torch.int32)
+    got = dsa.topk(x.to(cuda_device), pos.to(cuda_device), k, ctx_len=L).cpu().numpy()
+    check_sorted_unique(got, pos.numpy() + 1)
+    ref = oracle.topk(x[:, :L].contiguous(), pos, k)
+    for r in range(rows):
+        assert np.array_equal(got[r][got[r] >= 0], np.sort(ref[r][ref[r] >= 0])), f"row {r}"
+
+
 def test_topk_edge_cases(cuda_device):
     L = 4100
     rows = []
